@@ -1,0 +1,366 @@
+"""Benchmark of the key-gated GLA forward on B200: tokens/s and % of roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload batched] [--schedule auto|fused|three_phase]
+
+A step is one full GLA forward (every phase of the chunkwise operator) over
+one batch of the workload; steps alternate the workload's scan directions.
+Inputs are seeded synthetic tensors resident in HBM before the timed region;
+they are larger than L2, so no flush is needed between steps.  Timing uses
+CUDA events on the launching stream, W untimed warm-up steps, then exactly K
+timed steps bracketed by a barrier and a device synchronize; with N ranks
+(torchrun, one process per GPU) every rank runs its own batch (weak scaling,
+no collective on the data path) and the max time over ranks is reported.
+Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference that exists:
+the pages publish no code) on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from recurrent_vision_backbone_key_b200 import gtr_gla  # noqa: E402
+from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs  # noqa: E402
+from recurrent_vision_backbone_key_b200 import dist as rdist  # noqa: E402
+
+METRIC = "GLA forward tokens/s and % of roofline (HBM GB/s or TC util) at 1 B200"
+DIR_NAMES = ["L2R", "R2L", "T2B", "B2T"]
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+def describe(w):
+    dirs = "+".join(DIR_NAMES[d] for d in w.directions)
+    return (f"{w.name}: B{w.B} {w.grid_h}x{w.grid_w} grid ({w.N} tokens), {w.heads} heads, "
+            f"d_k={w.d_k} d_v={w.d_v}, chunk {w.chunk}, {w.gate} gates, directions {dirs} "
+            f"alternating per step")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nvml = None
+
+    def _sample(self):
+        try:
+            self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+            self.reasons |= int(self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            self._sample()
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "samples": len(self.samples), "reasons": names}
+
+
+def oracle_rate(w, q, k, v, g, budget_s, nthreads, directions):
+    """Times the fp64 oracle on (b, h) sequences of the workload until about
+    budget_s seconds of CPU work; returns (tokens/s, sample description)."""
+    from oracle import oracle
+    oracle.build()
+    rng = np.random.default_rng(0)
+    picks = [(int(b), int(h)) for b, h in zip(rng.integers(w.B, size=4096), rng.integers(w.heads, size=4096))]
+    done_th, elapsed, n_seq, i = 0, 0.0, 0, 0
+    batch = max(1, nthreads)
+    while elapsed < budget_s and n_seq < len(picks):
+        sel = picks[n_seq:n_seq + batch]
+        # gather the selected sequences as one [n, N, 1, d] problem
+        take = lambda x: torch.stack([x[b, :, h:h + 1, :] for b, h in sel]).cpu()
+        qs, ks, vs, gs = take(q), take(k), take(v), take(g)
+        d = directions[i % len(directions)]
+        t0 = time.perf_counter()
+        oracle.gla_serial(qs, ks, vs, gs, w.grid_h, w.grid_w, d, nthreads=nthreads)
+        elapsed += time.perf_counter() - t0
+        done_th += len(sel) * w.N
+        n_seq += len(sel)
+        i += 1
+        batch = max(batch, int(batch * min(4.0, 0.5 * budget_s / max(elapsed, 1e-3))))
+        batch = min(batch, 64 * max(1, nthreads))
+    tokens_per_s = done_th / elapsed  # one head of one token per unit; heads run in parallel
+    tokens_per_s /= w.heads  # a token is complete once all its heads are
+    sample = (f"{n_seq} (batch, head) sequences of {w.N} tokens drawn from the workload, "
+              f"serial fp64 recurrence, {elapsed:.1f} s")
+    return tokens_per_s, sample
+
+
+def run_reference(args, w):
+    rank, world = rdist.rank_world()
+    if rank != 0:
+        return 0
+    q, k, v, g = make_workload_inputs(w, seed=0, device="cpu")
+    nthreads = os.cpu_count() or 1
+    from oracle import oracle
+    oracle.build()
+    rng = np.random.default_rng(1)
+    per_step = max(1, nthreads)
+    def step(i):
+        sel = [(int(rng.integers(w.B)), int(rng.integers(w.heads))) for _ in range(per_step)]
+        take = lambda x: torch.stack([x[b, :, h:h + 1, :] for b, h in sel])
+        oracle.gla_serial(take(q), take(k), take(v), take(g), w.grid_h, w.grid_w,
+                          w.directions[i % len(w.directions)], nthreads=nthreads)
+        return len(sel) * w.N
+    for i in range(args.warmup):
+        step(i)
+    th = 0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        th += step(i)
+    dt = time.perf_counter() - t0
+    value = th / w.heads / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": describe(w), "B": w.B, "grid": [w.grid_h, w.grid_w],
+                   "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk,
+                   "step": f"fp64 CPU oracle on {per_step} sampled (batch, head) sequences"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{per_step} (batch, head) sequences of {w.N} tokens per step"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_steps(fn, steps, stream):
+    """Runs fn(i) for i in range(steps) between two events on `stream`; ms."""
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(steps):
+        fn(i)
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS))
+    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    rank, world = rdist.init_from_env(backend="nccl")
+    dev = rdist.local_device()
+    torch.cuda.set_device(dev)
+    lib = gtr_gla.load()
+    stream = torch.cuda.current_stream()
+    sched = {"auto": 0, "fused": 1, "three_phase": 2}[args.schedule]
+
+    q, k, v, g = make_workload_inputs(w, seed=rank, device=f"cuda:{dev}")
+    out = torch.empty((w.B, w.N, w.heads, w.d_v), dtype=torch.float16, device=f"cuda:{dev}")
+    dirs = list(w.directions)
+
+    def step(i):
+        gtr_gla.check(gtr_gla.gtr_gla_forward_ex(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w,
+                                                 w.d_k, w.d_v, dirs[i % len(dirs)], w.chunk, sched,
+                                                 out, stream))
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    rdist.barrier()
+    l0 = gtr_gla.gtr_gla_launch_count()
+    with ClockSampler(dev) as clocks:
+        torch.cuda.synchronize()
+        ms = time_steps(step, args.steps, stream)
+        torch.cuda.synchronize()
+    launches = gtr_gla.gtr_gla_launch_count() - l0
+    rdist.barrier()
+    assert gtr_gla.gtr_gla_get_last_device_status(stream) == 0
+    ms_max = rdist.max_over_ranks(ms)
+    tokens_all = float(w.B * w.N * args.steps * world)
+    value = tokens_all / (ms_max * 1e-3)
+
+    # Roofline of the dominant kernel: for the single-kernel schedule a step is
+    # one launch; for the three-phase schedule time its phases one by one.
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    alg_bytes = w.algorithmic_bytes()
+    per_launch_ms = ms / args.steps
+    dominant = "forward step"
+    phase_ms = None
+    if sched == 2 or (sched == 0 and launches > args.steps):
+        phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
+        dominant = max(phase_ms, key=phase_ms.get)
+        per_launch_ms = phase_ms[dominant]
+        alg_bytes = phase_alg_bytes(w)[dominant]
+    achieved = alg_bytes / (per_launch_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved / hbm_peak, "traffic": None,
+                "kernel": dominant, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+                "algorithmic_bytes_per_launch": alg_bytes,
+                "tensor_flops_per_step": w.algorithmic_flops(),
+                "tensor_frac_of_bf16_peak": w.algorithmic_flops() / (ms / args.steps * 1e-3) / 1e12 / tc_peak}
+    if phase_ms:
+        roofline["phase_ms"] = phase_ms
+
+    # End to end through the host-buffer entry point: pinned host inputs in,
+    # host output back, every step.
+    e2e = None
+    if args.e2e_steps > 0:
+        qh, kh, vh, gh = (x.cpu().pin_memory() for x in (q, k, v, g))
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        def e2e_step(i):
+            gtr_gla.check(gtr_gla.gtr_gla_forward_host(qh, kh, vh, gh, w.B, w.heads, w.grid_h,
+                                                       w.grid_w, w.d_k, w.d_v, dirs[i % len(dirs)],
+                                                       w.chunk, oh, stream))
+        e2e_step(0)
+        torch.cuda.synchronize()
+        rdist.barrier()
+        t0 = time.perf_counter()
+        for i in range(args.e2e_steps):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        e2e_s = rdist.max_over_ranks(time.perf_counter() - t0)
+        h2d = sum(x.numel() * x.element_size() for x in (q, k, v, g))
+        d2h = out.numel() * out.element_size()
+        e2e = {"value": float(w.B * w.N * args.e2e_steps * world / e2e_s), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": args.e2e_steps, "timer": "host wall clock around synchronous calls"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nthreads = os.cpu_count() or 1
+        val, sample = oracle_rate(w, q, k, v, g, args.cpu_budget, nthreads, dirs)
+        cpu = {"value": val, "unit": "tokens/s", "cores": nthreads, "kind": "oracle",
+               "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic",
+            "config": {"workload": describe(w), "B": w.B, "grid": [w.grid_h, w.grid_w],
+                       "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk,
+                       "schedule": args.schedule, "parallelism": f"dp{world} (independent batches)",
+                       "l2": f"inputs larger than L2 ({alg_bytes_total(w) / 1e6:.0f} MB per step), no flush"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    rdist.finalize()
+    return 0
+
+
+def alg_bytes_total(w):
+    return w.algorithmic_bytes()
+
+
+def phase_alg_bytes(w):
+    th = w.token_heads
+    nseq = w.B * w.heads
+    nc = (w.N + w.chunk - 1) // w.chunk
+    state = nseq * nc * w.d_k * w.d_v * 4
+    return {
+        "chunk_summary": th * (6 * w.d_k + 2 * w.d_v) + state + nseq * nc * w.d_k * 4,
+        "boundary_scan": 2 * state + nseq * nc * w.d_k * 4,
+        "chunk_output": w.algorithmic_bytes() + state,
+    }
+
+
+def time_phases(w, q, k, v, g, out, stream, reps):
+    nseq = w.B * w.heads
+    nc = (w.N + w.chunk - 1) // w.chunk
+    dS = torch.empty((nseq, nc, w.d_k, w.d_v), dtype=torch.float32, device=q.device)
+    gam = torch.empty((nseq, nc, w.d_k), dtype=torch.float32, device=q.device)
+    Se = torch.empty_like(dS)
+    d = w.directions[0]
+    calls = {
+        "chunk_summary": lambda i: gtr_gla.check(gtr_gla.gtr_gla_chunk_summary(
+            k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d, w.chunk, dS, gam, stream)),
+        "boundary_scan": lambda i: gtr_gla.check(gtr_gla.gtr_gla_boundary_scan(
+            dS, gam, w.B, w.heads, nc, w.d_k, w.d_v, Se, stream)),
+        "chunk_output": lambda i: gtr_gla.check(gtr_gla.gtr_gla_chunk_output(
+            q, k, v, g, Se, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d, w.chunk, out,
+            stream)),
+    }
+    res = {}
+    for name, fn in calls.items():
+        for i in range(3):
+            fn(i)
+        res[name] = time_steps(fn, reps, stream) / reps
+    del dS, gam, Se
+    return res
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * gtr_gla.h -- C ABI of the B200 (sm_100a) key-gated GLA token mixer.
+ *
+ * Operation (the GTR token mixer; sources by page and section):
+ *   For each batch b and head h, over the N = grid_h*grid_w patch tokens
+ *   visited in one scan order, with S_0 = 0:
+ *       S_t = diag(exp(g_t)) S_{t-1} + k_t^T v_t          (d_k x d_v state)
+ *       o_t = (q_t / sqrt(d_k)) S_t
+ *   and o_t written back at the token's own spatial position.
+ *   - key-only gated linear attention, value-side decay fixed at one; one
+ *     directional scan per block, spatial order restored afterwards:
+ *     ai.info summary of "GTR: Gated Token Recurrence for Efficient Dense
+ *     Prediction", section "Methodology in Plain English";
+ *   - scan orders left->right, right->left, top->bottom, bottom->top cycled
+ *     across the 12 blocks: GTR project page, section "How GTR Works";
+ *   - the inference operator: per-chunk summaries computed in parallel over
+ *     the chunk x head grid, a light coalesced scan of the chunk boundary
+ *     states, and an output kernel that fuses the intra-chunk score-value
+ *     product with the boundary-state readout; zero initial state; fp16:
+ *     GTR project page, section "A Kernel That Makes Recurrence Fast", and
+ *     the ai.info summary, "Methodology in Plain English".
+ *
+ * Conventions shared by every entry point:
+ *   - Buffers marked (device) are CUDA device pointers of the current device,
+ *     buffers marked (host) are host pointers.  The caller owns every buffer.
+ *   - fp16 buffers hold IEEE binary16 values (CUDA __half); fp32 buffers
+ *     hold IEEE binary32 values.
+ *   - Token layout: q, k and g are [B][N][heads][d_k], v and out are
+ *     [B][N][heads][d_v], contiguous, N = grid_h*grid_w tokens in row-major
+ *     spatial order (row r, column c -> token r*grid_w + c), both in and out.
+ *     The scan order is applied inside the kernels' loads and stores; no
+ *     permuted copy is ever made.
+ *   - Scan orders (gtr_dir_t): L2R visits t -> t; R2L visits t -> N-1-t;
+ *     T2B visits column-major, t -> (t mod grid_h)*grid_w + t div grid_h;
+ *     B2T visits the reverse of T2B.
+ *   - Supported sizes: d_k, d_v in {16, 32, 64, 128}; chunk in {16, 32, 64};
+ *     any grid_h, grid_w >= 1 (a ragged last chunk is masked), any B,
+ *     heads >= 1.  B == 0 or N == 0 is an empty problem: GTR_OK, nothing
+ *     is launched.
+ *   - Every device pointer must be 16-byte aligned (GTR_ERR_MISALIGNED).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device entry points are asynchronous: they enqueue work on
+ *     `stream` and return without synchronising.  On any error status
+ *     nothing is enqueued, except GTR_ERR_CUDA from a failed launch.
+ *   - Errors never cross the ABI as exceptions.  gtr_gla_last_error()
+ *     returns a short text for the calling thread's last failure.
+ *   - Thread safety: calls on distinct streams may run concurrently.  Calls
+ *     that use the library's internal workspace on the same stream are
+ *     ordered by that stream.
+ *   - log-gates g are expected to be <= 0 (the accuracy bound holds for
+ *     g <= 0); other values are accepted and computed, not clamped.
+ */
+#ifndef GTR_GLA_H
+#define GTR_GLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GTR_DIR_L2R = 0,
+    GTR_DIR_R2L = 1,
+    GTR_DIR_T2B = 2,
+    GTR_DIR_B2T = 3
+} gtr_dir_t;
+
+typedef enum {
+    GTR_OK = 0,
+    GTR_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad enum */
+    GTR_ERR_UNSUPPORTED_SHAPE = 2, /* d_k, d_v or chunk outside the supported set */
+    GTR_ERR_MISALIGNED = 3,        /* a device pointer not 16-byte aligned */
+    GTR_ERR_ALIAS = 4,             /* an output overlaps an input */
+    GTR_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    GTR_ERR_TIMEOUT = 6,           /* a bounded device-side wait gave up */
+    GTR_ERR_OOM = 7                /* the internal workspace could not grow */
+} gtr_status_t;
+
+typedef enum {
+    GTR_SCHED_AUTO = 0,        /* library choice (currently the fused kernel when built) */
+    GTR_SCHED_FUSED = 1,       /* one kernel: summaries, chained boundary states, outputs */
+    GTR_SCHED_THREE_PHASE = 2  /* chunk_summary -> boundary_scan -> chunk_output */
+} gtr_schedule_t;
+
+/* The GLA forward over all B*heads sequences (see the operation above).
+ *   q, k (device, fp16) [B][N][heads][d_k]; v (device, fp16) [B][N][heads][d_v];
+ *   g (device, fp32) [B][N][heads][d_k] log-gates; out (device, fp16)
+ *   [B][N][heads][d_v], written in full (every token, every head);
+ *   direction: gtr_dir_t; chunk: tokens per chunk of the chunkwise schedule.
+ * out must not overlap q, k, v or g (GTR_ERR_ALIAS).  Uses an internal
+ * per-device, per-stream workspace that grows on demand (GTR_ERR_OOM if it
+ * cannot); a call that has to grow it synchronises the device, so make the
+ * first call of the largest size outside any stream capture. */
+gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const float *g,
+                             int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                             int direction, int chunk, void *out, void *stream);
+
+/* gtr_gla_forward with an explicit schedule (gtr_schedule_t).  Both
+ * schedules compute the same recurrence; results agree to rounding. */
+gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, const float *g,
+                                int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                int direction, int chunk, int schedule, void *out, void *stream);
+
+/* End-to-end call on HOST buffers: copies q, k, v, g (host) to the device,
+ * runs gtr_gla_forward on `stream`, copies the result into out (host) and
+ * synchronises `stream` before returning.  Layouts as gtr_gla_forward.
+ * Device staging buffers come from the internal workspace.  Page-locked host
+ * buffers give the fastest copies; pageable ones work too. */
+gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, const float *g,
+                                  int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                  int direction, int chunk, void *out, void *stream);
+
+/* Phase 1, chunk summaries (GTR project page, "A Kernel That Makes
+ * Recurrence Fast": per-chunk summaries in parallel over the chunk x head
+ * grid).  With nc = ceil(N/chunk) and b_s the inclusive prefix sum of g
+ * inside chunk c (scan order), for every (b, h, c):
+ *   gamma[b][h][c][i]   = exp(b_last[i])
+ *   dS[b][h][c][i][j]   = sum_s exp(b_last[i] - b_s[i]) k_s[i] v_s[j]
+ * k (device, fp16), v (device, fp16), g (device, fp32) as in gtr_gla_forward;
+ * dS (device, fp32) [B][heads][nc][d_k][d_v]; gamma (device, fp32)
+ * [B][heads][nc][d_k].  Outputs must not overlap inputs. */
+gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g,
+                                   int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                   int direction, int chunk, float *dS, float *gamma,
+                                   void *stream);
+
+/* Phase 2, boundary-state scan (same section: only the boundary states are
+ * propagated sequentially).  For every (b, h):
+ *   S_enter[0] = 0,  S_enter[c+1][i][j] = gamma[c][i] * S_enter[c][i][j] + dS[c][i][j]
+ * dS, gamma (device, fp32) as written by gtr_gla_chunk_summary with
+ * n_chunks chunks; S_enter (device, fp32) [B][heads][n_chunks][d_k][d_v].
+ * S_enter may be the same buffer as dS (in place); any other overlap with
+ * the inputs is GTR_ERR_ALIAS. */
+gtr_status_t gtr_gla_boundary_scan(const float *dS, const float *gamma, int B, int heads,
+                                   int n_chunks, int d_k, int d_v, float *S_enter, void *stream);
+
+/* Phase 3, chunk outputs (same section: the output kernel fuses the
+ * within-chunk score-value product with the boundary-state readout).  For
+ * token t of chunk c:
+ *   o_t = sum_i q~_t[i] exp(b_t[i]) S_enter[c][i][:]
+ *       + sum_{s <= t in chunk} (sum_i q~_t[i] exp(b_t[i] - b_s[i]) k_s[i]) v_s
+ * with q~ = q / sqrt(d_k).  q, k, v, g, out as gtr_gla_forward; S_enter
+ * (device, fp32) as written by gtr_gla_boundary_scan. */
+gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, const float *g,
+                                  const float *S_enter, int B, int heads, int grid_h, int grid_w,
+                                  int d_k, int d_v, int direction, int chunk, void *out,
+                                  void *stream);
+
+/* Bytes of internal device workspace one gtr_gla_forward_ex call of this
+ * size and schedule uses (informational; 0 for invalid arguments). */
+size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                               int chunk, int schedule);
+
+/* Synchronises `stream`, then returns and clears the device-side status
+ * word of the current device: GTR_OK, or GTR_ERR_TIMEOUT if a bounded wait
+ * inside a kernel gave up since the last query. */
+gtr_status_t gtr_gla_get_last_device_status(void *stream);
+
+/* Frees every internal workspace of every device (synchronises each device
+ * that has one).  Later calls allocate again on demand. */
+gtr_status_t gtr_gla_release_workspace(void);
+
+/* Static text for a status code. */
+const char *gtr_gla_status_string(gtr_status_t status);
+
+/* Text describing the calling thread's most recent failed call ("" if none). */
+const char *gtr_gla_last_error(void);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t gtr_gla_launch_count(void);
+
+/* ABI version: major*10000 + minor*100 + patch. */
+int gtr_gla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTR_GLA_H */

@@ -1,0 +1,53 @@
+// gla_common.cuh -- pieces shared by the CUDA kernels of the GLA mixer.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gtr {
+
+// Problem geometry shared by every kernel.  Token layout [B][N][heads][d],
+// N = H*W tokens in row-major spatial order.
+struct Geom {
+    int B, heads, H, W;
+    int dk, dv;
+    int dir;     // 0 L->R, 1 R->L, 2 T->B, 3 B->T
+    int chunk;   // tokens per chunk
+    int N;       // H*W
+    int nc;      // ceil(N / chunk)
+};
+
+// G0, the scan-order index map: scan position t -> row-major token index.
+// Left->right is row-major order, right->left its reverse, top->bottom is
+// column-major order (t = col*H + row) and bottom->top its reverse (ai.info
+// summary of GTR, "Methodology in Plain English"; GTR project page, "How GTR
+// Works").  Folded into every load and store: no permuted copy exists.
+__device__ __forceinline__ int scan_pos(int dir, int t, int H, int W, int N) {
+    if (dir == 1) return N - 1 - t;
+    if (dir >= 2) {
+        int u = (dir == 3) ? (N - 1 - t) : t;
+        int col = u / H;
+        int row = u - col * H;
+        return row * W + col;
+    }
+    return t;
+}
+
+// Element offset of (b, token p, head h) in a [B][N][heads][d] tensor.
+__device__ __forceinline__ int64_t tok_offset(const Geom &g, int b, int p, int h, int d) {
+    return (((int64_t)b * g.N + p) * g.heads + h) * (int64_t)d;
+}
+
+}  // namespace gtr
+
+// Host-side launchers implemented in the .cu files (internal, C++ linkage).
+namespace gtr {
+cudaError_t launch_summary_v0(const __half *k, const __half *v, const float *g, const Geom &geo,
+                              float *dS, float *gamma, cudaStream_t st);
+cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                           float *S_enter, cudaStream_t st);
+cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, const float *g,
+                             const float *S_enter, const Geom &geo, __half *out, cudaStream_t st);
+void count_launch(int n = 1);
+}  // namespace gtr

@@ -1,0 +1,217 @@
+// gla_phases_simt.cu -- the three-phase chunkwise schedule on CUDA cores.
+//
+// GTR project page, "A Kernel That Makes Recurrence Fast": per-chunk
+// summaries in parallel over the chunk x head grid, a light coalesced scan
+// of the boundary states, then an output kernel fusing the within-chunk
+// score-value product with the boundary-state readout.  This file is the
+// plain-FP32 CUDA-core version of those three phases: every decay factor is
+// exp() of a difference of in-chunk prefix sums, so it is safe for any gate
+// values.  It is the straightforward schedule the tensor-core kernels are
+// checked and timed against.
+#include "gla_common.cuh"
+
+namespace gtr {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// Loads one chunk of a [B][N][heads][d] fp16 tensor into fp32 shared memory
+// rows of stride `ld`, visiting tokens in scan order; rows past N are zero.
+__device__ void load_rows_h(const __half *src, const Geom &g, int b, int h, int t0, int len,
+                            int d, float *dst, int ld) {
+    for (int idx = threadIdx.x; idx < g.chunk * d; idx += blockDim.x) {
+        int t = idx / d, i = idx - t * d;
+        float x = 0.f;
+        if (t < len) {
+            int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
+            x = __half2float(src[tok_offset(g, b, p, h, d) + i]);
+        }
+        dst[t * ld + i] = x;
+    }
+}
+
+__device__ void load_rows_f(const float *src, const Geom &g, int b, int h, int t0, int len, int d,
+                            float *dst, int ld) {
+    for (int idx = threadIdx.x; idx < g.chunk * d; idx += blockDim.x) {
+        int t = idx / d, i = idx - t * d;
+        float x = 0.f;
+        if (t < len) {
+            int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
+            x = src[tok_offset(g, b, p, h, d) + i];
+        }
+        dst[t * ld + i] = x;
+    }
+}
+
+// In-place inclusive prefix sum over the chunk's tokens, one thread per key
+// dimension.
+__device__ void prefix_rows(float *bs, int ld, int len, int dk) {
+    for (int i = threadIdx.x; i < dk; i += blockDim.x) {
+        float acc = 0.f;
+        for (int t = 0; t < len; ++t) {
+            acc += bs[t * ld + i];
+            bs[t * ld + i] = acc;
+        }
+    }
+}
+
+// Phase 1: gamma_c = exp(b_last), dS_c = sum_s exp(b_last - b_s) k_s^T v_s.
+__global__ void __launch_bounds__(kThreads) summary_simt_kernel(
+    const __half *__restrict__ k, const __half *__restrict__ v, const float *__restrict__ gl,
+    Geom g, float *__restrict__ dS, float *__restrict__ gamma) {
+    extern __shared__ float sm[];
+    const int c = (int)(blockIdx.x % (unsigned)g.nc);
+    const int seq_i = (int)(blockIdx.x / (unsigned)g.nc);
+    const int h = seq_i % g.heads, b = seq_i / g.heads;
+    const int C = g.chunk, dk = g.dk, dv = g.dv, ldk = dk + 1;
+    float *kw = sm;               // [C][dk+1]
+    float *bs = kw + C * ldk;     // [C][dk+1]
+    float *vv = bs + C * ldk;     // [C][dv]
+    const int t0 = c * C;
+    const int len = min(C, g.N - t0);
+    load_rows_h(k, g, b, h, t0, len, dk, kw, ldk);
+    load_rows_f(gl, g, b, h, t0, len, dk, bs, ldk);
+    load_rows_h(v, g, b, h, t0, len, dv, vv, dv);
+    __syncthreads();
+    prefix_rows(bs, ldk, len, dk);
+    __syncthreads();
+    const int64_t seq = (int64_t)b * g.heads + h;
+    for (int idx = threadIdx.x; idx < len * dk; idx += blockDim.x) {
+        int t = idx / dk, i = idx - t * dk;
+        kw[t * ldk + i] *= expf(bs[(len - 1) * ldk + i] - bs[t * ldk + i]);
+    }
+    for (int i = threadIdx.x; i < dk; i += blockDim.x)
+        gamma[(seq * g.nc + c) * dk + i] = expf(bs[(len - 1) * ldk + i]);
+    __syncthreads();
+    float *out = dS + (seq * g.nc + c) * (int64_t)dk * dv;
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) {
+        int i = e / dv, j = e - i * dv;
+        float acc = 0.f;
+        for (int t = 0; t < len; ++t) acc = fmaf(kw[t * ldk + i], vv[t * dv + j], acc);
+        out[e] = acc;
+    }
+}
+
+// Phase 2: one thread per state element, serial over chunks; consecutive
+// threads own consecutive elements, so every step is one coalesced sweep.
+// In place is allowed: element e of chunk c is read before it is written.
+__global__ void __launch_bounds__(kThreads) scan_simt_kernel(
+    const float *dS, const float *__restrict__ gamma, int nc, int dk, int dv, float *S_enter) {
+    const int per_seq = (dk * dv + blockDim.x - 1) / blockDim.x;
+    const int64_t seq = blockIdx.x / per_seq;
+    const int e = (blockIdx.x % per_seq) * blockDim.x + threadIdx.x;
+    if (e >= dk * dv) return;
+    const int i = e / dv;
+    const int64_t stride = (int64_t)dk * dv;
+    const float *src = dS + seq * nc * stride + e;
+    const float *gm = gamma + seq * nc * dk + i;
+    float *dst = S_enter + seq * nc * stride + e;
+    float S = 0.f;
+    for (int c = 0; c < nc; ++c) {
+        float x = src[c * stride];
+        float a = gm[(int64_t)c * dk];
+        dst[c * stride] = S;
+        S = fmaf(a, S, x);
+    }
+}
+
+// Phase 3: intra-chunk scores A[t][s] = sum_i q~_t[i] k_s[i] exp(b_t[i]-b_s[i])
+// for s <= t, then o_t = (q~_t * exp(b_t)) S_enter + sum_s A[t][s] v_s.
+__global__ void __launch_bounds__(kThreads) output_simt_kernel(
+    const __half *__restrict__ q, const __half *__restrict__ k, const __half *__restrict__ v,
+    const float *__restrict__ gl, const float *__restrict__ S_enter, Geom g,
+    __half *__restrict__ out) {
+    extern __shared__ float sm[];
+    const int c = (int)(blockIdx.x % (unsigned)g.nc);
+    const int seq_i = (int)(blockIdx.x / (unsigned)g.nc);
+    const int h = seq_i % g.heads, b = seq_i / g.heads;
+    const int C = g.chunk, dk = g.dk, dv = g.dv, ldk = dk + 1;
+    float *qs = sm;               // [C][dk+1]
+    float *ks = qs + C * ldk;     // [C][dk+1]
+    float *bs = ks + C * ldk;     // [C][dk+1]
+    float *vv = bs + C * ldk;     // [C][dv]
+    float *A = vv + C * dv;       // [C][C]
+    float *S = A + C * C;         // [dk][dv]
+    const int t0 = c * C;
+    const int len = min(C, g.N - t0);
+    const float scale = rsqrtf((float)dk);
+    load_rows_h(q, g, b, h, t0, len, dk, qs, ldk);
+    load_rows_h(k, g, b, h, t0, len, dk, ks, ldk);
+    load_rows_f(gl, g, b, h, t0, len, dk, bs, ldk);
+    load_rows_h(v, g, b, h, t0, len, dv, vv, dv);
+    const int64_t seq = (int64_t)b * g.heads + h;
+    const float *Sg = S_enter + (seq * g.nc + c) * (int64_t)dk * dv;
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[e] = Sg[e];
+    __syncthreads();
+    prefix_rows(bs, ldk, len, dk);
+    for (int idx = threadIdx.x; idx < C * dk; idx += blockDim.x) {
+        int t = idx / dk, i = idx - t * dk;
+        qs[t * ldk + i] *= scale;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < C * C; idx += blockDim.x) {
+        int t = idx / C, s = idx - t * C;
+        float a = 0.f;
+        if (s <= t && t < len) {
+            for (int i = 0; i < dk; ++i)
+                a = fmaf(qs[t * ldk + i] * ks[s * ldk + i], expf(bs[t * ldk + i] - bs[s * ldk + i]), a);
+        }
+        A[idx] = a;
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < C * dk; idx += blockDim.x) {
+        int t = idx / dk, i = idx - t * dk;
+        qs[t * ldk + i] *= expf(bs[t * ldk + i]);
+    }
+    __syncthreads();
+    for (int idx = threadIdx.x; idx < len * dv; idx += blockDim.x) {
+        int t = idx / dv, j = idx - t * dv;
+        float acc = 0.f;
+        for (int i = 0; i < dk; ++i) acc = fmaf(qs[t * ldk + i], S[i * dv + j], acc);
+        for (int s = 0; s <= t; ++s) acc = fmaf(A[t * C + s], vv[s * dv + j], acc);
+        int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
+        out[tok_offset(g, b, p, h, dv) + j] = __float2half_rn(acc);
+    }
+}
+
+size_t summary_smem(const Geom &g) { return sizeof(float) * (size_t)g.chunk * (2 * (g.dk + 1) + g.dv); }
+size_t output_smem(const Geom &g) {
+    return sizeof(float) * ((size_t)g.chunk * (3 * (g.dk + 1) + g.dv + g.chunk) + (size_t)g.dk * g.dv);
+}
+
+}  // namespace
+
+cudaError_t launch_summary_v0(const __half *k, const __half *v, const float *g, const Geom &geo,
+                              float *dS, float *gamma, cudaStream_t st) {
+    size_t smem = summary_smem(geo);
+    cudaError_t e = cudaFuncSetAttribute(summary_simt_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((int64_t)geo.nc * geo.B * geo.heads));
+    summary_simt_kernel<<<grid, kThreads, smem, st>>>(k, v, g, geo, dS, gamma);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                           float *S_enter, cudaStream_t st) {
+    dim3 grid((unsigned)((int64_t)((dk * dv + kThreads - 1) / kThreads) * nseq));
+    scan_simt_kernel<<<grid, kThreads, 0, st>>>(dS, gamma, nc, dk, dv, S_enter);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, const float *g,
+                             const float *S_enter, const Geom &geo, __half *out, cudaStream_t st) {
+    size_t smem = output_smem(geo);
+    cudaError_t e = cudaFuncSetAttribute(output_simt_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((int64_t)geo.nc * geo.B * geo.heads));
+    output_simt_kernel<<<grid, kThreads, smem, st>>>(q, k, v, g, S_enter, geo, out);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace gtr

@@ -1,0 +1,366 @@
+// gtr_gla_api.cu -- the C ABI (include/gtr_gla.h): argument checks, the
+// internal workspace, and dispatch to the kernels.  Host code only.
+#include "gtr_gla.h"
+
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "gla_common.cuh"
+
+namespace gtr {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+namespace {
+
+thread_local char t_err[256] = "";
+
+gtr_status_t fail(gtr_status_t s, const char *fmt, const char *detail = "") {
+    std::snprintf(t_err, sizeof t_err, fmt, detail);
+    return s;
+}
+
+gtr_status_t cuda_fail(cudaError_t e, const char *what) {
+    std::snprintf(t_err, sizeof t_err, "%s: %s", what, cudaGetErrorString(e));
+    return GTR_ERR_CUDA;
+}
+
+bool supported_d(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool supported_chunk(int c) { return c == 16 || c == 32 || c == 64; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;
+};
+Range span(const void *p, size_t bytes) {
+    uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return {a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi && a.hi > a.lo && b.hi > b.lo; }
+
+// Shape checks common to every token-layout entry point.  Sets `geo`.
+// Returns GTR_OK, or an error; `empty` is set when there is no work.
+gtr_status_t check_shape(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                         int direction, int chunk, Geom &geo, bool &empty) {
+    if (B < 0 || heads < 0 || grid_h < 0 || grid_w < 0)
+        return fail(GTR_ERR_INVALID_ARG, "negative size%s");
+    if (direction < 0 || direction > 3) return fail(GTR_ERR_INVALID_ARG, "bad direction%s");
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "d_k and d_v must be 16, 32, 64 or 128%s");
+    if (!supported_chunk(chunk))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "chunk must be 16, 32 or 64%s");
+    int64_t N = (int64_t)grid_h * grid_w;
+    if (N > (int64_t)1 << 30) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "more than 2^30 tokens%s");
+    empty = (B == 0 || heads == 0 || N == 0);
+    int64_t nc = (N + chunk - 1) / chunk;
+    if (!empty && nc * B * heads >= ((int64_t)1 << 31))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "more than 2^31 chunk tiles%s");
+    geo.B = B; geo.heads = heads; geo.H = grid_h; geo.W = grid_w;
+    geo.dk = d_k; geo.dv = d_v; geo.dir = direction; geo.chunk = chunk;
+    geo.N = (int)N; geo.nc = (int)nc;
+    return GTR_OK;
+}
+
+size_t tok_bytes(const Geom &g, int d, size_t elem) {
+    return (size_t)g.B * g.N * g.heads * d * elem;
+}
+
+// Internal workspace: one grow-only device buffer per (device, stream).
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+gtr_status_t get_workspace(size_t bytes, cudaStream_t st, void **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    Workspace &w = g_ws[{dev, st}];
+    if (w.bytes < bytes) {
+        if (w.ptr) {
+            e = cudaStreamSynchronize(st);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+            cudaFree(w.ptr);
+            w.ptr = nullptr;
+            w.bytes = 0;
+        }
+        size_t want = (bytes + 0xFFFFF) & ~(size_t)0xFFFFF;  // round up to 1 MiB
+        e = cudaMalloc(&w.ptr, want);
+        if (e != cudaSuccess) {
+            w.ptr = nullptr;
+            cudaGetLastError();
+            return fail(GTR_ERR_OOM, "workspace allocation failed%s");
+        }
+        e = cudaMemset(w.ptr, 0, want);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset");
+        w.bytes = want;
+    }
+    *out = w.ptr;
+    return GTR_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t three_phase_ws(const Geom &g) {
+    size_t nseq = (size_t)g.B * g.heads;
+    return align256(nseq * g.nc * g.dk * g.dv * sizeof(float)) +
+           align256(nseq * g.nc * g.dk * sizeof(float));
+}
+
+gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, const float *g,
+                             const Geom &geo, __half *out, cudaStream_t st) {
+    void *ws = nullptr;
+    gtr_status_t s = get_workspace(three_phase_ws(geo), st, &ws);
+    if (s != GTR_OK) return s;
+    size_t nseq = (size_t)geo.B * geo.heads;
+    float *dS = static_cast<float *>(ws);
+    float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
+                                             align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
+    cudaError_t e = launch_summary_v0(k, v, g, geo, dS, gamma, st);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
+    e = launch_scan_v0(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, st);
+    if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
+    e = launch_output_v0(q, k, v, g, dS, geo, out, st);
+    if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
+    return GTR_OK;
+}
+
+gtr_status_t forward_impl(const void *q, const void *k, const void *v, const float *g, int B,
+                          int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                          int chunk, int schedule, void *out, void *stream) {
+    t_err[0] = '\0';
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE)
+        return fail(GTR_ERR_INVALID_ARG, "bad schedule%s");
+    if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out))
+        return fail(GTR_ERR_MISALIGNED, "device pointers must be 16-byte aligned%s");
+    Range ro = span(out, tok_bytes(geo, d_v, 2));
+    if (overlap(ro, span(q, tok_bytes(geo, d_k, 2))) || overlap(ro, span(k, tok_bytes(geo, d_k, 2))) ||
+        overlap(ro, span(v, tok_bytes(geo, d_v, 2))) || overlap(ro, span(g, tok_bytes(geo, d_k, 4))))
+        return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
+    if (empty) return GTR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    return run_three_phase(static_cast<const __half *>(q), static_cast<const __half *>(k),
+                           static_cast<const __half *>(v), g, geo, static_cast<__half *>(out), st);
+}
+
+}  // namespace
+}  // namespace gtr
+
+using namespace gtr;
+
+extern "C" {
+
+gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const float *g, int B,
+                             int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                             int chunk, void *out, void *stream) {
+    return forward_impl(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
+                        GTR_SCHED_AUTO, out, stream);
+}
+
+gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, const float *g,
+                                int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                int direction, int chunk, int schedule, void *out, void *stream) {
+    return forward_impl(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
+                        schedule, out, stream);
+}
+
+gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, const float *g,
+                                  int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                  int direction, int chunk, void *out, void *stream) {
+    t_err[0] = '\0';
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (empty) return GTR_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t bq = align256(tok_bytes(geo, d_k, 2)), bv = align256(tok_bytes(geo, d_v, 2));
+    const size_t bg = align256(tok_bytes(geo, d_k, 4));
+    // Staging for inputs and output lives in the workspace of a private
+    // key (the stream's workspace is used by the forward call itself).
+    void *stage = nullptr;
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+        size_t need = 2 * bq + 2 * bv + bg;
+        std::lock_guard<std::mutex> lk(g_ws_mu);
+        // distinct key: the stream handle with its lowest bit set can never
+        // be a real stream handle (those are at least 8-byte aligned)
+        cudaStream_t key = reinterpret_cast<cudaStream_t>(reinterpret_cast<uintptr_t>(st) | 1u);
+        Workspace &w = g_ws[{dev, key}];
+        if (w.bytes < need) {
+            if (w.ptr) {
+                e = cudaStreamSynchronize(st);
+                if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+                cudaFree(w.ptr);
+                w.ptr = nullptr;
+                w.bytes = 0;
+            }
+            e = cudaMalloc(&w.ptr, need);
+            if (e != cudaSuccess) {
+                w.ptr = nullptr;
+                cudaGetLastError();
+                return fail(GTR_ERR_OOM, "staging allocation failed%s");
+            }
+            w.bytes = need;
+        }
+        stage = w.ptr;
+    }
+    char *p = static_cast<char *>(stage);
+    void *dq = p, *dk_ = p + bq, *dv_ = p + 2 * bq, *dg = p + 2 * bq + bv, *dout = p + 2 * bq + bv + bg;
+    cudaError_t e;
+    if ((e = cudaMemcpyAsync(dq, q, tok_bytes(geo, d_k, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dk_, k, tok_bytes(geo, d_k, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dv_, v, tok_bytes(geo, d_v, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
+        (e = cudaMemcpyAsync(dg, g, tok_bytes(geo, d_k, 4), cudaMemcpyHostToDevice, st)) != cudaSuccess)
+        return cuda_fail(e, "host-to-device copy");
+    s = forward_impl(dq, dk_, dv_, static_cast<const float *>(dg), B, heads, grid_h, grid_w, d_k, d_v,
+                     direction, chunk, GTR_SCHED_AUTO, dout, stream);
+    if (s != GTR_OK) return s;
+    if ((e = cudaMemcpyAsync(out, dout, tok_bytes(geo, d_v, 2), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+        return cuda_fail(e, "device-to-host copy");
+    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    return GTR_OK;
+}
+
+gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g, int B, int heads,
+                                   int grid_h, int grid_w, int d_k, int d_v, int direction,
+                                   int chunk, float *dS, float *gamma, void *stream) {
+    t_err[0] = '\0';
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (!k || !v || !g || !dS || !gamma) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(dS) || !aligned16(gamma))
+        return fail(GTR_ERR_MISALIGNED, "device pointers must be 16-byte aligned%s");
+    size_t nseq = (size_t)geo.B * geo.heads;
+    Range rs = span(dS, nseq * geo.nc * d_k * d_v * 4), rg = span(gamma, nseq * geo.nc * d_k * 4);
+    Range in[3] = {span(k, tok_bytes(geo, d_k, 2)), span(v, tok_bytes(geo, d_v, 2)),
+                   span(g, tok_bytes(geo, d_k, 4))};
+    for (const Range &r : in)
+        if (overlap(rs, r) || overlap(rg, r)) return fail(GTR_ERR_ALIAS, "an output overlaps an input%s");
+    if (overlap(rs, rg)) return fail(GTR_ERR_ALIAS, "dS overlaps gamma%s");
+    if (empty) return GTR_OK;
+    cudaError_t e = launch_summary_v0(static_cast<const __half *>(k), static_cast<const __half *>(v),
+                                      g, geo, dS, gamma, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk summary launch");
+}
+
+gtr_status_t gtr_gla_boundary_scan(const float *dS, const float *gamma, int B, int heads,
+                                   int n_chunks, int d_k, int d_v, float *S_enter, void *stream) {
+    t_err[0] = '\0';
+    if (B < 0 || heads < 0 || n_chunks < 0) return fail(GTR_ERR_INVALID_ARG, "negative size%s");
+    if (!supported_d(d_k) || !supported_d(d_v))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "d_k and d_v must be 16, 32, 64 or 128%s");
+    if (!dS || !gamma || !S_enter) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(dS) || !aligned16(gamma) || !aligned16(S_enter))
+        return fail(GTR_ERR_MISALIGNED, "device pointers must be 16-byte aligned%s");
+    int64_t nseq = (int64_t)B * heads;
+    if (nseq * (((int64_t)d_k * d_v + 255) / 256) >= ((int64_t)1 << 31))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "too many sequences%s");
+    size_t sb = (size_t)nseq * n_chunks * d_k * d_v * 4;
+    Range rs = span(S_enter, sb);
+    if (S_enter != dS && overlap(rs, span(dS, sb))) return fail(GTR_ERR_ALIAS, "S_enter partially overlaps dS%s");
+    if (overlap(rs, span(gamma, (size_t)nseq * n_chunks * d_k * 4)))
+        return fail(GTR_ERR_ALIAS, "S_enter overlaps gamma%s");
+    if (nseq == 0 || n_chunks == 0) return GTR_OK;
+    cudaError_t e = launch_scan_v0(dS, gamma, (int)nseq, n_chunks, d_k, d_v, S_enter,
+                                   static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "boundary scan launch");
+}
+
+gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, const float *g,
+                                  const float *S_enter, int B, int heads, int grid_h, int grid_w,
+                                  int d_k, int d_v, int direction, int chunk, void *out,
+                                  void *stream) {
+    t_err[0] = '\0';
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (!q || !k || !v || !g || !S_enter || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(S_enter) ||
+        !aligned16(out))
+        return fail(GTR_ERR_MISALIGNED, "device pointers must be 16-byte aligned%s");
+    size_t nseq = (size_t)geo.B * geo.heads;
+    Range ro = span(out, tok_bytes(geo, d_v, 2));
+    Range in[5] = {span(q, tok_bytes(geo, d_k, 2)), span(k, tok_bytes(geo, d_k, 2)),
+                   span(v, tok_bytes(geo, d_v, 2)), span(g, tok_bytes(geo, d_k, 4)),
+                   span(S_enter, nseq * geo.nc * d_k * d_v * 4)};
+    for (const Range &r : in)
+        if (overlap(ro, r)) return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
+    if (empty) return GTR_OK;
+    cudaError_t e = launch_output_v0(static_cast<const __half *>(q), static_cast<const __half *>(k),
+                                     static_cast<const __half *>(v), g, S_enter, geo,
+                                     static_cast<__half *>(out), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk output launch");
+}
+
+size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                               int chunk, int schedule) {
+    Geom geo;
+    bool empty = false;
+    if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return 0;
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE || empty) return 0;
+    return three_phase_ws(geo);
+}
+
+gtr_status_t gtr_gla_get_last_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    return GTR_OK;
+}
+
+gtr_status_t gtr_gla_release_workspace(void) {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto &kv : g_ws) {
+        if (kv.second.ptr) {
+            cudaSetDevice(kv.first.first);
+            cudaDeviceSynchronize();
+            cudaFree(kv.second.ptr);
+        }
+    }
+    g_ws.clear();
+    cudaSetDevice(cur);
+    return GTR_OK;
+}
+
+const char *gtr_gla_status_string(gtr_status_t s) {
+    switch (s) {
+    case GTR_OK: return "ok";
+    case GTR_ERR_INVALID_ARG: return "invalid argument";
+    case GTR_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case GTR_ERR_MISALIGNED: return "misaligned pointer";
+    case GTR_ERR_ALIAS: return "output aliases an input";
+    case GTR_ERR_CUDA: return "CUDA error";
+    case GTR_ERR_TIMEOUT: return "device wait timed out";
+    case GTR_ERR_OOM: return "out of device memory";
+    }
+    return "unknown status";
+}
+
+const char *gtr_gla_last_error(void) { return t_err; }
+
+uint64_t gtr_gla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int gtr_gla_version(void) { return 100; }
+
+}  // extern "C"

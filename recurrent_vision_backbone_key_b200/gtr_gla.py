@@ -1,0 +1,181 @@
+"""ctypes binding of libgtr_gla.so (the C ABI in include/gtr_gla.h).
+
+Argument marshalling only: every step of the GLA forward runs in the CUDA
+library.  Functions named ``gtr_gla_*`` mirror the C entry points one to one
+and accept torch tensors (their ``data_ptr()`` is passed) or raw integer
+addresses; a ``stream`` argument may be a ``torch.cuda.Stream``, a raw
+``cudaStream_t`` integer, or None for torch's current stream.  Each returns
+the integer status; :func:`check` turns a non-zero status into
+:class:`GtrError`.  :func:`forward` is the tensor-level convenience call.
+
+The library must be built (``python -m recurrent_vision_backbone_key_b200.build``);
+loading fails loudly otherwise -- there is no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgtr_gla.so")
+
+GTR_OK = 0
+STATUS_NAMES = {
+    0: "GTR_OK", 1: "GTR_ERR_INVALID_ARG", 2: "GTR_ERR_UNSUPPORTED_SHAPE",
+    3: "GTR_ERR_MISALIGNED", 4: "GTR_ERR_ALIAS", 5: "GTR_ERR_CUDA", 6: "GTR_ERR_TIMEOUT",
+    7: "GTR_ERR_OOM",
+}
+DIRECTIONS = {"l2r": 0, "r2l": 1, "t2b": 2, "b2t": 3}
+SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2}
+
+# Every symbol include/gtr_gla.h declares, with (restype, argtypes).
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+SIGNATURES = {
+    "gtr_gla_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_forward_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_chunk_summary": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gtr_gla_boundary_scan": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "gtr_gla_get_last_device_status": (_I, [_P]),
+    "gtr_gla_release_workspace": (_I, []),
+    "gtr_gla_status_string": (ctypes.c_char_p, [_I]),
+    "gtr_gla_last_error": (ctypes.c_char_p, []),
+    "gtr_gla_launch_count": (ctypes.c_uint64, []),
+    "gtr_gla_version": (_I, []),
+}
+
+_lib = None
+
+
+class GtrError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m recurrent_vision_backbone_key_b200.build`"
+                " (no CPU fallback exists)")
+        lib = ctypes.CDLL(path)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _addr(x):
+    if x is None:
+        return None
+    if isinstance(x, torch.Tensor):
+        return x.data_ptr()
+    return int(x)
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dir(d):
+    return DIRECTIONS[d] if isinstance(d, str) else int(d)
+
+
+def last_error() -> str:
+    return load().gtr_gla_last_error().decode()
+
+
+def check(status: int) -> int:
+    if status != GTR_OK:
+        raise GtrError(status, last_error())
+    return status
+
+
+def gtr_gla_forward(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                    stream=None) -> int:
+    return load().gtr_gla_forward(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h, grid_w,
+                                  d_k, d_v, _dir(direction), chunk, _addr(out), _stream(stream))
+
+
+def gtr_gla_forward_ex(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, schedule,
+                       out, stream=None) -> int:
+    sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    return load().gtr_gla_forward_ex(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h,
+                                     grid_w, d_k, d_v, _dir(direction), chunk, sched, _addr(out),
+                                     _stream(stream))
+
+
+def gtr_gla_forward_host(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                         stream=None) -> int:
+    return load().gtr_gla_forward_host(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h,
+                                       grid_w, d_k, d_v, _dir(direction), chunk, _addr(out),
+                                       _stream(stream))
+
+
+def gtr_gla_chunk_summary(k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, dS, gamma,
+                          stream=None) -> int:
+    return load().gtr_gla_chunk_summary(_addr(k), _addr(v), _addr(g), B, heads, grid_h, grid_w,
+                                        d_k, d_v, _dir(direction), chunk, _addr(dS), _addr(gamma),
+                                        _stream(stream))
+
+
+def gtr_gla_boundary_scan(dS, gamma, B, heads, n_chunks, d_k, d_v, S_enter, stream=None) -> int:
+    return load().gtr_gla_boundary_scan(_addr(dS), _addr(gamma), B, heads, n_chunks, d_k, d_v,
+                                        _addr(S_enter), _stream(stream))
+
+
+def gtr_gla_chunk_output(q, k, v, g, S_enter, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
+                         out, stream=None) -> int:
+    return load().gtr_gla_chunk_output(_addr(q), _addr(k), _addr(v), _addr(g), _addr(S_enter), B,
+                                       heads, grid_h, grid_w, d_k, d_v, _dir(direction), chunk,
+                                       _addr(out), _stream(stream))
+
+
+def gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule=0) -> int:
+    return int(load().gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule))
+
+
+def gtr_gla_get_last_device_status(stream=None) -> int:
+    return load().gtr_gla_get_last_device_status(_stream(stream))
+
+
+def gtr_gla_release_workspace() -> int:
+    return load().gtr_gla_release_workspace()
+
+
+def gtr_gla_status_string(status: int) -> str:
+    return load().gtr_gla_status_string(status).decode()
+
+
+def gtr_gla_launch_count() -> int:
+    return int(load().gtr_gla_launch_count())
+
+
+def gtr_gla_version() -> int:
+    return int(load().gtr_gla_version())
+
+
+def forward(q, k, v, g, grid_h, grid_w, direction=0, chunk=64, schedule=0, out=None, stream=None):
+    """Tensor-level GLA forward: shapes taken from q [B,N,heads,d_k] and
+    v [B,N,heads,d_v]; allocates ``out`` if not given; raises GtrError."""
+    B, N, heads, d_k = q.shape
+    d_v = v.shape[3]
+    if out is None:
+        out = torch.empty((B, N, heads, d_v), dtype=torch.float16, device=v.device)
+    check(gtr_gla_forward_ex(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
+                             schedule, out, stream))
+    return out

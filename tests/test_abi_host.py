@@ -1,0 +1,99 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, it
+exports every function include/gtr_gla.h declares, and argument validation
+returns the documented status before any CUDA call is made."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from recurrent_vision_backbone_key_b200 import build as libbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    libbuild.build()
+    from recurrent_vision_backbone_key_b200 import gtr_gla
+    return gtr_gla
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(gtr_\w+)\s*\(", text))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    cdll = lib.load()
+    for n in sorted(names):
+        assert hasattr(cdll, n), n
+    assert names <= set(lib.SIGNATURES), names - set(lib.SIGNATURES)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.gtr_gla_version() >= 100
+    assert lib.gtr_gla_status_string(0) == "ok"
+    assert lib.gtr_gla_status_string(6) == "device wait timed out"
+
+
+A = 1 << 20  # fake, 16-byte aligned "device" addresses; never dereferenced
+
+
+def fwd(lib, **kw):
+    args = dict(q=A, k=2 * A, v=3 * A, g=4 * A, B=1, heads=2, grid_h=4, grid_w=4, d_k=16,
+                d_v=16, direction=0, chunk=16, out=5 * A, stream=0)
+    args.update(kw)
+    return lib.gtr_gla_forward(**args)
+
+
+def test_error_paths(lib):
+    assert fwd(lib, q=None) == 1
+    assert fwd(lib, out=None) == 1
+    assert fwd(lib, direction=4) == 1
+    assert fwd(lib, direction=-1) == 1
+    assert fwd(lib, B=-1) == 1
+    assert fwd(lib, d_k=48) == 2
+    assert fwd(lib, d_v=256) == 2
+    assert fwd(lib, chunk=128) == 2
+    assert fwd(lib, chunk=0) == 2
+    assert fwd(lib, q=A + 8) == 3
+    assert fwd(lib, g=4 * A + 4) == 3
+    # out overlapping q (q spans 1*16*2*16*2 = 1 KiB)
+    assert fwd(lib, out=A + 512) == 4
+    assert fwd(lib, out=4 * A) == 4
+    assert "overlaps" in lib.last_error()
+
+
+def test_empty_problems_launch_nothing(lib):
+    before = lib.gtr_gla_launch_count()
+    assert fwd(lib, B=0) == 0
+    assert fwd(lib, grid_h=0) == 0
+    assert fwd(lib, heads=0) == 0
+    assert lib.gtr_gla_launch_count() == before
+
+
+def test_phase_entry_points_validate(lib):
+    assert lib.gtr_gla_chunk_summary(2 * A, 3 * A, 4 * A, 1, 1, 4, 4, 16, 16, 0, 16, None, 6 * A, 0) == 1
+    assert lib.gtr_gla_chunk_summary(2 * A, 3 * A, 4 * A, 1, 1, 4, 4, 16, 16, 0, 16, 2 * A, 6 * A, 0) == 4
+    assert lib.gtr_gla_boundary_scan(A, 2 * A, 1, 1, 3, 16, 24, 3 * A, 0) == 2
+    assert lib.gtr_gla_boundary_scan(A, 2 * A, 1, 1, 0, 16, 16, 3 * A, 0) == 0
+    # partial overlap of S_enter with dS is an error, exact in-place is fine
+    assert lib.gtr_gla_boundary_scan(A, 2 * A, 1, 1, 2, 16, 16, A + 16, 0) == 4
+    assert lib.gtr_gla_chunk_output(A, 2 * A, 3 * A, 4 * A, 6 * A, 1, 1, 4, 4, 16, 16, 5, 16, 5 * A, 0) == 1
+    assert lib.gtr_gla_chunk_output(A, 2 * A, 3 * A, 4 * A, 6 * A, 1, 1, 4, 4, 16, 16, 0, 16, 6 * A, 0) == 4
+
+
+def test_workspace_bytes(lib):
+    # three-phase: dS (nseq*nc*dk*dv fp32) + gamma (nseq*nc*dk fp32), 256-byte aligned
+    n = lib.gtr_gla_workspace_bytes(2, 3, 10, 10, 32, 64, 16, 2)
+    nc = (100 + 15) // 16
+    assert n >= 6 * nc * 32 * 64 * 4 + 6 * nc * 32 * 4
+    assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 24, 16, 16, 2) == 0

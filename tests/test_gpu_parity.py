@@ -1,0 +1,220 @@
+"""GPU parity: the CUDA path against the fp64 oracle on the same seeded inputs.
+
+Bar: max |o_gpu - o_ref| <= 2e-3 * max |o_ref| (fp16 I/O, fp32 accumulate),
+and bit-exact agreement of the scan-order index maps.  Small cases are
+compared in full; the full-size workloads are compared on sampled (b, h)
+sequences that the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from recurrent_vision_backbone_key_b200 import gtr_gla
+from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs, make_inputs
+from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, slice_of
+
+pytestmark = pytest.mark.gpu
+
+SCHEDULES = ["auto", "three_phase"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    gtr_gla.load()
+
+
+def oracle_full(oracle_mod, q, k, v, g, H, W, direction):
+    return oracle_mod.gla_serial(q.cpu(), k.cpu(), v.cpu(), g.cpu(), H, W, direction)
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_tiny(oracle_mod, schedule):
+    w = WORKLOADS["tiny"]
+    q, k, v, g = gpu_inputs(w.B, w.grid_h, w.grid_w, w.heads, w.d_k, w.d_v, seed=0)
+    out = run_forward(q, k, v, g, w.grid_h, w.grid_w, 0, w.chunk, schedule)
+    compare(out, oracle_full(oracle_mod, q, k, v, g, w.grid_h, w.grid_w, 0))
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+@pytest.mark.parametrize("chunk", [16, 32, 64])
+def test_ragged_grid(oracle_mod, schedule, direction, chunk):
+    # 7 x 9 = 63 tokens (ragged last chunk), 9 x 15 = 135 tokens (several chunks)
+    for (H, W) in [(7, 9), (9, 15)]:
+        q, k, v, g = gpu_inputs(2, H, W, 3, 32, 64, seed=100 + direction + chunk)
+        out = run_forward(q, k, v, g, H, W, direction, chunk, schedule)
+        compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, direction))
+
+
+@pytest.mark.parametrize("dk", [16, 32, 64, 128])
+@pytest.mark.parametrize("dv", [16, 32, 64, 128])
+def test_all_head_dims(oracle_mod, dk, dv):
+    H, W = 5, 23  # 115 tokens
+    q, k, v, g = gpu_inputs(1, H, W, 2, dk, dv, seed=dk * 1000 + dv)
+    for schedule in SCHEDULES:
+        for chunk in (16, 64):
+            out = run_forward(q, k, v, g, H, W, 3, chunk, schedule)
+            compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, 3))
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("shape", [(1, 1), (1, 37), (37, 1), (2, 2), (16, 16)])
+def test_degenerate_grids(oracle_mod, schedule, shape):
+    H, W = shape
+    q, k, v, g = gpu_inputs(2, H, W, 2, 64, 64, seed=H * 100 + W)
+    for direction in range(4):
+        out = run_forward(q, k, v, g, H, W, direction, 64, schedule)
+        compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, direction))
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_special_gates(oracle_mod, schedule):
+    H, W = 12, 11
+    q, k, v, g = gpu_inputs(1, H, W, 2, 64, 32, seed=7)
+    cases = {
+        "open": torch.zeros_like(g),                      # causal linear attention
+        "closed": torch.full_like(g, -1.0e4),             # memoryless
+        "strong": gpu_inputs(1, H, W, 2, 64, 32, seed=7, gate="strong")[3],
+        "mixed": torch.where(torch.rand_like(g) < 0.5, torch.zeros_like(g), g * 40.0),
+    }
+    for name, gg in cases.items():
+        out = run_forward(q, k, v, gg, H, W, 2, 64, schedule)
+        compare(out, oracle_full(oracle_mod, q, k, v, gg, H, W, 2))
+
+
+@pytest.mark.parametrize("direction", [0, 1, 2, 3])
+def test_gtr_s_640_all_directions(oracle_mod, direction):
+    w = WORKLOADS["gtr_s_640"]
+    q, k, v, g = gpu_inputs(w.B, w.grid_h, w.grid_w, w.heads, w.d_k, w.d_v, seed=direction)
+    ref = oracle_full(oracle_mod, q, k, v, g, w.grid_h, w.grid_w, direction)
+    for schedule in SCHEDULES:
+        out = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk, schedule)
+        compare(out, ref)
+
+
+def test_phases_against_oracle_intermediates(oracle_mod):
+    """chunk_summary, boundary_scan and chunk_output one by one."""
+    H, W, heads, dk, dv, chunk = 10, 13, 2, 32, 64, 32
+    q, k, v, g = gpu_inputs(2, H, W, heads, dk, dv, seed=77)
+    direction = 3
+    ref_out, ref_dS, ref_gamma, ref_Se = oracle_mod.gla_chunked(
+        q.cpu(), k.cpu(), v.cpu(), g.cpu(), H, W, direction, chunk)
+    B, nc = 2, (H * W + chunk - 1) // chunk
+    dS = torch.empty((B, heads, nc, dk, dv), device="cuda", dtype=torch.float32)
+    gamma = torch.empty((B, heads, nc, dk), device="cuda", dtype=torch.float32)
+    gtr_gla.check(gtr_gla.gtr_gla_chunk_summary(k, v, g, B, heads, H, W, dk, dv, direction, chunk,
+                                                dS, gamma))
+    torch.cuda.synchronize()
+    compare(dS, ref_dS, tol=1e-5)
+    compare(gamma, ref_gamma, tol=1e-5)
+    Se = torch.empty_like(dS)
+    gtr_gla.check(gtr_gla.gtr_gla_boundary_scan(dS, gamma, B, heads, nc, dk, dv, Se))
+    torch.cuda.synchronize()
+    compare(Se, ref_Se, tol=1e-5)
+    # in place
+    dS2 = dS.clone()
+    gtr_gla.check(gtr_gla.gtr_gla_boundary_scan(dS2, gamma, B, heads, nc, dk, dv, dS2))
+    torch.cuda.synchronize()
+    assert torch.equal(dS2, Se)
+    # output from the oracle's own boundary states
+    out = torch.empty_like(v)
+    Se_ref = torch.from_numpy(ref_Se).float().cuda()
+    gtr_gla.check(gtr_gla.gtr_gla_chunk_output(q, k, v, g, Se_ref, B, heads, H, W, dk, dv,
+                                               direction, chunk, out))
+    torch.cuda.synchronize()
+    compare(out, ref_out)
+
+
+def _rot(x):
+    return x.flip(1).contiguous()
+
+
+def _tr(x, H, W):
+    B, N, h, d = x.shape
+    return x.reshape(B, H, W, h, d).transpose(1, 2).reshape(B, N, h, d).contiguous()
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+@pytest.mark.parametrize("shape", [(40, 40), (7, 19)])
+def test_direction_maps_bit_exact(schedule, shape):
+    """T->B equals L->R on the transposed grid, R->L equals L->R on the
+    rotated grid, B->T equals T->B on the rotated grid: bit for bit."""
+    H, W = shape
+    q, k, v, g = gpu_inputs(2, H, W, 3, 64, 64, seed=5)
+    X = (q, k, v, g)
+    f = lambda d, Y, h, w: run_forward(*Y, h, w, d, 64, schedule)
+    assert torch.equal(f(1, X, H, W), _rot(f(0, tuple(_rot(a) for a in X), H, W)))
+    assert torch.equal(f(2, X, H, W), _tr(f(0, tuple(_tr(a, H, W) for a in X), W, H), W, H))
+    assert torch.equal(f(3, X, H, W), _rot(f(2, tuple(_rot(a) for a in X), H, W)))
+
+
+def _sampled_check(oracle_mod, w, q, k, v, g, out, direction, n_slices, seed):
+    errs = []
+    for (b, h) in sample_slices(w.B, w.heads, n_slices, seed):
+        ref = oracle_mod.gla_serial(slice_of(q, b, h), slice_of(k, b, h), slice_of(v, b, h),
+                                    slice_of(g, b, h), w.grid_h, w.grid_w, direction)
+        errs.append(compare(out[b:b + 1, :, h:h + 1, :], ref)[0])
+    return max(errs)
+
+
+@pytest.mark.parametrize("direction", [0, 2])
+def test_batched_full_size_sampled(oracle_mod, direction):
+    w = WORKLOADS["batched"]
+    q, k, v, g = make_workload_inputs(w, seed=direction, device="cuda")
+    out = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk)
+    assert torch.isfinite(out).all()
+    _sampled_check(oracle_mod, w, q, k, v, g, out, direction, 6, seed=direction)
+
+
+def test_highres_twelve_block_stack_sampled(oracle_mod):
+    """Twelve consecutive calls cycling L->R, R->L, T->B, B->T, each call with
+    fresh inputs from the same recipe."""
+    w = WORKLOADS["highres_1280"]
+    for i in range(12):
+        direction = i % 4
+        q, k, v, g = make_workload_inputs(w, seed=1000 + i, device="cuda")
+        out = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk)
+        _sampled_check(oracle_mod, w, q, k, v, g, out, direction, 2, seed=i)
+
+
+@pytest.mark.parametrize("grid", [32, 64, 128, 256])
+@pytest.mark.parametrize("batch", [1, 8])
+@pytest.mark.parametrize("gate", ["mild", "strong"])
+def test_resolution_sweep_sampled(oracle_mod, grid, batch, gate):
+    w = WORKLOADS[f"sweep_b{batch}_{grid}_{gate}"]
+    q, k, v, g = make_workload_inputs(w, seed=grid + batch, device="cuda")
+    for direction in range(4):
+        out = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk)
+        n = 2 if grid >= 128 else 3
+        _sampled_check(oracle_mod, w, q, k, v, g, out, direction, n, seed=direction)
+        del out
+    torch.cuda.empty_cache()
+
+
+def test_host_entry_point_matches_device_call(oracle_mod):
+    H, W, heads, dk, dv = 20, 20, 2, 64, 64
+    q, k, v, g = make_inputs(1, H, W, heads, dk, dv, seed=3)
+    pin = lambda x: x.pin_memory()
+    qh, kh, vh, gh = (pin(x) for x in (q, k, v, g))
+    out_h = torch.empty((1, H * W, heads, dv), dtype=torch.float16).pin_memory()
+    gtr_gla.check(gtr_gla.gtr_gla_forward_host(qh, kh, vh, gh, 1, heads, H, W, dk, dv, 2, 64, out_h))
+    out_d = run_forward(q.cuda(), k.cuda(), v.cuda(), g.cuda(), H, W, 2, 64)
+    assert torch.equal(out_h, out_d.cpu())
+    compare(out_h, oracle_mod.gla_serial(q, k, v, g, H, W, 2))
+
+
+def test_empty_and_streams():
+    q, k, v, g = gpu_inputs(1, 4, 4, 1, 16, 16, seed=1)
+    out = torch.zeros_like(v)
+    before = gtr_gla.gtr_gla_launch_count()
+    assert gtr_gla.gtr_gla_forward(q, k, v, g, 0, 1, 4, 4, 16, 16, 0, 16, out) == 0
+    assert gtr_gla.gtr_gla_launch_count() == before
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        o1 = gtr_gla.forward(q, k, v, g, 4, 4, chunk=16)
+    s.synchronize()
+    o2 = run_forward(q, k, v, g, 4, 4, 0, 16)
+    assert torch.equal(o1, o2)
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0
