@@ -112,6 +112,28 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
                                   int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                   int direction, int chunk, void *out, void *stream);
 
+/* gtr_gla_forward without any device allocation.  The GTR pages have no
+ * counterpart to this call; it exists for callers that cannot let a library
+ * call cudaMalloc while they run: hosts that own every byte of device memory
+ * through their own allocator or a fixed budget (engine plugins, serving
+ * runtimes) and real-time loops that forbid allocation after start-up.
+ * Same arguments, layouts, checks and result as gtr_gla_forward (three-phase
+ * schedule).  Its scratch is a 16 MiB array in the library's own device
+ * memory, which every GPU that loads the library holds until the process
+ * exits.  Problems needing more, i.e. B*heads*ceil(N/chunk)*d_k*(d_v+1)*4
+ * bytes above 16 MiB (after 256-byte rounding of the two parts), are
+ * rejected with GTR_ERR_UNSUPPORTED_SHAPE and nothing is launched.
+ * The first call on a device looks up that device's scratch address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * All calls on a device share the one scratch array: calls whose kernels may
+ * overlap on the GPU (different streams without ordering between them)
+ * race and give wrong results; order them on one stream or with events.
+ * The scratch keeps the last call's contents; every entry a call reads is
+ * first written by the same call, so nothing needs clearing. */
+gtr_status_t gtr_gla_forward_noalloc(const void *q, const void *k, const void *v, const float *g,
+                                     int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                     int direction, int chunk, void *out, void *stream);
+
 /* Phase 1, chunk summaries (GTR project page, "A Kernel That Makes
  * Recurrence Fast": per-chunk summaries in parallel over the chunk x head
  * grid).  With nc = ceil(N/chunk) and b_s the inclusive prefix sum of g

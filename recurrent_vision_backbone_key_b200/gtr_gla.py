@@ -37,6 +37,7 @@ SIGNATURES = {
     "gtr_gla_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_summary": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gtr_gla_boundary_scan": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -124,6 +125,13 @@ def gtr_gla_forward_host(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, directi
     return load().gtr_gla_forward_host(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h,
                                        grid_w, d_k, d_v, _dir(direction), chunk, _addr(out),
                                        _stream(stream))
+
+
+def gtr_gla_forward_noalloc(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                            stream=None) -> int:
+    return load().gtr_gla_forward_noalloc(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h,
+                                          grid_w, d_k, d_v, _dir(direction), chunk, _addr(out),
+                                          _stream(stream))
 
 
 def gtr_gla_chunk_summary(k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, dS, gamma,
