@@ -207,7 +207,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS))
-    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase", "three_phase_simt"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -223,7 +223,7 @@ def main():
     torch.cuda.set_device(dev)
     lib = gtr_gla.load()
     stream = torch.cuda.current_stream()
-    sched = {"auto": 0, "fused": 1, "three_phase": 2}[args.schedule]
+    sched = gtr_gla.SCHEDULES[args.schedule]
 
     q, k, v, g = make_workload_inputs(w, seed=rank, device=f"cuda:{dev}")
     out = torch.empty((w.B, w.N, w.heads, w.d_v), dtype=torch.float16, device=f"cuda:{dev}")
@@ -257,7 +257,7 @@ def main():
     per_launch_ms = ms / args.steps
     dominant = "forward step"
     phase_ms = None
-    if sched == 2 or (sched == 0 and launches > args.steps):
+    if sched in (2, 3):
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
         dominant = max(phase_ms, key=phase_ms.get)
         per_launch_ms = phase_ms[dominant]

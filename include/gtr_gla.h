@@ -79,9 +79,10 @@ typedef enum {
 } gtr_status_t;
 
 typedef enum {
-    GTR_SCHED_AUTO = 0,        /* library choice (currently the fused kernel when built) */
-    GTR_SCHED_FUSED = 1,       /* one kernel: summaries, chained boundary states, outputs */
-    GTR_SCHED_THREE_PHASE = 2  /* chunk_summary -> boundary_scan -> chunk_output */
+    GTR_SCHED_AUTO = 0,             /* library choice: the fused kernel */
+    GTR_SCHED_FUSED = 1,            /* one kernel: summaries, chained boundary states, outputs */
+    GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output (tensor cores) */
+    GTR_SCHED_THREE_PHASE_SIMT = 3  /* the same three phases on CUDA cores only (comparison) */
 } gtr_schedule_t;
 
 /* The GLA forward over all B*heads sequences (see the operation above).
@@ -179,6 +180,18 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k
  * word of the current device: GTR_OK, or GTR_ERR_TIMEOUT if a bounded wait
  * inside a kernel gave up since the last query. */
 gtr_status_t gtr_gla_get_last_device_status(void *stream);
+
+/* Test hook for the bounded wait of the fused schedule: runs
+ * gtr_gla_forward_ex(..., GTR_SCHED_FUSED, ...) except that the tile of
+ * sequence hold_seq (= b*heads + h), chunk hold_chunk never publishes its
+ * boundary state, and each wait gives up after spin_limit polls (> 0).  The
+ * successor tile then times out, records GTR_ERR_TIMEOUT in the device status
+ * word (read it with gtr_gla_get_last_device_status) and the kernel still
+ * finishes; its output is not meaningful.  hold_seq = -1 disables the hold. */
+gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const void *v, const float *g,
+                                         int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                         int direction, int chunk, int hold_seq, int hold_chunk,
+                                         long long spin_limit, void *out, void *stream);
 
 /* Frees every internal workspace of every device (synchronises each device
  * that has one).  Later calls allocate again on demand. */

@@ -10,6 +10,7 @@
 #include <utility>
 
 #include "gla_common.cuh"
+#include "gla_tc.cuh"
 
 namespace gtr {
 
@@ -70,20 +71,33 @@ size_t tok_bytes(const Geom &g, int d, size_t elem) {
     return (size_t)g.B * g.N * g.heads * d * elem;
 }
 
-// Internal workspace: one grow-only device buffer per (device, stream).
+// Internal workspaces: one grow-only, zero-initialised device buffer per
+// (device, stream, kind).  Kinds keep the schedules apart: the fused
+// kernel's control words must never be overwritten by another schedule.
+enum WsKind { WS_THREE_PHASE = 0, WS_FUSED = 1, WS_STAGING = 2, WS_STATUS = 3 };
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
 };
+struct WsKey {
+    int dev;
+    cudaStream_t st;
+    int kind;
+    bool operator<(const WsKey &o) const {
+        if (dev != o.dev) return dev < o.dev;
+        if (st != o.st) return st < o.st;
+        return kind < o.kind;
+    }
+};
 std::mutex g_ws_mu;
-std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<WsKey, Workspace> g_ws;
 
-gtr_status_t get_workspace(size_t bytes, cudaStream_t st, void **out) {
+gtr_status_t get_workspace(size_t bytes, cudaStream_t st, void **out, int kind = WS_THREE_PHASE) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(g_ws_mu);
-    Workspace &w = g_ws[{dev, st}];
+    Workspace &w = g_ws[WsKey{dev, kind == WS_STATUS ? nullptr : st, kind}];
     if (w.bytes < bytes) {
         if (w.ptr) {
             e = cudaStreamSynchronize(st);
@@ -115,8 +129,71 @@ size_t three_phase_ws(const Geom &g) {
            align256(nseq * g.nc * g.dk * sizeof(float));
 }
 
+// Fused kernel: control words (ticket, exit count, one flag per sequence)
+// then a two-slot ring of boundary states per sequence.
+size_t fused_ctrl_bytes(const Geom &g) { return align256(((size_t)g.B * g.heads + 2) * sizeof(int)); }
+size_t fused_ws(const Geom &g) {
+    return fused_ctrl_bytes(g) + (size_t)g.B * g.heads * 2 * g.dk * g.dv * sizeof(float);
+}
+
+// Device status word of the current device (zeroed at creation).
+gtr_status_t status_word(unsigned **out) {
+    void *p = nullptr;
+    gtr_status_t s = get_workspace(256, nullptr, &p, WS_STATUS);
+    *out = static_cast<unsigned *>(p);
+    return s;
+}
+
+constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
+
+TcArgs make_args(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo) {
+    TcArgs a;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.geo = geo;
+    a.dS = nullptr; a.gamma = nullptr; a.S_enter = nullptr; a.out = nullptr;
+    a.ctrl = nullptr; a.ring = nullptr; a.status = nullptr;
+    a.spin_limit = kSpinLimit; a.hold_seq = -1; a.hold_chunk = -1;
+    return a;
+}
+
+gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const float *g,
+                       const Geom &geo, __half *out, cudaStream_t st, int hold_seq = -1,
+                       int hold_chunk = -1, long long spin_limit = kSpinLimit) {
+    void *ws = nullptr;
+    gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
+    if (s != GTR_OK) return s;
+    unsigned *status = nullptr;
+    if ((s = status_word(&status)) != GTR_OK) return s;
+    TcArgs a = make_args(q, k, v, g, geo);
+    a.out = out;
+    a.ctrl = static_cast<int *>(ws);
+    a.ring = reinterpret_cast<float *>(static_cast<char *>(ws) + fused_ctrl_bytes(geo));
+    a.status = status;
+    a.spin_limit = spin_limit;
+    a.hold_seq = hold_seq;
+    a.hold_chunk = hold_chunk;
+    cudaError_t e = launch_tc(a, TC_FUSED, st);
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
+}
+
+cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
+                       float *gamma, cudaStream_t st) {
+    TcArgs a = make_args(nullptr, k, v, g, geo);
+    a.dS = dS;
+    a.gamma = gamma;
+    return launch_tc(a, TC_SUMMARY, st);
+}
+
+cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const float *g,
+                      const float *S_enter, const Geom &geo, __half *out, cudaStream_t st) {
+    TcArgs a = make_args(q, k, v, g, geo);
+    a.S_enter = S_enter;
+    a.out = out;
+    return launch_tc(a, TC_OUTPUT, st);
+}
+
+// Three-phase schedule; `simt` selects the CUDA-core summary/output kernels.
 gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, const float *g,
-                             const Geom &geo, __half *out, cudaStream_t st) {
+                             const Geom &geo, __half *out, cudaStream_t st, bool simt) {
     void *ws = nullptr;
     gtr_status_t s = get_workspace(three_phase_ws(geo), st, &ws);
     if (s != GTR_OK) return s;
@@ -124,11 +201,12 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     float *dS = static_cast<float *>(ws);
     float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                              align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
-    cudaError_t e = launch_summary_v0(k, v, g, geo, dS, gamma, st);
+    cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
+                         : summary_tc(k, v, g, geo, dS, gamma, st);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     e = launch_scan_v0(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, st);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
-    e = launch_output_v0(q, k, v, g, dS, geo, out, st);
+    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
     return GTR_OK;
 }
@@ -141,7 +219,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     bool empty = false;
     gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
     if (s != GTR_OK) return s;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE)
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE_SIMT)
         return fail(GTR_ERR_INVALID_ARG, "bad schedule%s");
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out))
@@ -152,8 +230,12 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
         return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
     if (empty) return GTR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    return run_three_phase(static_cast<const __half *>(q), static_cast<const __half *>(k),
-                           static_cast<const __half *>(v), g, geo, static_cast<__half *>(out), st);
+    const __half *hq = static_cast<const __half *>(q), *hk = static_cast<const __half *>(k);
+    const __half *hv = static_cast<const __half *>(v);
+    __half *ho = static_cast<__half *>(out);
+    if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
+    if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
+    return run_fused(hq, hk, hv, g, geo, ho, st);
 }
 
 }  // namespace
@@ -199,10 +281,7 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
         size_t need = 2 * bq + 2 * bv + bg;
         std::lock_guard<std::mutex> lk(g_ws_mu);
-        // distinct key: the stream handle with its lowest bit set can never
-        // be a real stream handle (those are at least 8-byte aligned)
-        cudaStream_t key = reinterpret_cast<cudaStream_t>(reinterpret_cast<uintptr_t>(st) | 1u);
-        Workspace &w = g_ws[{dev, key}];
+        Workspace &w = g_ws[WsKey{dev, st, WS_STAGING}];
         if (w.bytes < need) {
             if (w.ptr) {
                 e = cudaStreamSynchronize(st);
@@ -257,8 +336,8 @@ gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g,
         if (overlap(rs, r) || overlap(rg, r)) return fail(GTR_ERR_ALIAS, "an output overlaps an input%s");
     if (overlap(rs, rg)) return fail(GTR_ERR_ALIAS, "dS overlaps gamma%s");
     if (empty) return GTR_OK;
-    cudaError_t e = launch_summary_v0(static_cast<const __half *>(k), static_cast<const __half *>(v),
-                                      g, geo, dS, gamma, static_cast<cudaStream_t>(stream));
+    cudaError_t e = summary_tc(static_cast<const __half *>(k), static_cast<const __half *>(v), g, geo,
+                               dS, gamma, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk summary launch");
 }
 
@@ -306,9 +385,9 @@ gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, c
     for (const Range &r : in)
         if (overlap(ro, r)) return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
     if (empty) return GTR_OK;
-    cudaError_t e = launch_output_v0(static_cast<const __half *>(q), static_cast<const __half *>(k),
-                                     static_cast<const __half *>(v), g, S_enter, geo,
-                                     static_cast<__half *>(out), static_cast<cudaStream_t>(stream));
+    cudaError_t e = output_tc(static_cast<const __half *>(q), static_cast<const __half *>(k),
+                              static_cast<const __half *>(v), g, S_enter, geo, static_cast<__half *>(out),
+                              static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk output launch");
 }
 
@@ -317,14 +396,44 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k
     Geom geo;
     bool empty = false;
     if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return 0;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE || empty) return 0;
-    return three_phase_ws(geo);
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE_SIMT || empty) return 0;
+    if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT)
+        return three_phase_ws(geo);
+    return fused_ws(geo);
 }
 
 gtr_status_t gtr_gla_get_last_device_status(void *stream) {
+    t_err[0] = '\0';
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    unsigned *word = nullptr;
+    gtr_status_t s = status_word(&word);
+    if (s != GTR_OK) return s;
+    unsigned v = 0;
+    if ((e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+        return cuda_fail(e, "status read");
+    if (v != 0) {
+        if ((e = cudaMemset(word, 0, sizeof v)) != cudaSuccess) return cuda_fail(e, "status reset");
+        return fail(GTR_ERR_TIMEOUT, "a bounded device wait gave up%s");
+    }
     return GTR_OK;
+}
+
+gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const void *v, const float *g,
+                                         int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                         int direction, int chunk, int hold_seq, int hold_chunk,
+                                         long long spin_limit, void *out, void *stream) {
+    t_err[0] = '\0';
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (spin_limit < 1) return fail(GTR_ERR_INVALID_ARG, "spin_limit must be positive%s");
+    if (empty) return GTR_OK;
+    return run_fused(static_cast<const __half *>(q), static_cast<const __half *>(k),
+                     static_cast<const __half *>(v), g, geo, static_cast<__half *>(out),
+                     static_cast<cudaStream_t>(stream), hold_seq, hold_chunk, spin_limit);
 }
 
 gtr_status_t gtr_gla_release_workspace(void) {
@@ -333,7 +442,7 @@ gtr_status_t gtr_gla_release_workspace(void) {
     cudaGetDevice(&cur);
     for (auto &kv : g_ws) {
         if (kv.second.ptr) {
-            cudaSetDevice(kv.first.first);
+            cudaSetDevice(kv.first.dev);
             cudaDeviceSynchronize();
             cudaFree(kv.second.ptr);
         }

@@ -28,7 +28,7 @@ STATUS_NAMES = {
     7: "GTR_ERR_OOM",
 }
 DIRECTIONS = {"l2r": 0, "r2l": 1, "t2b": 2, "b2t": 3}
-SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2}
+SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3}
 
 # Every symbol include/gtr_gla.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -43,6 +43,8 @@ SIGNATURES = {
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gtr_gla_get_last_device_status": (_I, [_P]),
+    "gtr_gla_debug_forward_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                         ctypes.c_longlong, _P, _P]),
     "gtr_gla_release_workspace": (_I, []),
     "gtr_gla_status_string": (ctypes.c_char_p, [_I]),
     "gtr_gla_last_error": (ctypes.c_char_p, []),
@@ -159,6 +161,14 @@ def gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule=
 
 def gtr_gla_get_last_device_status(stream=None) -> int:
     return load().gtr_gla_get_last_device_status(_stream(stream))
+
+
+def gtr_gla_debug_forward_fused(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
+                                hold_seq, hold_chunk, spin_limit, out, stream=None) -> int:
+    return load().gtr_gla_debug_forward_fused(_addr(q), _addr(k), _addr(v), _addr(g), B, heads,
+                                              grid_h, grid_w, d_k, d_v, _dir(direction), chunk,
+                                              hold_seq, hold_chunk, spin_limit, _addr(out),
+                                              _stream(stream))
 
 
 def gtr_gla_release_workspace() -> int:

@@ -15,7 +15,7 @@ from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, s
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["auto", "three_phase"]
+SCHEDULES = ["fused", "three_phase", "three_phase_simt"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -107,12 +107,13 @@ def test_phases_against_oracle_intermediates(oracle_mod):
     gtr_gla.check(gtr_gla.gtr_gla_chunk_summary(k, v, g, B, heads, H, W, dk, dv, direction, chunk,
                                                 dS, gamma))
     torch.cuda.synchronize()
-    compare(dS, ref_dS, tol=1e-5)
+    # fp16 tensor-core operands: the summary carries fp16 rounding of k*decay
+    compare(dS, ref_dS, tol=2e-3)
     compare(gamma, ref_gamma, tol=1e-5)
     Se = torch.empty_like(dS)
     gtr_gla.check(gtr_gla.gtr_gla_boundary_scan(dS, gamma, B, heads, nc, dk, dv, Se))
     torch.cuda.synchronize()
-    compare(Se, ref_Se, tol=1e-5)
+    compare(Se, ref_Se, tol=2e-3)
     # in place
     dS2 = dS.clone()
     gtr_gla.check(gtr_gla.gtr_gla_boundary_scan(dS2, gamma, B, heads, nc, dk, dv, dS2))
@@ -217,4 +218,40 @@ def test_empty_and_streams():
     s.synchronize()
     o2 = run_forward(q, k, v, g, 4, 4, 0, 16)
     assert torch.equal(o1, o2)
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0
+
+
+def test_fused_repeated_calls_reset_control_words(oracle_mod):
+    """The fused kernel resets its ticket and flags itself: back-to-back
+    calls, interleaved with the three-phase schedule on the same stream,
+    all stay correct."""
+    H, W, heads = 24, 24, 4
+    for i in range(4):
+        q, k, v, g = gpu_inputs(2, H, W, heads, 64, 64, seed=300 + i)
+        out = run_forward(q, k, v, g, H, W, i % 4, 64, "fused")
+        compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, i % 4))
+        run_forward(q, k, v, g, H, W, i % 4, 64, "three_phase")
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0
+
+
+def test_fused_bounded_wait_times_out_cleanly(oracle_mod):
+    """A tile that never publishes its state: the successor's wait gives up
+    after the spin limit, the status word reports GTR_ERR_TIMEOUT, the
+    kernel finishes, and the next call is correct again."""
+    H, W, heads = 8, 8, 2
+    q, k, v, g = gpu_inputs(1, H, W, heads, 64, 64, seed=9)
+    out = torch.zeros_like(v)
+    st = gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, 64, 64, 0, 16,
+                                             1, 1, 2000, out)
+    assert st == 0
+    assert gtr_gla.gtr_gla_get_last_device_status() == 6  # GTR_ERR_TIMEOUT
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0  # cleared by the read
+    out2 = run_forward(q, k, v, g, H, W, 0, 16, "fused")
+    compare(out2, oracle_full(oracle_mod, q, k, v, g, H, W, 0))
+    # the hook with no hold changes nothing
+    out3 = torch.zeros_like(v)
+    assert gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, 64, 64, 0, 16,
+                                               -1, -1, 1 << 22, out3) == 0
+    torch.cuda.synchronize()
+    assert torch.equal(out3, out2)
     assert gtr_gla.gtr_gla_get_last_device_status() == 0
