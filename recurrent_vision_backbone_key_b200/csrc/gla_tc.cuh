@@ -17,20 +17,20 @@
 //             between tiles; the wait is bounded).
 //
 // Numerics (fp16 tensor-core operands, fp32 accumulation):
-//   Inside a chunk the tokens are split into sub-chunks of 16.  With beta_t
-//   the inclusive prefix sum of g inside the sub-chunk (per key dimension),
-//     qs_t = q~_t exp(beta_t)               (<= |q~_t|)
-//     ke_s = k_s exp(beta_end - beta_s)     (<= |k_s|)
-//     qe_t = q~_t exp(b_t)                  (b: prefix sum from the chunk start)
-//   a local state L runs over the sub-chunks of the chunk from zero,
-//     L_{u+1} = diag(exp(beta_end,u)) L_u + ke_u^T V_u,
-//   so every factor that meets an fp16 operand is at most one; only the
-//   16 x 16 diagonal blocks need exp(beta_t - beta_s) directly.  Those use a
-//   reference point in the middle of the sub-chunk (factors within e^{+-R},
-//   fp16 tensor-core product) when R <= kDiagRange, and exact per-pair
-//   exponentials in fp32 otherwise.  Then
-//     o_t = qs_t L_u + sum_{s<=t in u} A_ts v_s + qe_t S_enter,
-//     S_leave = diag(exp(b_last)) S_enter + L_last.
+//   The chunk's tokens form sub-chunks of 16.  Per key dimension, with
+//   a_t = exp(g_t), P_t = a_0..a_t (decay since the sub-chunk start) and
+//   Suf_t = a_{t+1}..a_15 (decay to the sub-chunk end):
+//     qs_t = q~_t P_t      ke_s = k_s Suf_s      (both <= the raw operand)
+//   A local state runs over the sub-chunks of the chunk from zero,
+//     L_{u+1} = diag(P_15,u) L_u + ke_u^T V_u,
+//   so every factor that meets an fp16 operand is at most one.  Only the
+//   16 x 16 diagonal blocks need exp(b_t - b_s) directly: when the decay
+//   over the sub-chunk is at most kDiagRange nats they use the reference
+//   token 7 (qd = qs / P_7, kd = ke / Suf_7, factors within e^{+-kDiagRange},
+//   fp16 tensor-core product); otherwise exact per-pair exponentials in fp32.
+//   Then, with E_u the decay from the chunk start to sub-chunk u,
+//     o_t = qs_t L_u + sum_{s<=t in u} A_ts v_s + (qs_t E_u) S_enter,
+//     S_leave = diag(gamma_c) S_enter + L_last.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -42,9 +42,11 @@ namespace gtr {
 
 enum TcMode : int { TC_SUMMARY = 0, TC_OUTPUT = 1, TC_FUSED = 2 };
 
-// Largest within-sub-chunk decay (natural-log units, either side of the
-// reference point) for which the diagonal block uses fp16 factors.
-constexpr float kDiagRange = 6.0f;
+// Largest decay over a 16-token sub-chunk (nats, either sign) for which the
+// diagonal block uses fp16 factors around the reference token.
+constexpr float kDiagRange = 5.0f;
+// Largest |q~| or |k| for that path (keeps e^{kDiagRange} * value in fp16).
+constexpr float kDiagMaxAbs = 64.0f;
 
 struct TcArgs {
     const __half *q, *k, *v;
@@ -71,9 +73,8 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool fu
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
                  "r"(full ? 16 : 0));
 }
-__device__ __forceinline__ void cp_async_commit_wait() {
-    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void *p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
@@ -98,6 +99,14 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+__device__ __forceinline__ float2 unpack_h2(uint32_t x) {
+    return __half22float2(*reinterpret_cast<__half2 *>(&x));
+}
+// Packed fp16 pair times a packed fp16 pair.
+__device__ __forceinline__ uint32_t hmul2u(uint32_t x, uint32_t s) {
+    __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&x), *reinterpret_cast<__half2 *>(&s));
+    return *reinterpret_cast<uint32_t *>(&r);
 }
 
 // 2^x with the MUFU approximation (flushes tiny results to zero).
@@ -126,27 +135,25 @@ struct TcLayout {
     static constexpr int LDA = 24;      // 16x16 diagonal block rows (halves)
     static constexpr int NW = DV / 16;  // warps: one 16-wide value slice each
     static constexpr int NT = NW * 32;
-    // byte offsets for a chunk of C tokens
-    __host__ __device__ static size_t q(int) { return 0; }
-    __host__ __device__ static size_t k(int C) { return q(C) + (size_t)C * LDK * 2; }
-    __host__ __device__ static size_t v(int C) { return k(C) + (size_t)C * LDK * 2; }
-    __host__ __device__ static size_t g(int C) { return v(C) + (size_t)C * LDV * 2; }
-    __host__ __device__ static size_t qd(int C) { return g(C) + (size_t)C * DK * 4; }
-    __host__ __device__ static size_t kd(int C) { return qd(C) + (size_t)C * LDK * 2; }
-    __host__ __device__ static size_t a(int C) { return kd(C) + (size_t)C * LDK * 2; }
-    __host__ __device__ static size_t bend(int C) { return a(C) + (size_t)(C / 16) * 16 * LDA * 2; }
-    __host__ __device__ static size_t gu(int C) { return bend(C) + (size_t)(C / 16) * DK * 4; }
-    __host__ __device__ static size_t eb(int C) { return gu(C) + (size_t)(C / 16) * DK * 4; }
-    __host__ __device__ static size_t gc(int C) { return eb(C) + (size_t)(C / 16) * DK * 4; }
-    __host__ __device__ static size_t flags(int C) { return gc(C) + (size_t)DK * 4; }
-    // output staging: the qd/kd region when it is large enough, else its own
-    __host__ __device__ static bool out_alias(int C) { return (size_t)C * LDV <= (size_t)2 * C * LDK; }
-    __host__ __device__ static size_t out(int C) { return out_alias(C) ? qd(C) : flags(C) + 64; }
-    __host__ __device__ static size_t bytes(int C) {
-        size_t end = flags(C) + 64;
-        if (!out_alias(C)) end += (size_t)C * LDV * 2;
-        return end;
+    // byte offsets for a chunk of C tokens (nsub = C/16 sub-chunks)
+    __host__ __device__ static size_t q(int) { return 0; }                                 // qs fp16 [C][LDK]
+    __host__ __device__ static size_t k(int C) { return q(C) + (size_t)C * LDK * 2; }      // ke fp16 [C][LDK]
+    __host__ __device__ static size_t v(int C) { return k(C) + (size_t)C * LDK * 2; }      // v  fp16 [C][LDV]
+    __host__ __device__ static size_t a(int C) { return v(C) + (size_t)C * LDV * 2; }      // A  fp16 [nsub][16][LDA]
+    __host__ __device__ static size_t gu(int C) { return a(C) + (size_t)(C / 16) * 16 * LDA * 2; }  // P_15 per (u,d)
+    __host__ __device__ static size_t rp(int C) { return gu(C) + (size_t)(C / 16) * DK * 4; }  // 1/P_7 (fp16)
+    __host__ __device__ static size_t rs(int C) { return rp(C) + (size_t)(C / 16) * DK * 2; }  // 1/Suf_7 (fp16)
+    __host__ __device__ static size_t eb(int C) { return rs(C) + (size_t)(C / 16) * DK * 2; }  // E_u (fp16)
+    __host__ __device__ static size_t gc(int C) { return eb(C) + (size_t)(C / 16) * DK * 2; }  // gamma_c
+    __host__ __device__ static size_t row(int C) { return gc(C) + (size_t)DK * 4; }            // token-head row index
+    __host__ __device__ static size_t flags(int C) { return row(C) + (size_t)C * 8; }
+    // scratch: output staging, or the exact diagonal path's raw operands
+    __host__ __device__ static size_t scratch(int C) { return flags(C) + 64; }
+    __host__ __device__ static size_t scratch_bytes(int C) {
+        size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8;
+        return o > e ? o : e;
     }
+    __host__ __device__ static size_t bytes(int C) { return scratch(C) + scratch_bytes(C); }
 };
 
 // The last fused tile to finish resets the ticket, the exit count and the
@@ -175,7 +182,7 @@ template <int DK, int DV, int MODE>
 __global__ void __launch_bounds__(TcLayout<DK, DV>::NT)
 gla_tc_kernel(const TcArgs args) {
     using Lay = TcLayout<DK, DV>;
-    constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT;
+    constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
     extern __shared__ __align__(128) unsigned char smem[];
     const Geom &geo = args.geo;
@@ -186,16 +193,15 @@ gla_tc_kernel(const TcArgs args) {
     __half *sQ = reinterpret_cast<__half *>(smem + Lay::q(C));
     __half *sK = reinterpret_cast<__half *>(smem + Lay::k(C));
     __half *sV = reinterpret_cast<__half *>(smem + Lay::v(C));
-    float *sG = reinterpret_cast<float *>(smem + Lay::g(C));
-    __half *sQD = reinterpret_cast<__half *>(smem + Lay::qd(C));
-    __half *sKD = reinterpret_cast<__half *>(smem + Lay::kd(C));
     __half *sA = reinterpret_cast<__half *>(smem + Lay::a(C));
-    float *sBend = reinterpret_cast<float *>(smem + Lay::bend(C));
     float *sGu = reinterpret_cast<float *>(smem + Lay::gu(C));
-    float *sEb = reinterpret_cast<float *>(smem + Lay::eb(C));
+    __half *sRp = reinterpret_cast<__half *>(smem + Lay::rp(C));
+    __half *sRs = reinterpret_cast<__half *>(smem + Lay::rs(C));
+    __half *sEb = reinterpret_cast<__half *>(smem + Lay::eb(C));
     float *sGc = reinterpret_cast<float *>(smem + Lay::gc(C));
-    int *sFlags = reinterpret_cast<int *>(smem + Lay::flags(C));  // [0..3] diag range bits, [4..7] overflow, [8] tile
-    __half *sOut = reinterpret_cast<__half *>(smem + Lay::out(C));
+    int64_t *sRow = reinterpret_cast<int64_t *>(smem + Lay::row(C));  // (b*N + p)*heads + h, or -1
+    int *sFlags = reinterpret_cast<int *>(smem + Lay::flags(C));  // [0..3] exact-path sub-chunks, [8] tile, [9] last
+    unsigned char *sScr = smem + Lay::scratch(C);
 
     // ------------------------------------------------ which tile
     const int nseq = geo.B * geo.heads;
@@ -205,20 +211,18 @@ gla_tc_kernel(const TcArgs args) {
         if (tid == 0) sFlags[8] = atomicAdd(&args.ctrl[0], 1);
         __syncthreads();
         tile = sFlags[8];
+        // A ticket past the grid can only come from control words left behind
+        // by an aborted launch: record it and only take part in the reset.
+        if (tile >= geo.nc * nseq) {
+            if (tid == 0) atomicOr(args.status, 6u);
+            fused_finish(args, nseq, sFlags, NT);
+            return;
+        }
     } else {
         tile = blockIdx.x;
-        __syncthreads();
     }
-    // A ticket past the grid can only come from control words left behind by
-    // an aborted launch: record it and only take part in the reset below.
-    if (MODE == TC_FUSED && tile >= geo.nc * nseq) {
-        if (tid == 0) atomicOr(args.status, 6u);
-        fused_finish(args, nseq, sFlags, NT);
-        return;
-    }
-    // FUSED: chunk-major tickets; other modes: sequence-major blocks
     int c, seq;
-    if (MODE == TC_FUSED) {
+    if (MODE == TC_FUSED) {  // chunk-major: chunk c of every sequence before chunk c+1
         c = tile / nseq;
         seq = tile - c * nseq;
     } else {
@@ -229,165 +233,176 @@ gla_tc_kernel(const TcArgs args) {
     const int t0 = c * C;
     const int len = min(C, geo.N - t0);
     const float qscale = rsqrtf((float)DK);
+    // ------------------------------------------------ S0: the scan-order row table
+    // Row t of the chunk is token-head row (b*N + p)*heads + h of every
+    // [B][N][heads][d] tensor; -1 past the end of the sequence.
+    for (int t = tid; t < C; t += NT)
+        sRow[t] = (t < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
+                            : (int64_t)-1;
+    __syncthreads();
 
-    // ------------------------------------------------ A: stage the chunk
+    // ------------------------------------------------ S1: stage v, prepare qs / ke
     {
-        constexpr int QCH = DK / 8, VCH = DV / 8, GCH = DK / 4;  // 16-byte pieces per row
-        for (int idx = tid; idx < C * (2 * QCH + VCH + GCH); idx += NT) {
-            int t, j, which;
-            if (idx < C * QCH) { which = 0; t = idx / QCH; j = idx - t * QCH; }
-            else if (idx < 2 * C * QCH) { which = 1; int r = idx - C * QCH; t = r / QCH; j = r - t * QCH; }
-            else if (idx < C * (2 * QCH + VCH)) { which = 2; int r = idx - 2 * C * QCH; t = r / VCH; j = r - t * VCH; }
-            else { which = 3; int r = idx - C * (2 * QCH + VCH); t = r / GCH; j = r - t * GCH; }
-            const bool in = t < len;
-            const int p = in ? scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N) : 0;
-            if (MODE == TC_SUMMARY && which == 0) continue;  // q unused
-            switch (which) {
-            case 0: cp_async16(sQ + t * LDK + j * 8, args.q + tok_offset(geo, b, p, h, DK) + j * 8, in); break;
-            case 1: cp_async16(sK + t * LDK + j * 8, args.k + tok_offset(geo, b, p, h, DK) + j * 8, in); break;
-            case 2: cp_async16(sV + t * LDV + j * 8, args.v + tok_offset(geo, b, p, h, DV) + j * 8, in); break;
-            default: cp_async16(sG + t * DK + j * 4, args.g + tok_offset(geo, b, p, h, DK) + j * 4, in); break;
-            }
+        constexpr int VCH = DV / 8;
+        for (int idx = tid; idx < C * VCH; idx += NT) {
+            const int t = idx / VCH, j = idx - t * VCH;
+            const int64_t r = sRow[t];
+            cp_async16(sV + t * LDV + j * 8, args.v + (r < 0 ? 0 : r) * DV + j * 8, r >= 0);
         }
-        cp_async_commit_wait();
-        __syncthreads();
+        cp_async_commit();
     }
-
-    // ------------------------------------------------ B: in-sub-chunk prefix sums (log2 units)
-    for (int task = tid; task < DK * nsub; task += NT) {
-        const int d = task % DK, u = task / DK;
-        float acc = 0.f, b7 = 0.f, b0 = 0.f;
+    for (int task = tid; task < (DK / 2) * nsub; task += NT) {
+        const int dp = task % (DK / 2), u = task / (DK / 2);
+        const int d0 = 2 * dp;
+        __half2 qv[16], kv[16];
+        float2 av[16];
+#pragma unroll
         for (int t = 0; t < 16; ++t) {
-            float *p = sG + (16 * u + t) * DK + d;
-            acc += *p * kLog2e;
-            *p = acc;
-            if (t == 0) b0 = acc;
-            if (t == 7) b7 = acc;
-        }
-        sBend[u * DK + d] = acc;
-        float r = fmaxf(fmaxf(b0 - b7, b7 - acc), 0.f);  // decay either side of the reference
-        atomicMax(&sFlags[u], __float_as_int(r));
-    }
-    __syncthreads();
-    for (int task = tid; task < DK * nsub; task += NT) {
-        const int d = task % DK, u = task / DK;
-        float base = 0.f, tot = 0.f;
-        for (int w = 0; w < nsub; ++w) {
-            float be = sBend[w * DK + d];
-            if (w < u) base += be;
-            tot += be;
-        }
-        sGu[u * DK + d] = ex2(sBend[u * DK + d]);
-        sEb[u * DK + d] = ex2(base);
-        if (u == 0) sGc[d] = ex2(tot);
-    }
-    __syncthreads();
-
-    // ------------------------------------------------ C1: diagonal-block factors
-    // qd_t = q~_t 2^(beta_t - beta_7), kd_s = k_s 2^(beta_7 - beta_s) for the
-    // sub-chunks whose decay range allows fp16 factors; an fp16 overflow
-    // sends that sub-chunk to the exact path as well.
-    if (MODE != TC_SUMMARY) {
-        for (int task = tid; task < DK * nsub; task += NT) {
-            const int d = task % DK, u = task / DK;
-            if (!(__int_as_float(sFlags[u]) <= kDiagRange * kLog2e)) continue;
-            const float b7 = sG[(16 * u + 7) * DK + d];
-            bool ovf = false;
-            for (int t = 0; t < 16; ++t) {
-                const int row = 16 * u + t;
-                const float bt = sG[row * DK + d];
-                const __half hq = __float2half_rn(__half2float(sQ[row * LDK + d]) * qscale * ex2(bt - b7));
-                const __half hk = __float2half_rn(__half2float(sK[row * LDK + d]) * ex2(b7 - bt));
-                ovf |= __hisinf(hq) | __hisinf(hk);
-                sQD[row * LDK + d] = hq;
-                sKD[row * LDK + d] = hk;
-            }
-            if (ovf) sFlags[4 + u] = 1;
-        }
-        __syncthreads();
-
-        // ------------------------------------------------ D: diagonal 16x16 blocks
-        for (int u = warp; u < nsub; u += Lay::NW) {
-            const bool fast = __int_as_float(sFlags[u]) <= kDiagRange * kLog2e && sFlags[4 + u] == 0;
-            __half *Au = sA + u * 16 * LDA;
-            if (fast) {
-                float acc[2][4] = {};
-#pragma unroll
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    uint32_t af[4], bf[4];
-                    const int r = lane & 7, m = lane >> 3;
-                    ldsm_x4(af, sQD + (16 * u + r + 8 * (m & 1)) * LDK + 16 * kk + 8 * (m >> 1));
-                    ldsm_x4(bf, sKD + (16 * u + r + 8 * (m >> 1)) * LDK + 16 * kk + 8 * (m & 1));
-                    mma16816(acc[0], af, bf[0], bf[1]);
-                    mma16816(acc[1], af, bf[2], bf[3]);
-                }
-                const int tr = lane >> 2, tc = 2 * (lane & 3);
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-#pragma unroll
-                    for (int hlf = 0; hlf < 2; ++hlf) {
-                        const int t = tr + 8 * hlf;
-                        const int s0 = 8 * j + tc;
-                        const float x0 = (s0 <= t) ? acc[j][2 * hlf] : 0.f;
-                        const float x1 = (s0 + 1 <= t) ? acc[j][2 * hlf + 1] : 0.f;
-                        *reinterpret_cast<uint32_t *>(Au + t * LDA + s0) = pack_h2(x0, x1);
-                    }
-                }
+            const int64_t r = sRow[16 * u + t];
+            if (r >= 0) {
+                const int64_t o = r * DK + d0;
+                if (MODE != TC_SUMMARY) qv[t] = __ldg(reinterpret_cast<const __half2 *>(args.q + o));
+                kv[t] = __ldg(reinterpret_cast<const __half2 *>(args.k + o));
+                av[t] = __ldg(reinterpret_cast<const float2 *>(args.g + o));
             } else {
-                // exact: A_ts = sum_d q~_td k_sd 2^(beta_td - beta_sd) from the raw
-                // operands; lane -> one query t and eight keys s
-                const int t = lane >> 1, sb = 8 * (lane & 1);
-                float acc[8] = {};
-                for (int d = 0; d < DK; ++d) {
-                    const float qv = __half2float(sQ[(16 * u + t) * LDK + d]) * qscale;
-                    const float bt = sG[(16 * u + t) * DK + d];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const int s = sb + j;
-                        if (s <= t) {
-                            const float kv = __half2float(sK[(16 * u + s) * LDK + d]);
-                            acc[j] = fmaf(qv * kv, ex2(bt - sG[(16 * u + s) * DK + d]), acc[j]);
-                        }
-                    }
-                }
-#pragma unroll
-                for (int j = 0; j < 8; j += 2)
-                    *reinterpret_cast<uint32_t *>(Au + t * LDA + sb + j) = pack_h2(acc[j], acc[j + 1]);
+                qv[t] = __float2half2_rn(0.f); kv[t] = qv[t]; av[t] = make_float2(0.f, 0.f);
             }
         }
-        __syncthreads();
+        // forward: a_t = exp(g_t), P_t = prod a_0..a_t, qs_t = q~_t P_t
+        float2 P = make_float2(1.f, 1.f), P7 = P;
+        __half2 qmax = __float2half2_rn(0.f), kmax = qmax;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            av[t].x = ex2(av[t].x * kLog2e);
+            av[t].y = ex2(av[t].y * kLog2e);
+            P.x *= av[t].x;
+            P.y *= av[t].y;
+            if (t == 7) P7 = P;
+            if (MODE != TC_SUMMARY) {
+                qmax = __hmax2(qmax, __habs2(qv[t]));
+                *reinterpret_cast<__half2 *>(sQ + (16 * u + t) * LDK + d0) =
+                    __hmul2(qv[t], __floats2half2_rn(P.x * qscale, P.y * qscale));
+            }
+        }
+        // backward: Suf_t = prod a_{t+1}..a_15, ke_t = k_t Suf_t
+        float2 S = make_float2(1.f, 1.f), S7 = S;
+#pragma unroll
+        for (int t = 15; t >= 0; --t) {
+            if (t == 7) S7 = S;
+            kmax = __hmax2(kmax, __habs2(kv[t]));
+            *reinterpret_cast<__half2 *>(sK + (16 * u + t) * LDK + d0) = __hmul2(kv[t], __floats2half2_rn(S.x, S.y));
+            S.x *= av[t].x;
+            S.y *= av[t].y;
+        }
+        *reinterpret_cast<float2 *>(sGu + u * DK + d0) = P;
+        if (MODE != TC_SUMMARY) {
+            const float lo = 6.737947e-3f /* e^-5 */, hi = 148.41316f /* e^5 */;
+            const float2 qm = __half22float2(qmax), km = __half22float2(kmax);
+            const bool fast = P.x >= lo && P.y >= lo && P.x <= hi && P.y <= hi &&
+                              fmaxf(qm.x, qm.y) * qscale <= kDiagMaxAbs && fmaxf(km.x, km.y) <= kDiagMaxAbs;
+            if (!fast) sFlags[u] = 1;
+            *reinterpret_cast<__half2 *>(sRp + u * DK + d0) =
+                __floats2half2_rn(P7.x > 0.f ? 1.f / P7.x : 0.f, P7.y > 0.f ? 1.f / P7.y : 0.f);
+            *reinterpret_cast<__half2 *>(sRs + u * DK + d0) =
+                __floats2half2_rn(S7.x > 0.f ? 1.f / S7.x : 0.f, S7.y > 0.f ? 1.f / S7.y : 0.f);
+        }
+    }
+    cp_async_wait_all();
+    __syncthreads();
+
+    // ------------------------------------------------ S2: decay to each sub-chunk, chunk decay
+    for (int d = tid; d < DK; d += NT) {
+        float e = 1.f;
+        for (int u = 0; u < nsub; ++u) {
+            sEb[u * DK + d] = __float2half_rn(e);
+            e *= sGu[u * DK + d];
+        }
+        sGc[d] = e;
     }
 
-    // ------------------------------------------------ C2: qs, ke in place
-    for (int task = tid; task < DK * nsub; task += NT) {
-        const int d = task % DK, u = task / DK;
-        const float bend = sBend[u * DK + d];
-        for (int t = 0; t < 16; ++t) {
-            const int row = 16 * u + t;
-            const float bt = sG[row * DK + d];
-            if (MODE != TC_SUMMARY) {
-                const float qv = __half2float(sQ[row * LDK + d]) * qscale;
-                sQ[row * LDK + d] = __float2half_rn(qv * ex2(bt));
+    const int r8 = lane & 7, m4 = lane >> 3;
+    const int kc = 2 * (lane & 3);  // key column pair inside an 8-wide tile
+
+    // ------------------------------------------------ S3: diagonal 16x16 blocks
+    if (MODE != TC_SUMMARY) {
+        for (int u = warp; u < nsub; u += NW) {
+            if (sFlags[u]) continue;
+            float acc[2][4] = {};
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                uint32_t af[4], bf[4];
+                ldsm_x4(af, sQ + (16 * u + r8 + 8 * (m4 & 1)) * LDK + 16 * kk + 8 * (m4 >> 1));
+                ldsm_x4(bf, sK + (16 * u + r8 + 8 * (m4 >> 1)) * LDK + 16 * kk + 8 * (m4 & 1));
+                const uint32_t p0 = *reinterpret_cast<const uint32_t *>(sRp + u * DK + 16 * kk + kc);
+                const uint32_t p1 = *reinterpret_cast<const uint32_t *>(sRp + u * DK + 16 * kk + 8 + kc);
+                const uint32_t s0 = *reinterpret_cast<const uint32_t *>(sRs + u * DK + 16 * kk + kc);
+                const uint32_t s1 = *reinterpret_cast<const uint32_t *>(sRs + u * DK + 16 * kk + 8 + kc);
+                af[0] = hmul2u(af[0], p0); af[1] = hmul2u(af[1], p0);
+                af[2] = hmul2u(af[2], p1); af[3] = hmul2u(af[3], p1);
+                bf[0] = hmul2u(bf[0], s0); bf[2] = hmul2u(bf[2], s0);
+                bf[1] = hmul2u(bf[1], s1); bf[3] = hmul2u(bf[3], s1);
+                mma16816(acc[0], af, bf[0], bf[1]);
+                mma16816(acc[1], af, bf[2], bf[3]);
             }
-            const float kv = __half2float(sK[row * LDK + d]);
-            sK[row * LDK + d] = __float2half_rn(kv * ex2(bend - bt));
+            __half *Au = sA + u * 16 * LDA;
+            const int tr = lane >> 2;
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                for (int hlf = 0; hlf < 2; ++hlf) {
+                    const int t = tr + 8 * hlf;
+                    const int s0i = 8 * j + kc;
+                    const float x0 = (s0i <= t) ? acc[j][2 * hlf] : 0.f;
+                    const float x1 = (s0i + 1 <= t) ? acc[j][2 * hlf + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(Au + t * LDA + s0i) = pack_h2(x0, x1);
+                }
+            }
+        }
+        // Exact path, one flagged sub-chunk at a time by the whole CTA:
+        // A_ts = sum_d q~_td k_sd 2^(beta_td - beta_sd) with beta the in-sub-chunk
+        // prefix sum of g*log2(e), from the raw operands.
+        const int any_exact = sFlags[0] | sFlags[1] | sFlags[2] | sFlags[3];
+        if (any_exact) {
+            __half *xq = reinterpret_cast<__half *>(sScr);
+            __half *xk = xq + 16 * DK;
+            float *xb = reinterpret_cast<float *>(xk + 16 * DK);
+            for (int u = 0; u < nsub; ++u) {
+                if (!sFlags[u]) continue;
+                for (int idx = tid; idx < 16 * DK; idx += NT) {
+                    const int t = idx / DK, d = idx - t * DK;
+                    const int64_t r = sRow[16 * u + t];
+                    const int64_t o = (r < 0 ? 0 : r) * DK + d;
+                    xq[idx] = r >= 0 ? args.q[o] : __float2half(0.f);
+                    xk[idx] = r >= 0 ? args.k[o] : __float2half(0.f);
+                    xb[idx] = r >= 0 ? args.g[o] * kLog2e : 0.f;
+                }
+                __syncthreads();
+                for (int d = tid; d < DK; d += NT) {
+                    float acc = 0.f;
+                    for (int t = 0; t < 16; ++t) {
+                        acc += xb[t * DK + d];
+                        xb[t * DK + d] = acc;
+                    }
+                }
+                __syncthreads();
+                for (int pr = tid; pr < 256; pr += NT) {
+                    const int t = pr >> 4, s = pr & 15;
+                    float acc = 0.f;
+                    if (s <= t) {
+                        for (int d = 0; d < DK; ++d)
+                            acc = fmaf(__half2float(xq[t * DK + d]) * __half2float(xk[s * DK + d]),
+                                       ex2(xb[t * DK + d] - xb[s * DK + d]), acc);
+                        acc *= qscale;
+                    }
+                    sA[u * 16 * LDA + t * LDA + s] = __float2half_rn(acc);
+                }
+                __syncthreads();
+            }
         }
     }
     __syncthreads();
-    // qe_t = qs_t 2^(base_u) into the sQD region (the diagonal blocks are done with it)
-    if (MODE != TC_SUMMARY) {
-        for (int task = tid; task < DK * nsub; task += NT) {
-            const int d = task % DK, u = task / DK;
-            const float e = sEb[u * DK + d];
-            for (int t = 0; t < 16; ++t) {
-                const int row = 16 * u + t;
-                sQD[row * LDK + d] = __float2half_rn(__half2float(sQ[row * LDK + d]) * e);
-            }
-        }
-        // made visible to every warp by the barrier at the top of phase H
-    }
 
-    // ------------------------------------------------ F: local state over sub-chunks
+    // ------------------------------------------------ S4: local state over sub-chunks
     // Warp w owns value columns [16w, 16w+16).  L^T (16 x DK) lives in the
     // accumulator layout: Lt[n][0..3] covers key columns 8n..8n+7.
     const int v0 = 16 * warp;
@@ -400,8 +415,6 @@ gla_tc_kernel(const TcArgs args) {
 #pragma unroll
         for (int j = 0; j < 2; ++j) o[u][j][0] = o[u][j][1] = o[u][j][2] = o[u][j][3] = 0.f;
 
-    const int r8 = lane & 7, m4 = lane >> 3;
-    const int kc = 2 * (lane & 3);  // key column pair inside an 8-wide tile
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
         if (u >= nsub) break;
@@ -412,12 +425,10 @@ gla_tc_kernel(const TcArgs args) {
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     uint32_t af[4];
                     ldsm_x4(af, sQ + (16 * u + r8 + 8 * (m4 & 1)) * LDK + 16 * kk + 8 * (m4 >> 1));
-                    const uint32_t b00 = pack_h2(Lt[2 * kk][0], Lt[2 * kk][1]);
-                    const uint32_t b01 = pack_h2(Lt[2 * kk + 1][0], Lt[2 * kk + 1][1]);
-                    const uint32_t b10 = pack_h2(Lt[2 * kk][2], Lt[2 * kk][3]);
-                    const uint32_t b11 = pack_h2(Lt[2 * kk + 1][2], Lt[2 * kk + 1][3]);
-                    mma16816(o[u][0], af, b00, b01);
-                    mma16816(o[u][1], af, b10, b11);
+                    mma16816(o[u][0], af, pack_h2(Lt[2 * kk][0], Lt[2 * kk][1]),
+                             pack_h2(Lt[2 * kk + 1][0], Lt[2 * kk + 1][1]));
+                    mma16816(o[u][1], af, pack_h2(Lt[2 * kk][2], Lt[2 * kk][3]),
+                             pack_h2(Lt[2 * kk + 1][2], Lt[2 * kk + 1][3]));
                 }
             }
             // diagonal block: o_u += A_uu V_u
@@ -429,13 +440,13 @@ gla_tc_kernel(const TcArgs args) {
                 mma16816(o[u][1], af, bf[2], bf[3]);
             }
         }
-        // update: L = diag(gamma_u) L + V_u^T ke_u
+        // update: L = diag(P_15,u) L + V_u^T ke_u
         {
             const float *gu = sGu + u * DK;
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
-                const float g0 = gu[8 * n + kc], g1 = gu[8 * n + kc + 1];
-                Lt[n][0] *= g0; Lt[n][1] *= g1; Lt[n][2] *= g0; Lt[n][3] *= g1;
+                const float2 gg = *reinterpret_cast<const float2 *>(gu + 8 * n + kc);
+                Lt[n][0] *= gg.x; Lt[n][1] *= gg.y; Lt[n][2] *= gg.x; Lt[n][3] *= gg.y;
             }
             uint32_t af[4];
             // A = V^T (rows: value columns of this warp, cols: 16 tokens)
@@ -467,7 +478,7 @@ gla_tc_kernel(const TcArgs args) {
         return;
     }
 
-    // ------------------------------------------------ G: the state entering the chunk
+    // ------------------------------------------------ S5: the state entering the chunk
     float Se[KT][4];
     bool have_state = c > 0;
     if (MODE == TC_OUTPUT) {
@@ -514,43 +525,48 @@ gla_tc_kernel(const TcArgs args) {
                 args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
-                const float g0 = sGc[8 * n + kc], g1 = sGc[8 * n + kc + 1];
+                const float2 gg = *reinterpret_cast<const float2 *>(sGc + 8 * n + kc);
                 float4 x;
-                x.x = fmaf(g0, Se[n][0], Lt[n][0]);
-                x.y = fmaf(g1, Se[n][1], Lt[n][1]);
-                x.z = fmaf(g0, Se[n][2], Lt[n][2]);
-                x.w = fmaf(g1, Se[n][3], Lt[n][3]);
+                x.x = fmaf(gg.x, Se[n][0], Lt[n][0]);
+                x.y = fmaf(gg.y, Se[n][1], Lt[n][1]);
+                x.z = fmaf(gg.x, Se[n][2], Lt[n][2]);
+                x.w = fmaf(gg.y, Se[n][3], Lt[n][3]);
                 __stcg(dst + ((warp * KT + n) * 32 + lane), x);
             }
-            __threadfence();
             __syncthreads();
             if (tid == 0) st_release(&flags[seq], c + 1);
         }
     }
 
-    // ------------------------------------------------ H: readout of the entering state
-    __syncthreads();  // qe visible to every warp
+    // ------------------------------------------------ S6: readout of the entering state
+    // qe_t = qs_t E_u is formed in registers from the qs fragments.
     if (have_state) {
+        uint32_t Sb[KT][2];  // the entering state as fp16 B fragments
+#pragma unroll
+        for (int n = 0; n < KT; ++n) {
+            Sb[n][0] = pack_h2(Se[n][0], Se[n][1]);
+            Sb[n][1] = pack_h2(Se[n][2], Se[n][3]);
+        }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             if (u >= nsub) break;
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
                 uint32_t af[4];
-                ldsm_x4(af, sQD + (16 * u + r8 + 8 * (m4 & 1)) * LDK + 16 * kk + 8 * (m4 >> 1));
-                const uint32_t b00 = pack_h2(Se[2 * kk][0], Se[2 * kk][1]);
-                const uint32_t b01 = pack_h2(Se[2 * kk + 1][0], Se[2 * kk + 1][1]);
-                const uint32_t b10 = pack_h2(Se[2 * kk][2], Se[2 * kk][3]);
-                const uint32_t b11 = pack_h2(Se[2 * kk + 1][2], Se[2 * kk + 1][3]);
-                mma16816(o[u][0], af, b00, b01);
-                mma16816(o[u][1], af, b10, b11);
+                ldsm_x4(af, sQ + (16 * u + r8 + 8 * (m4 & 1)) * LDK + 16 * kk + 8 * (m4 >> 1));
+                const uint32_t e0 = *reinterpret_cast<const uint32_t *>(sEb + u * DK + 16 * kk + kc);
+                const uint32_t e1 = *reinterpret_cast<const uint32_t *>(sEb + u * DK + 16 * kk + 8 + kc);
+                af[0] = hmul2u(af[0], e0); af[1] = hmul2u(af[1], e0);
+                af[2] = hmul2u(af[2], e1); af[3] = hmul2u(af[3], e1);
+                mma16816(o[u][0], af, Sb[2 * kk][0], Sb[2 * kk + 1][0]);
+                mma16816(o[u][1], af, Sb[2 * kk][1], Sb[2 * kk + 1][1]);
             }
         }
     }
 
-    // ------------------------------------------------ I: store the outputs
-    __syncthreads();  // every warp is done reading sQD (the staging may alias it)
+    // ------------------------------------------------ S7: store the outputs
     {
+        __half *sOut = reinterpret_cast<__half *>(sScr);
         const int tr = lane >> 2;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -562,14 +578,11 @@ gla_tc_kernel(const TcArgs args) {
                 *reinterpret_cast<uint32_t *>(sOut + (16 * u + tr + 8) * LDV + col) = pack_h2(o[u][j][2], o[u][j][3]);
             }
         }
-    }
-    __syncthreads();
-    {
+        __syncthreads();
         constexpr int VCH = DV / 8;
         for (int idx = tid; idx < len * VCH; idx += NT) {
             const int t = idx / VCH, j = idx - t * VCH;
-            const int p = scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N);
-            *reinterpret_cast<int4 *>(args.out + tok_offset(geo, b, p, h, DV) + j * 8) =
+            *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
                 *reinterpret_cast<const int4 *>(sOut + t * LDV + j * 8);
         }
     }
