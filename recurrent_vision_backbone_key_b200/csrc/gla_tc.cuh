@@ -147,11 +147,13 @@ struct TcLayout {
     __host__ __device__ static size_t gc(int C) { return eb(C) + (size_t)(C / 16) * DK * 2; }  // gamma_c
     __host__ __device__ static size_t row(int C) { return gc(C) + (size_t)DK * 4; }            // token-head row index
     __host__ __device__ static size_t flags(int C) { return row(C) + (size_t)C * 8; }
-    // scratch: output staging, or the exact diagonal path's raw operands
+    // scratch, used in turn for the staged g rows (fp32 [C][DK]), the exact
+    // diagonal path's raw operands and the output staging
     __host__ __device__ static size_t scratch(int C) { return flags(C) + 64; }
     __host__ __device__ static size_t scratch_bytes(int C) {
-        size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8;
-        return o > e ? o : e;
+        size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8, gs = (size_t)C * DK * 4;
+        size_t m = o > e ? o : e;
+        return m > gs ? m : gs;
     }
     __host__ __device__ static size_t bytes(int C) { return scratch(C) + scratch_bytes(C); }
 };
@@ -241,15 +243,34 @@ gla_tc_kernel(const TcArgs args) {
                             : (int64_t)-1;
     __syncthreads();
 
-    // ------------------------------------------------ S1: stage v, prepare qs / ke
+    // ------------------------------------------------ S1: stage q, k, v, g; prepare qs / ke
+    // Every row of the chunk is requested at once (cp.async, 16 bytes per
+    // request, rows past the sequence end zero-filled), so the whole tile is
+    // in flight together; q and k land in the operand buffers and are turned
+    // into qs / ke in place, g lands in the scratch region.
+    float *sG = reinterpret_cast<float *>(sScr);
     {
-        constexpr int VCH = DV / 8;
+        constexpr int QCH = DK / 8, VCH = DV / 8, GCH = DK / 4;
         for (int idx = tid; idx < C * VCH; idx += NT) {
             const int t = idx / VCH, j = idx - t * VCH;
             const int64_t r = sRow[t];
             cp_async16(sV + t * LDV + j * 8, args.v + (r < 0 ? 0 : r) * DV + j * 8, r >= 0);
         }
+        for (int idx = tid; idx < C * QCH; idx += NT) {
+            const int t = idx / QCH, j = idx - t * QCH;
+            const int64_t r = sRow[t];
+            const int64_t o = (r < 0 ? 0 : r) * DK + j * 8;
+            if (MODE != TC_SUMMARY) cp_async16(sQ + t * LDK + j * 8, args.q + o, r >= 0);
+            cp_async16(sK + t * LDK + j * 8, args.k + o, r >= 0);
+        }
+        for (int idx = tid; idx < C * GCH; idx += NT) {
+            const int t = idx / GCH, j = idx - t * GCH;
+            const int64_t r = sRow[t];
+            cp_async16(sG + t * DK + j * 4, args.g + (r < 0 ? 0 : r) * DK + j * 4, r >= 0);
+        }
         cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
     }
     for (int task = tid; task < (DK / 2) * nsub; task += NT) {
         const int dp = task % (DK / 2), u = task / (DK / 2);
@@ -258,15 +279,10 @@ gla_tc_kernel(const TcArgs args) {
         float2 av[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-            const int64_t r = sRow[16 * u + t];
-            if (r >= 0) {
-                const int64_t o = r * DK + d0;
-                if (MODE != TC_SUMMARY) qv[t] = __ldg(reinterpret_cast<const __half2 *>(args.q + o));
-                kv[t] = __ldg(reinterpret_cast<const __half2 *>(args.k + o));
-                av[t] = __ldg(reinterpret_cast<const float2 *>(args.g + o));
-            } else {
-                qv[t] = __float2half2_rn(0.f); kv[t] = qv[t]; av[t] = make_float2(0.f, 0.f);
-            }
+            const int row = 16 * u + t;
+            if (MODE != TC_SUMMARY) qv[t] = *reinterpret_cast<const __half2 *>(sQ + row * LDK + d0);
+            kv[t] = *reinterpret_cast<const __half2 *>(sK + row * LDK + d0);
+            av[t] = *reinterpret_cast<const float2 *>(sG + row * DK + d0);
         }
         // forward: a_t = exp(g_t), P_t = prod a_0..a_t, qs_t = q~_t P_t
         float2 P = make_float2(1.f, 1.f), P7 = P;
@@ -307,7 +323,6 @@ gla_tc_kernel(const TcArgs args) {
                 __floats2half2_rn(S7.x > 0.f ? 1.f / S7.x : 0.f, S7.y > 0.f ? 1.f / S7.y : 0.f);
         }
     }
-    cp_async_wait_all();
     __syncthreads();
 
     // ------------------------------------------------ S2: decay to each sub-chunk, chunk decay
@@ -625,5 +640,6 @@ cudaError_t launch_tc_dk(const TcArgs &a, int mode, cudaStream_t st) {
 
 size_t tc_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_tc(const TcArgs &a, int mode, cudaStream_t st);
+
 
 }  // namespace gtr
