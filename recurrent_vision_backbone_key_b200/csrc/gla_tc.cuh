@@ -56,7 +56,7 @@ struct TcArgs {
     float *gamma;          // SUMMARY: [nseq][nc][dk]
     const float *S_enter;  // OUTPUT:  [nseq][nc][dk][dv]
     __half *out;           // OUTPUT / FUSED
-    int *ctrl;             // FUSED: [0] ticket, [1] exit count, then nseq flags
+    int *ctrl;             // FUSED: [0] ticket, [1] unused, then nseq flags; zeroed before each launch
     float *ring;           // FUSED: [nseq][2][dk*dv] fragment-ordered states
     unsigned *status;      // FUSED: device status word (GTR_ERR_TIMEOUT on a give-up)
     long long spin_limit;  // FUSED: polls before a wait gives up
@@ -158,26 +158,6 @@ struct TcLayout {
     __host__ __device__ static size_t bytes(int C) { return scratch(C) + scratch_bytes(C); }
 };
 
-// The last fused tile to finish resets the ticket, the exit count and the
-// flags, so the next launch starts from zero without a memset.  Called by
-// every thread of a CTA (uniform branch).
-__device__ __forceinline__ void fused_finish(const TcArgs &args, int nseq, int *sFlags, int nt) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        sFlags[9] = (atomicAdd(&args.ctrl[1], 1) == (int)gridDim.x - 1);
-    }
-    __syncthreads();
-    if (sFlags[9]) {
-        __threadfence();
-        for (int i = threadIdx.x; i < nseq; i += nt) args.ctrl[2 + i] = 0;
-        if (threadIdx.x == 0) {
-            args.ctrl[0] = 0;
-            args.ctrl[1] = 0;
-        }
-    }
-}
-
 // --------------------------------------------------------------- the kernel
 
 template <int DK, int DV, int MODE>
@@ -202,7 +182,7 @@ gla_tc_kernel(const TcArgs args) {
     __half *sEb = reinterpret_cast<__half *>(smem + Lay::eb(C));
     float *sGc = reinterpret_cast<float *>(smem + Lay::gc(C));
     int64_t *sRow = reinterpret_cast<int64_t *>(smem + Lay::row(C));  // (b*N + p)*heads + h, or -1
-    int *sFlags = reinterpret_cast<int *>(smem + Lay::flags(C));  // [0..3] exact-path sub-chunks, [8] tile, [9] last
+    int *sFlags = reinterpret_cast<int *>(smem + Lay::flags(C));  // [0..3] exact-path sub-chunks, [8] tile
     unsigned char *sScr = smem + Lay::scratch(C);
 
     // ------------------------------------------------ which tile
@@ -213,11 +193,10 @@ gla_tc_kernel(const TcArgs args) {
         if (tid == 0) sFlags[8] = atomicAdd(&args.ctrl[0], 1);
         __syncthreads();
         tile = sFlags[8];
-        // A ticket past the grid can only come from control words left behind
-        // by an aborted launch: record it and only take part in the reset.
+        // The control words are zeroed before every launch, so a ticket past
+        // the grid cannot happen; guard the indexing anyway.
         if (tile >= geo.nc * nseq) {
             if (tid == 0) atomicOr(args.status, 6u);
-            fused_finish(args, nseq, sFlags, NT);
             return;
         }
     } else {
@@ -602,7 +581,6 @@ gla_tc_kernel(const TcArgs args) {
         }
     }
 
-    if (MODE == TC_FUSED) fused_finish(args, nseq, sFlags, NT);
 }
 
 // Launch helper used by the per-d_k translation units.

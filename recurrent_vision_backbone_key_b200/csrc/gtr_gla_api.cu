@@ -171,7 +171,10 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     a.spin_limit = spin_limit;
     a.hold_seq = hold_seq;
     a.hold_chunk = hold_chunk;
-    cudaError_t e = launch_tc(a, TC_FUSED, st);
+    // Ticket and flags start from zero for every launch.
+    cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
+    if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
+    e = launch_tc(a, TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 

@@ -222,9 +222,9 @@ def test_empty_and_streams():
 
 
 def test_fused_repeated_calls_reset_control_words(oracle_mod):
-    """The fused kernel resets its ticket and flags itself: back-to-back
-    calls, interleaved with the three-phase schedule on the same stream,
-    all stay correct."""
+    """The fused kernel's ticket and flags start from zero on every call:
+    back-to-back calls, interleaved with the three-phase schedule on the same
+    stream, all stay correct."""
     H, W, heads = 24, 24, 4
     for i in range(4):
         q, k, v, g = gpu_inputs(2, H, W, heads, 64, 64, seed=300 + i)
