@@ -10,11 +10,13 @@
 //             (phase 3: the within-chunk score-value product fused with the
 //             boundary-state readout);
 //   FUSED   : summary, boundary state and output of a tile in one kernel.
-//             Tiles are handed out in chunk-major order by an atomic ticket;
-//             the state entering chunk c is passed from the tile of chunk c-1
-//             of the same sequence through a two-slot ring in L2 with a
-//             release/acquire flag (the boundary scan, done as a chain
-//             between tiles; the wait is bounded).
+//             A tile is one chunk, or two consecutive chunks of a sequence
+//             (d_v <= 64).  Tiles are handed out in chunk-major order by an
+//             atomic ticket; the state entering a tile is passed from the
+//             tile before it in the same sequence through a ring slot in L2
+//             with a release/acquire flag, and from the first chunk of a
+//             tile to the second through shared memory (the boundary scan,
+//             done as a chain between tiles; the wait is bounded).
 //
 // Numerics (fp16 tensor-core operands, fp32 accumulation):
 //   The chunk's tokens form sub-chunks of 16.  Per key dimension, with
@@ -40,7 +42,7 @@
 
 namespace gtr {
 
-enum TcMode : int { TC_SUMMARY = 0, TC_OUTPUT = 1, TC_FUSED = 2 };
+enum TcMode : int { TC_SUMMARY = 0, TC_OUTPUT = 1, TC_FUSED = 2, TC_FUSED_PAIR = 3 };
 
 // Largest decay over a 16-token sub-chunk (nats, either sign) for which the
 // diagonal block uses fp16 factors around the reference token.
@@ -128,14 +130,15 @@ __device__ __forceinline__ void st_release(int *p, int v) {
 
 // ------------------------------------------------------------ smem layout
 
-template <int DK, int DV>
+// One block of shared memory per chunk of the tile (NCH chunks per tile).
+template <int DK, int DV, int NCH>
 struct TcLayout {
     static constexpr int LDK = DK + 8;  // fp16 row stride (halves): 16-byte rows, conflict-free ldmatrix
     static constexpr int LDV = DV + 8;
     static constexpr int LDA = 24;      // 16x16 diagonal block rows (halves)
-    static constexpr int NW = DV / 16;  // warps: one 16-wide value slice each
-    static constexpr int NT = NW * 32;
-    // byte offsets for a chunk of C tokens (nsub = C/16 sub-chunks)
+    static constexpr int NW = DV / 16;  // warps per chunk: one 16-wide value slice each
+    static constexpr int NT = NW * 32 * NCH;
+    // byte offsets inside a chunk block, for a chunk of C tokens (nsub = C/16 sub-chunks)
     __host__ __device__ static size_t q(int) { return 0; }                                 // qs fp16 [C][LDK]
     __host__ __device__ static size_t k(int C) { return q(C) + (size_t)C * LDK * 2; }      // ke fp16 [C][LDK]
     __host__ __device__ static size_t v(int C) { return k(C) + (size_t)C * LDK * 2; }      // v  fp16 [C][LDV]
@@ -146,114 +149,146 @@ struct TcLayout {
     __host__ __device__ static size_t eb(int C) { return rs(C) + (size_t)(C / 16) * DK * 2; }  // E_u (fp16)
     __host__ __device__ static size_t gc(int C) { return eb(C) + (size_t)(C / 16) * DK * 2; }  // gamma_c
     __host__ __device__ static size_t row(int C) { return gc(C) + (size_t)DK * 4; }            // token-head row index
-    __host__ __device__ static size_t flags(int C) { return row(C) + (size_t)C * 8; }
+    __host__ __device__ static size_t flags(int C) { return row(C) + (size_t)C * 8; }          // exact-path sub-chunks
     // scratch, used in turn for the staged g rows (fp32 [C][DK]), the exact
-    // diagonal path's raw operands and the output staging
+    // diagonal path's raw operands, the state handed from the first chunk of
+    // a tile to the second, and the output staging
     __host__ __device__ static size_t scratch(int C) { return flags(C) + 64; }
     __host__ __device__ static size_t scratch_bytes(int C) {
         size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8, gs = (size_t)C * DK * 4;
+        size_t hs = NCH > 1 ? (size_t)DK * DV * 4 : 0;
         size_t m = o > e ? o : e;
-        return m > gs ? m : gs;
+        m = m > gs ? m : gs;
+        return m > hs ? m : hs;
     }
-    __host__ __device__ static size_t bytes(int C) { return scratch(C) + scratch_bytes(C); }
+    __host__ __device__ static size_t block(int C) { return (scratch(C) + scratch_bytes(C) + 127) & ~(size_t)127; }
+    __host__ __device__ static size_t misc(int C) { return NCH * block(C); }  // tile index
+    __host__ __device__ static size_t bytes(int C) { return misc(C) + 64; }
 };
 
 // --------------------------------------------------------------- the kernel
+//
+// NCH chunks per tile (2 for the fused schedule with d_v <= 64, else 1):
+// warps [NW*ch, NW*ch + NW) work on chunk ch of the tile.  The state enters
+// the tile's first chunk from the ring and is handed to the second chunk
+// through shared memory, so only every NCH-th chunk boundary goes through L2.
 
-template <int DK, int DV, int MODE>
-__global__ void __launch_bounds__(TcLayout<DK, DV>::NT)
+template <int DK, int DV, int MODE, int NCH>
+__global__ void __launch_bounds__(TcLayout<DK, DV, NCH>::NT)
 gla_tc_kernel(const TcArgs args) {
-    using Lay = TcLayout<DK, DV>;
+    using Lay = TcLayout<DK, DV, NCH>;
     constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
+    static_assert(NCH == 1 || MODE == TC_FUSED, "multi-chunk tiles are for the fused schedule");
     extern __shared__ __align__(128) unsigned char smem[];
     const Geom &geo = args.geo;
     const int C = geo.chunk;
     const int nsub = C / 16;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int ch = warp / NW, wl = warp - ch * NW;  // chunk of this warp, value slice within it
+    const size_t BLK = Lay::block(C);
+    int *sTile = reinterpret_cast<int *>(smem + Lay::misc(C));
 
-    __half *sQ = reinterpret_cast<__half *>(smem + Lay::q(C));
-    __half *sK = reinterpret_cast<__half *>(smem + Lay::k(C));
-    __half *sV = reinterpret_cast<__half *>(smem + Lay::v(C));
-    __half *sA = reinterpret_cast<__half *>(smem + Lay::a(C));
-    float *sGu = reinterpret_cast<float *>(smem + Lay::gu(C));
-    __half *sRp = reinterpret_cast<__half *>(smem + Lay::rp(C));
-    __half *sRs = reinterpret_cast<__half *>(smem + Lay::rs(C));
-    __half *sEb = reinterpret_cast<__half *>(smem + Lay::eb(C));
-    float *sGc = reinterpret_cast<float *>(smem + Lay::gc(C));
-    int64_t *sRow = reinterpret_cast<int64_t *>(smem + Lay::row(C));  // (b*N + p)*heads + h, or -1
-    int *sFlags = reinterpret_cast<int *>(smem + Lay::flags(C));  // [0..3] exact-path sub-chunks, [8] tile
-    unsigned char *sScr = smem + Lay::scratch(C);
+    // per-chunk views
+    auto blk = [&](int i) { return smem + (size_t)i * BLK; };
+    auto Q_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::q(C)); };
+    auto K_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::k(C)); };
+    auto V_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::v(C)); };
+    auto A_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::a(C)); };
+    auto Gu_ = [&](int i) { return reinterpret_cast<float *>(blk(i) + Lay::gu(C)); };
+    auto Rp_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::rp(C)); };
+    auto Rs_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::rs(C)); };
+    auto Eb_ = [&](int i) { return reinterpret_cast<__half *>(blk(i) + Lay::eb(C)); };
+    auto Gc_ = [&](int i) { return reinterpret_cast<float *>(blk(i) + Lay::gc(C)); };
+    auto Row_ = [&](int i) { return reinterpret_cast<int64_t *>(blk(i) + Lay::row(C)); };  // (b*N + p)*heads + h, or -1
+    auto Fl_ = [&](int i) { return reinterpret_cast<int *>(blk(i) + Lay::flags(C)); };
+    auto Scr_ = [&](int i) { return blk(i) + Lay::scratch(C); };
 
     // ------------------------------------------------ which tile
     const int nseq = geo.B * geo.heads;
-    if (tid < 16 && tid != 8) sFlags[tid] = 0;
+    if (tid < 4 * NCH) Fl_(tid >> 2)[tid & 3] = 0;
     int tile;
     if (MODE == TC_FUSED) {
-        if (tid == 0) sFlags[8] = atomicAdd(&args.ctrl[0], 1);
+        if (tid == 0) sTile[0] = atomicAdd(&args.ctrl[0], 1);
         __syncthreads();
-        tile = sFlags[8];
+        tile = sTile[0];
         // The control words are zeroed before every launch, so a ticket past
         // the grid cannot happen; guard the indexing anyway.
-        if (tile >= geo.nc * nseq) {
+        if (tile >= ((geo.nc + NCH - 1) / NCH) * nseq) {
             if (tid == 0) atomicOr(args.status, 6u);
             return;
         }
     } else {
         tile = blockIdx.x;
     }
-    int c, seq;
-    if (MODE == TC_FUSED) {  // chunk-major: chunk c of every sequence before chunk c+1
-        c = tile / nseq;
-        seq = tile - c * nseq;
+    int c0, seq;
+    if (MODE == TC_FUSED) {  // chunk-major: chunk group g of every sequence before group g+1
+        const int grp = tile / nseq;
+        seq = tile - grp * nseq;
+        c0 = grp * NCH;
     } else {
         seq = tile / geo.nc;
-        c = tile - seq * geo.nc;
+        c0 = tile - seq * geo.nc;
     }
     const int b = seq / geo.heads, h = seq - b * geo.heads;
-    const int t0 = c * C;
-    const int len = min(C, geo.N - t0);
     const float qscale = rsqrtf((float)DK);
-    // ------------------------------------------------ S0: the scan-order row table
-    // Row t of the chunk is token-head row (b*N + p)*heads + h of every
+    auto chunk_len = [&](int i) {
+        const int cc = c0 + i;
+        return cc < geo.nc ? min(C, geo.N - cc * C) : 0;
+    };
+
+    // ------------------------------------------------ S0: the scan-order row tables
+    // Row t of chunk i is token-head row (b*N + p)*heads + h of every
     // [B][N][heads][d] tensor; -1 past the end of the sequence.
-    for (int t = tid; t < C; t += NT)
-        sRow[t] = (t < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
-                            : (int64_t)-1;
+    // chunk of a flat index over NCH equal parts of size `part` (no division)
+    auto part_of = [](int idx, int part) { return (NCH > 1 && idx >= part) ? 1 : 0; };
+    for (int idx = tid; idx < NCH * C; idx += NT) {
+        const int i = part_of(idx, C), t = idx - i * C;
+        const int cc = c0 + i;
+        Row_(i)[t] = (t < chunk_len(i))
+                         ? ((int64_t)b * geo.N + scan_pos(geo.dir, cc * C + t, geo.H, geo.W, geo.N)) * geo.heads + h
+                         : (int64_t)-1;
+    }
     __syncthreads();
 
     // ------------------------------------------------ S1: stage q, k, v, g; prepare qs / ke
-    // Every row of the chunk is requested at once (cp.async, 16 bytes per
+    // Every row of the tile is requested at once (cp.async, 16 bytes per
     // request, rows past the sequence end zero-filled), so the whole tile is
     // in flight together; q and k land in the operand buffers and are turned
     // into qs / ke in place, g lands in the scratch region.
-    float *sG = reinterpret_cast<float *>(sScr);
     {
         constexpr int QCH = DK / 8, VCH = DV / 8, GCH = DK / 4;
-        for (int idx = tid; idx < C * VCH; idx += NT) {
-            const int t = idx / VCH, j = idx - t * VCH;
-            const int64_t r = sRow[t];
-            cp_async16(sV + t * LDV + j * 8, args.v + (r < 0 ? 0 : r) * DV + j * 8, r >= 0);
+        for (int idx = tid; idx < NCH * C * VCH; idx += NT) {
+            const int i = part_of(idx, C * VCH), rem = idx - i * (C * VCH);
+            const int t = rem / VCH, j = rem - t * VCH;
+            const int64_t r = Row_(i)[t];
+            cp_async16(V_(i) + t * LDV + j * 8, args.v + (r < 0 ? 0 : r) * DV + j * 8, r >= 0);
         }
-        for (int idx = tid; idx < C * QCH; idx += NT) {
-            const int t = idx / QCH, j = idx - t * QCH;
-            const int64_t r = sRow[t];
+        for (int idx = tid; idx < NCH * C * QCH; idx += NT) {
+            const int i = part_of(idx, C * QCH), rem = idx - i * (C * QCH);
+            const int t = rem / QCH, j = rem - t * QCH;
+            const int64_t r = Row_(i)[t];
             const int64_t o = (r < 0 ? 0 : r) * DK + j * 8;
-            if (MODE != TC_SUMMARY) cp_async16(sQ + t * LDK + j * 8, args.q + o, r >= 0);
-            cp_async16(sK + t * LDK + j * 8, args.k + o, r >= 0);
+            if (MODE != TC_SUMMARY) cp_async16(Q_(i) + t * LDK + j * 8, args.q + o, r >= 0);
+            cp_async16(K_(i) + t * LDK + j * 8, args.k + o, r >= 0);
         }
-        for (int idx = tid; idx < C * GCH; idx += NT) {
-            const int t = idx / GCH, j = idx - t * GCH;
-            const int64_t r = sRow[t];
-            cp_async16(sG + t * DK + j * 4, args.g + (r < 0 ? 0 : r) * DK + j * 4, r >= 0);
+        for (int idx = tid; idx < NCH * C * GCH; idx += NT) {
+            const int i = part_of(idx, C * GCH), rem = idx - i * (C * GCH);
+            const int t = rem / GCH, j = rem - t * GCH;
+            const int64_t r = Row_(i)[t];
+            cp_async16(reinterpret_cast<float *>(Scr_(i)) + t * DK + j * 4, args.g + (r < 0 ? 0 : r) * DK + j * 4,
+                       r >= 0);
         }
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
     }
-    for (int task = tid; task < (DK / 2) * nsub; task += NT) {
-        const int dp = task % (DK / 2), u = task / (DK / 2);
+    for (int task = tid; task < NCH * (DK / 2) * nsub; task += NT) {
+        const int i = part_of(task, (DK / 2) * nsub), rem = task - i * ((DK / 2) * nsub);
+        const int dp = rem % (DK / 2), u = rem / (DK / 2);
         const int d0 = 2 * dp;
+        __half *sQ = Q_(i), *sK = K_(i);
+        const float *sG = reinterpret_cast<const float *>(Scr_(i));
         __half2 qv[16], kv[16];
         float2 av[16];
 #pragma unroll
@@ -289,29 +324,30 @@ gla_tc_kernel(const TcArgs args) {
             S.x *= av[t].x;
             S.y *= av[t].y;
         }
-        *reinterpret_cast<float2 *>(sGu + u * DK + d0) = P;
+        *reinterpret_cast<float2 *>(Gu_(i) + u * DK + d0) = P;
         if (MODE != TC_SUMMARY) {
             const float lo = 6.737947e-3f /* e^-5 */, hi = 148.41316f /* e^5 */;
             const float2 qm = __half22float2(qmax), km = __half22float2(kmax);
             const bool fast = P.x >= lo && P.y >= lo && P.x <= hi && P.y <= hi &&
                               fmaxf(qm.x, qm.y) * qscale <= kDiagMaxAbs && fmaxf(km.x, km.y) <= kDiagMaxAbs;
-            if (!fast) sFlags[u] = 1;
-            *reinterpret_cast<__half2 *>(sRp + u * DK + d0) =
+            if (!fast) Fl_(i)[u] = 1;
+            *reinterpret_cast<__half2 *>(Rp_(i) + u * DK + d0) =
                 __floats2half2_rn(P7.x > 0.f ? 1.f / P7.x : 0.f, P7.y > 0.f ? 1.f / P7.y : 0.f);
-            *reinterpret_cast<__half2 *>(sRs + u * DK + d0) =
+            *reinterpret_cast<__half2 *>(Rs_(i) + u * DK + d0) =
                 __floats2half2_rn(S7.x > 0.f ? 1.f / S7.x : 0.f, S7.y > 0.f ? 1.f / S7.y : 0.f);
         }
     }
     __syncthreads();
 
     // ------------------------------------------------ S2: decay to each sub-chunk, chunk decay
-    for (int d = tid; d < DK; d += NT) {
+    for (int task = tid; task < NCH * DK; task += NT) {
+        const int i = part_of(task, DK), d = task - i * DK;
         float e = 1.f;
         for (int u = 0; u < nsub; ++u) {
-            sEb[u * DK + d] = __float2half_rn(e);
-            e *= sGu[u * DK + d];
+            Eb_(i)[u * DK + d] = __float2half_rn(e);
+            e *= Gu_(i)[u * DK + d];
         }
-        sGc[d] = e;
+        Gc_(i)[d] = e;
     }
 
     const int r8 = lane & 7, m4 = lane >> 3;
@@ -319,8 +355,10 @@ gla_tc_kernel(const TcArgs args) {
 
     // ------------------------------------------------ S3: diagonal 16x16 blocks
     if (MODE != TC_SUMMARY) {
-        for (int u = warp; u < nsub; u += NW) {
-            if (sFlags[u]) continue;
+        for (int pr = warp; pr < NCH * nsub; pr += NCH * NW) {
+            const int i = part_of(pr, nsub), u = pr - i * nsub;
+            if (Fl_(i)[u]) continue;
+            const __half *sQ = Q_(i), *sK = K_(i), *sRp = Rp_(i), *sRs = Rs_(i);
             float acc[2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
@@ -338,7 +376,7 @@ gla_tc_kernel(const TcArgs args) {
                 mma16816(acc[0], af, bf[0], bf[1]);
                 mma16816(acc[1], af, bf[2], bf[3]);
             }
-            __half *Au = sA + u * 16 * LDA;
+            __half *Au = A_(i) + u * 16 * LDA;
             const int tr = lane >> 2;
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -355,13 +393,16 @@ gla_tc_kernel(const TcArgs args) {
         // Exact path, one flagged sub-chunk at a time by the whole CTA:
         // A_ts = sum_d q~_td k_sd 2^(beta_td - beta_sd) with beta the in-sub-chunk
         // prefix sum of g*log2(e), from the raw operands.
-        const int any_exact = sFlags[0] | sFlags[1] | sFlags[2] | sFlags[3];
-        if (any_exact) {
-            __half *xq = reinterpret_cast<__half *>(sScr);
+        for (int i = 0; i < NCH; ++i) {
+            int *fl = Fl_(i);
+            if (!(fl[0] | fl[1] | fl[2] | fl[3])) continue;
+            __half *xq = reinterpret_cast<__half *>(Scr_(i));
             __half *xk = xq + 16 * DK;
             float *xb = reinterpret_cast<float *>(xk + 16 * DK);
+            const int64_t *sRow = Row_(i);
+            __half *sA = A_(i);
             for (int u = 0; u < nsub; ++u) {
-                if (!sFlags[u]) continue;
+                if (!fl[u]) continue;
                 for (int idx = tid; idx < 16 * DK; idx += NT) {
                     const int t = idx / DK, d = idx - t * DK;
                     const int64_t r = sRow[16 * u + t];
@@ -397,9 +438,13 @@ gla_tc_kernel(const TcArgs args) {
     __syncthreads();
 
     // ------------------------------------------------ S4: local state over sub-chunks
-    // Warp w owns value columns [16w, 16w+16).  L^T (16 x DK) lives in the
-    // accumulator layout: Lt[n][0..3] covers key columns 8n..8n+7.
-    const int v0 = 16 * warp;
+    // Warp (ch, wl) owns value columns [16wl, 16wl+16) of chunk ch.  L^T
+    // (16 x DK) lives in the accumulator layout: Lt[n][0..3] covers key
+    // columns 8n..8n+7.
+    const __half *sQ = Q_(ch), *sK = K_(ch), *sV = V_(ch), *sA = A_(ch), *sEb = Eb_(ch);
+    const float *sGu = Gu_(ch), *sGc = Gc_(ch);
+    const int v0 = 16 * wl;
+    const int c = c0 + ch;
     float Lt[KT][4];
 #pragma unroll
     for (int n = 0; n < KT; ++n) Lt[n][0] = Lt[n][1] = Lt[n][2] = Lt[n][3] = 0.f;
@@ -472,7 +517,7 @@ gla_tc_kernel(const TcArgs args) {
         return;
     }
 
-    // ------------------------------------------------ S5: the state entering the chunk
+    // ------------------------------------------------ S5: the state entering each chunk
     float Se[KT][4];
     bool have_state = c > 0;
     if (MODE == TC_OUTPUT) {
@@ -489,10 +534,15 @@ gla_tc_kernel(const TcArgs args) {
         have_state = true;
     } else {  // FUSED
         int *flags = args.ctrl + 2;
-        if (c > 0) {
+        // ring slot of the state entering the tile and of the one it leaves
+        // (two alternating slots with one chunk per tile; a single slot with
+        // two, since the tile reads it before it writes it)
+        const int slot_in = NCH == 1 ? ((c0 - 1) & 1) : 0;
+        const int slot_out = NCH == 1 ? (c0 & 1) : 0;
+        if (c0 > 0) {
             if (tid == 0) {
                 long long spins = 0;
-                while (ld_acquire(&flags[seq]) < c) {
+                while (ld_acquire(&flags[seq]) < c0) {
                     if (++spins > args.spin_limit) {
                         atomicOr(args.status, 6u);  // GTR_ERR_TIMEOUT
                         break;
@@ -501,34 +551,60 @@ gla_tc_kernel(const TcArgs args) {
                 }
             }
             __syncthreads();
-            const float4 *src = reinterpret_cast<const float4 *>(
-                args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
+            if (ch == 0) {
+                const float4 *src = reinterpret_cast<const float4 *>(
+                    args.ring + ((int64_t)seq * 2 + slot_in) * (DK * DV));
 #pragma unroll
-            for (int n = 0; n < KT; ++n) {
-                float4 x = __ldcg(src + ((warp * KT + n) * 32 + lane));
-                Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
+                for (int n = 0; n < KT; ++n) {
+                    float4 x = __ldcg(src + ((wl * KT + n) * 32 + lane));
+                    Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
+                }
             }
-        } else {
+        } else if (ch == 0) {
 #pragma unroll
             for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
         }
-        // publish S_leave = diag(gamma_c) S_enter + L for the next chunk
-        const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
-        if (c + 1 < geo.nc && !hold) {
-            float4 *dst = reinterpret_cast<float4 *>(
-                args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
+        if (NCH > 1) {
+            // chunk c0 hands diag(gamma) S_enter + L to chunk c0+1 through shared memory
+            float4 *hand = reinterpret_cast<float4 *>(Scr_(1));
+            if (ch == 0) {
 #pragma unroll
-            for (int n = 0; n < KT; ++n) {
-                const float2 gg = *reinterpret_cast<const float2 *>(sGc + 8 * n + kc);
-                float4 x;
-                x.x = fmaf(gg.x, Se[n][0], Lt[n][0]);
-                x.y = fmaf(gg.y, Se[n][1], Lt[n][1]);
-                x.z = fmaf(gg.x, Se[n][2], Lt[n][2]);
-                x.w = fmaf(gg.y, Se[n][3], Lt[n][3]);
-                __stcg(dst + ((warp * KT + n) * 32 + lane), x);
+                for (int n = 0; n < KT; ++n) {
+                    const float2 gg = *reinterpret_cast<const float2 *>(sGc + 8 * n + kc);
+                    hand[(wl * KT + n) * 32 + lane] =
+                        make_float4(fmaf(gg.x, Se[n][0], Lt[n][0]), fmaf(gg.y, Se[n][1], Lt[n][1]),
+                                    fmaf(gg.x, Se[n][2], Lt[n][2]), fmaf(gg.y, Se[n][3], Lt[n][3]));
+                }
             }
             __syncthreads();
-            if (tid == 0) st_release(&flags[seq], c + 1);
+            if (ch == NCH - 1) {
+#pragma unroll
+                for (int n = 0; n < KT; ++n) {
+                    const float4 x = hand[(wl * KT + n) * 32 + lane];
+                    Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
+                }
+                have_state = true;
+            }
+            __syncthreads();  // the hand-over region is reused for output staging below
+        }
+        // the tile's last chunk publishes diag(gamma_c) S_enter + L for the next tile
+        const bool hold = (seq == args.hold_seq && args.hold_chunk >= c0 && args.hold_chunk < c0 + NCH);
+        if (c0 + NCH < geo.nc && !hold) {
+            if (ch == NCH - 1) {
+                float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + slot_out) * (DK * DV));
+#pragma unroll
+                for (int n = 0; n < KT; ++n) {
+                    const float2 gg = *reinterpret_cast<const float2 *>(sGc + 8 * n + kc);
+                    float4 x;
+                    x.x = fmaf(gg.x, Se[n][0], Lt[n][0]);
+                    x.y = fmaf(gg.y, Se[n][1], Lt[n][1]);
+                    x.z = fmaf(gg.x, Se[n][2], Lt[n][2]);
+                    x.w = fmaf(gg.y, Se[n][3], Lt[n][3]);
+                    __stcg(dst + ((wl * KT + n) * 32 + lane), x);
+                }
+            }
+            __syncthreads();
+            if (tid == 0) st_release(&flags[seq], c0 + NCH);
         }
     }
 
@@ -560,7 +636,7 @@ gla_tc_kernel(const TcArgs args) {
 
     // ------------------------------------------------ S7: store the outputs
     {
-        __half *sOut = reinterpret_cast<__half *>(sScr);
+        __half *sOut = reinterpret_cast<__half *>(Scr_(ch));
         const int tr = lane >> 2;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -574,35 +650,44 @@ gla_tc_kernel(const TcArgs args) {
         }
         __syncthreads();
         constexpr int VCH = DV / 8;
-        for (int idx = tid; idx < len * VCH; idx += NT) {
-            const int t = idx / VCH, j = idx - t * VCH;
-            *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
-                *reinterpret_cast<const int4 *>(sOut + t * LDV + j * 8);
+        for (int i = 0; i < NCH; ++i) {
+            const int len = chunk_len(i);
+            const __half *so = reinterpret_cast<const __half *>(Scr_(i));
+            const int64_t *sRow = Row_(i);
+            for (int idx = tid; idx < len * VCH; idx += NT) {
+                const int t = idx / VCH, j = idx - t * VCH;
+                *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
+                    *reinterpret_cast<const int4 *>(so + t * LDV + j * 8);
+            }
         }
     }
-
 }
 
 // Launch helper used by the per-d_k translation units.
-template <int DK, int DV, int MODE>
+template <int DK, int DV, int MODE, int NCH>
 cudaError_t launch_tc_mode(const TcArgs &a, cudaStream_t st) {
-    using Lay = TcLayout<DK, DV>;
+    using Lay = TcLayout<DK, DV, NCH>;
     const size_t smem = Lay::bytes(a.geo.chunk);
-    cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel<DK, DV, MODE>,
+    cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel<DK, DV, MODE, NCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((int64_t)a.geo.nc * a.geo.B * a.geo.heads);
-    gla_tc_kernel<DK, DV, MODE><<<grid, Lay::NT, smem, st>>>(a);
+    const int64_t groups = (a.geo.nc + NCH - 1) / NCH;
+    const unsigned grid = (unsigned)(groups * a.geo.B * a.geo.heads);
+    gla_tc_kernel<DK, DV, MODE, NCH><<<grid, Lay::NT, smem, st>>>(a);
     count_launch();
     return cudaGetLastError();
 }
 
+// mode TC_FUSED_PAIR: the fused schedule with two chunks per tile (d_v <= 64).
 template <int DK, int DV>
 cudaError_t launch_tc_dv(const TcArgs &a, int mode, cudaStream_t st) {
     switch (mode) {
-    case TC_SUMMARY: return launch_tc_mode<DK, DV, TC_SUMMARY>(a, st);
-    case TC_OUTPUT: return launch_tc_mode<DK, DV, TC_OUTPUT>(a, st);
-    default: return launch_tc_mode<DK, DV, TC_FUSED>(a, st);
+    case TC_SUMMARY: return launch_tc_mode<DK, DV, TC_SUMMARY, 1>(a, st);
+    case TC_OUTPUT: return launch_tc_mode<DK, DV, TC_OUTPUT, 1>(a, st);
+    case TC_FUSED_PAIR:
+        if constexpr (DV <= 64) return launch_tc_mode<DK, DV, TC_FUSED, 2>(a, st);
+        return launch_tc_mode<DK, DV, TC_FUSED, 1>(a, st);
+    default: return launch_tc_mode<DK, DV, TC_FUSED, 1>(a, st);
     }
 }
 
@@ -616,8 +701,6 @@ cudaError_t launch_tc_dk(const TcArgs &a, int mode, cudaStream_t st) {
     }
 }
 
-size_t tc_smem_bytes(int dk, int dv, int chunk);
 cudaError_t launch_tc(const TcArgs &a, int mode, cudaStream_t st);
-
 
 }  // namespace gtr

@@ -146,6 +146,24 @@ gtr_status_t status_word(unsigned **out) {
 
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
 
+// Streaming multiprocessors of the current device (cached per device).
+cudaError_t sm_count(int *out) {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lk(mu);
+    auto it = cache.find(dev);
+    if (it == cache.end()) {
+        int n = 0;
+        if ((e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        it = cache.emplace(dev, n).first;
+    }
+    *out = it->second;
+    return cudaSuccess;
+}
+
 TcArgs make_args(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo) {
     TcArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.geo = geo;
@@ -174,7 +192,13 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     // Ticket and flags start from zero for every launch.
     cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
     if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
-    e = launch_tc(a, TC_FUSED, st);
+    // Few sequences leave the chain of boundary states as the critical path:
+    // then two chunks per tile halve its length.  Many sequences keep every
+    // SM busy anyway: then one chunk per tile gives more resident CTAs.
+    int sms = 0;
+    if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
+    const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
+    e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 
