@@ -50,6 +50,28 @@ def measured_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
+def profiled_traffic(w, schedule):
+    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+    if that summary was taken on this workload from the current kernel source."""
+    import hashlib
+    prof = os.path.join(ROOT, "profiles", "gla_tc_fused_d64_batched.md")
+    if w.name != "batched" or schedule not in ("auto", "fused") or not os.path.exists(prof):
+        return None
+    src = os.path.join(ROOT, "recurrent_vision_backbone_key_b200", "csrc")
+    h = hashlib.sha256()
+    for f in ("gla_tc.cuh", "gla_common.cuh"):
+        with open(os.path.join(src, f), "rb") as fh:
+            h.update(fh.read())
+    fields = {}
+    for line in open(prof):
+        if ":" in line and line.split(":")[0].strip() in ("kernel_source_sha256_16", "traffic_bytes_per_launch"):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip()
+    if fields.get("kernel_source_sha256_16") != h.hexdigest()[:16]:
+        return None
+    return int(fields["traffic_bytes_per_launch"])
+
+
 def describe(w):
     dirs = "+".join(DIR_NAMES[d] for d in w.directions)
     return (f"{w.name}: B{w.B} {w.grid_h}x{w.grid_w} grid ({w.N} tokens), {w.heads} heads, "
@@ -257,14 +279,15 @@ def main():
     per_launch_ms = ms / args.steps
     dominant = "forward step"
     phase_ms = None
-    if sched in (2, 3):
+    if sched == 2:
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
         dominant = max(phase_ms, key=phase_ms.get)
         per_launch_ms = phase_ms[dominant]
         alg_bytes = phase_alg_bytes(w)[dominant]
     achieved = alg_bytes / (per_launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved / hbm_peak, "traffic": None,
+                "frac": achieved / hbm_peak,
+                "traffic": profiled_traffic(w, args.schedule) if phase_ms is None else None,
                 "kernel": dominant, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "tensor_flops_per_step": w.algorithmic_flops(),
