@@ -229,7 +229,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS))
-    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase", "three_phase_simt"])
+    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase", "three_phase_simt", "fused_tcgen05"])
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)

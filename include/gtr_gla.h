@@ -82,7 +82,10 @@ typedef enum {
     GTR_SCHED_AUTO = 0,             /* library choice: the fused kernel */
     GTR_SCHED_FUSED = 1,            /* one kernel: summaries, chained boundary states, outputs */
     GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output (tensor cores) */
-    GTR_SCHED_THREE_PHASE_SIMT = 3  /* the same three phases on CUDA cores only (comparison) */
+    GTR_SCHED_THREE_PHASE_SIMT = 3, /* the same three phases on CUDA cores only (comparison) */
+    GTR_SCHED_FUSED_TCGEN05 = 4     /* fused, whole-chunk products on tcgen05 tensor cores with
+                                       tensor-memory accumulators (d_k = d_v = 64, chunk 64;
+                                       other shapes run GTR_SCHED_FUSED) */
 } gtr_schedule_t;
 
 /* The GLA forward over all B*heads sequences (see the operation above).

@@ -702,5 +702,7 @@ cudaError_t launch_tc_dk(const TcArgs &a, int mode, cudaStream_t st) {
 }
 
 cudaError_t launch_tc(const TcArgs &a, int mode, cudaStream_t st);
+// tcgen05 fused kernel (d_k = d_v = 64, chunk 64), gla_umma.cu.
+cudaError_t launch_fused_umma(const TcArgs &a, cudaStream_t st);
 
 }  // namespace gtr

@@ -1,0 +1,483 @@
+// gla_umma.cuh -- fused GLA forward on the 5th-generation tensor cores
+// (tcgen05 MMAs from shared-memory descriptors into tensor memory) for
+// d_k = d_v = 64 and chunks of 64 tokens.
+//
+// Same schedule as the fused mode of gla_tc.cuh (one (sequence, chunk) tile
+// per CTA, chunk-major tickets, boundary state chained through an L2 ring with
+// release/acquire flags, bounded waits), with the chunk's dense products done
+// as whole-chunk 64x64x64 MMAs:
+//   with a_t = exp(g_t), E_t = a_0..a_t (decay since the chunk start),
+//   Suf_t = a_{t+1}..a_63 (decay to the chunk end), gamma_c = E_63:
+//     ke_s  = k_s Suf_s                       (<= |k|)
+//     qh_t  = q~_t E_t / gamma_c = q~_t / Suf_t
+//     A     = qh ke^T            -> A_ts = sum_d q~_td k_sd exp(b_td - b_sd)
+//     dS^T  = V^T ke             (the chunk summary; value rows)
+//     O     = tril(A) V + qh (gamma_c . S_enter)
+//     S_leave = diag(gamma_c) S_enter + dS
+//   GTR project page, "A Kernel That Makes Recurrence Fast": the summary
+//   (dS), the boundary scan (the chain), and the output product fused with
+//   the boundary readout.
+// qh grows like exp(chunk decay); the whole-chunk form is used when the decay
+// over the chunk is at most kChunkRange nats in every key dimension.  Other
+// chunks keep the three MMAs with the safe operands qe_t = q~_t E_t (<= |q~|)
+// and compute the score matrix exactly on CUDA cores.
+//
+// Operands live in shared memory as 64 x 64 fp16 row-major tiles with 128-byte
+// rows in the 128-byte swizzled canonical layout (16-byte chunk j of row r
+// stored at chunk j ^ (r mod 8)), read as K-major or MN-major by the MMA
+// descriptors.  Accumulators: TMEM columns [0,64) hold A and then O, columns
+// [64,128) hold dS^T; with M = 64, row m sits in TMEM lane (m mod 16) + 32 (m / 16),
+// so warp w reads rows 16w..16w+15 with the 16x256b load, in the m16n8
+// accumulator-fragment layout.
+#pragma once
+
+#include "gla_tc.cuh"
+
+namespace gtr {
+
+// Largest total decay over a chunk (nats) for the whole-chunk tensor-core form.
+constexpr float kChunkRange = 8.0f;
+
+// ---------------------------------------------------------------- tcgen05 helpers
+
+// Shared-memory matrix descriptor, 128-byte swizzle, version 1 (sm_100).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version
+    d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor: kind::f16, fp16 A and B, fp32 D, M = 64, N = 64.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int a_mn_major, int b_mn_major) {
+    return (1u << 4)                       // D format fp32
+           | (0u << 7) | (0u << 10)        // A, B fp16
+           | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16)
+           | ((64u >> 3) << 17)            // N
+           | ((64u >> 4) << 24);           // M
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}\n"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t mbar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(mbar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// 16 TMEM lanes x 64 fp32 columns -> 32 registers in the m16n8 fragment
+// layout: r[4n + i] is element i of the 8-column tile n.
+__device__ __forceinline__ void tmem_ld_16x64(uint32_t taddr, float (&r)[32]) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+          "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+          "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(mbar), "r"(count) : "memory");
+}
+// Bounded wait for the given phase parity; returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long long limit) {
+    for (long long i = 0; i < limit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(mbar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// Byte offset of element (row, col) in a 64 x 64 fp16 tile with 128-byte rows,
+// 128-byte swizzle.
+__device__ __forceinline__ uint32_t sw128(int row, int col) {
+    return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + ((col & 7) << 1));
+}
+
+// ---------------------------------------------------------------- layout
+struct UmmaLayout {
+    // all offsets relative to a 1024-byte aligned base
+    static constexpr uint32_t QH = 0;          // raw q rows, then the qh (or qe) tile in place
+    static constexpr uint32_t KE = 8192;       // raw k rows, then the ke tile in place
+    static constexpr uint32_t RQ = QH;
+    static constexpr uint32_t RK = KE;
+    static constexpr uint32_t V = 16384;       // v tile (also read as MN-major)
+    static constexpr uint32_t G = 24576;       // raw g rows fp32 [64][64] (16 KB); then the exact
+                                               // path's staging; then P + S'; then the output staging
+    static constexpr uint32_t P = G;           // masked scores
+    static constexpr uint32_t SP = G + 8192;   // (scaled entering state)^T, rows = value columns
+    static constexpr uint32_t VEC = 40960;     // gamma_c[64], sc[64], sub-chunk totals [4][64] (fp32)
+    static constexpr uint32_t ROW = VEC + 6 * 64 * 4;  // int64 [64]
+    static constexpr uint32_t MISC = ROW + 64 * 8;     // tile, exact flag, tmem base, mbarrier (8-aligned)
+    static constexpr uint32_t BYTES = MISC + 64;
+    static constexpr uint32_t ALLOC = BYTES + 1024;    // slack for aligning the base
+};
+
+// ---------------------------------------------------------------- the kernel
+__global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
+    using L = UmmaLayout;
+    constexpr int DK = 64, DV = 64, C = 64, KT = 8;
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    // 1024-byte aligned base (the swizzled operand tiles need it)
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t base_addr = (raw_addr + 1023u) & ~1023u;
+    unsigned char *base = smem_raw + (base_addr - raw_addr);
+    const Geom &geo = args.geo;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tr = lane >> 2, kc = 2 * (lane & 3);
+    float *vGc = reinterpret_cast<float *>(base + L::VEC);
+    float *vSc = vGc + 64;
+    float *vTot = vSc + 64;  // [4][64]
+    int64_t *sRow = reinterpret_cast<int64_t *>(base + L::ROW);
+    int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [1] exact [2] tmem base [3] pad; mbar at +16
+    const uint32_t mbar = base_addr + L::MISC + 16;
+    const int nseq = geo.B * geo.heads;
+
+    // ---- tensor memory first (before the ticket: a CTA waiting for TMEM holds no ticket)
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;\n" ::"r"(base_addr + L::MISC + 8)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        misc[0] = atomicAdd(&args.ctrl[0], 1);
+        misc[1] = 0;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[2];
+    const int tile = misc[0];
+    bool ok_tile = tile < geo.nc * nseq;
+    if (!ok_tile && tid == 0) atomicOr(args.status, 6u);
+
+    const int c = ok_tile ? tile / nseq : 0;
+    const int seq = ok_tile ? tile - c * nseq : 0;
+    const int b = seq / geo.heads, h = seq - b * geo.heads;
+    const int t0 = c * C;
+    const int len = ok_tile ? min(C, geo.N - t0) : 0;
+    const float qscale = rsqrtf((float)DK);
+
+    if (ok_tile) {
+        // ---- row table
+        if (tid < C)
+            sRow[tid] = (tid < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + tid, geo.H, geo.W, geo.N)) * geo.heads + h
+                                    : (int64_t)-1;
+        __syncthreads();
+
+        // ---- stage q, k, g rows (raw) and v (swizzled operand tile), one cp.async batch
+        for (int idx = tid; idx < C * 8; idx += 128) {
+            const int t = idx >> 3, j = idx & 7;
+            const int64_t r = sRow[t];
+            const int64_t o = (r < 0 ? 0 : r) * 64 + j * 8;
+            cp_async16(base + L::RQ + t * 128 + j * 16, args.q + o, r >= 0);
+            cp_async16(base + L::RK + t * 128 + j * 16, args.k + o, r >= 0);
+            cp_async16(base + L::V + t * 128 + (((j ^ (t & 7)) & 7) << 4), args.v + o, r >= 0);
+        }
+        for (int idx = tid; idx < C * 16; idx += 128) {
+            const int t = idx >> 4, j = idx & 15;
+            const int64_t r = sRow[t];
+            cp_async16(base + L::G + t * 256 + j * 16, args.g + (r < 0 ? 0 : r) * 64 + j * 4, r >= 0);
+        }
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncthreads();
+
+        // ---- operand prep: task (dim pair dp, sub-chunk u), 16 tokens each
+        const int dp = tid & 31, u = tid >> 5;
+        const int d0 = 2 * dp;
+        __half2 qv[16], kv[16];
+        float2 av[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            const int row = 16 * u + t;
+            qv[t] = *reinterpret_cast<const __half2 *>(base + L::RQ + row * 128 + d0 * 2);
+            kv[t] = *reinterpret_cast<const __half2 *>(base + L::RK + row * 128 + d0 * 2);
+            const float2 gv = *reinterpret_cast<const float2 *>(base + L::G + row * 256 + d0 * 4);
+            av[t] = make_float2(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e));
+        }
+        float2 tot = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            tot.x *= av[t].x;
+            tot.y *= av[t].y;
+        }
+        *reinterpret_cast<float2 *>(vTot + u * 64 + d0) = tot;
+        __syncthreads();  // sub-chunk totals visible; raw q / k / g all read
+        float2 Ebase = make_float2(1.f, 1.f), Sbase = make_float2(1.f, 1.f), gam = make_float2(1.f, 1.f);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float2 tw = *reinterpret_cast<const float2 *>(vTot + w * 64 + d0);
+            if (w < u) { Ebase.x *= tw.x; Ebase.y *= tw.y; }
+            if (w > u) { Sbase.x *= tw.x; Sbase.y *= tw.y; }
+            gam.x *= tw.x;
+            gam.y *= tw.y;
+        }
+        const float lo = 3.3546263e-4f;  // e^-kChunkRange
+        __half2 qmax = __float2half2_rn(0.f);
+#pragma unroll
+        for (int t = 0; t < 16; ++t) qmax = __hmax2(qmax, __habs2(qv[t]));
+        const float2 qm = __half22float2(qmax);
+        const bool fast = gam.x >= lo && gam.y >= lo && gam.x <= 1.f / lo && gam.y <= 1.f / lo &&
+                          fmaxf(qm.x, qm.y) * qscale <= 16.f;
+        if (!fast) misc[1] = 1;
+        if (u == 0) {
+            *reinterpret_cast<float2 *>(vGc + d0) = gam;
+        }
+        __syncthreads();
+        const bool exact = misc[1] != 0;
+        // qh = q~ E_t / gamma_c (whole-chunk form) or qe = q~ E_t (exact form)
+        const float2 rg = exact ? make_float2(1.f, 1.f) : make_float2(1.f / gam.x, 1.f / gam.y);
+        if (u == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
+        float2 E = Ebase;
+#pragma unroll
+        for (int t = 0; t < 16; ++t) {
+            E.x *= av[t].x;
+            E.y *= av[t].y;
+            *reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0)) =
+                __hmul2(qv[t], __floats2half2_rn(E.x * rg.x * qscale, E.y * rg.y * qscale));
+        }
+        float2 S = Sbase;  // decay after token t to the chunk end
+#pragma unroll
+        for (int t = 15; t >= 0; --t) {
+            *reinterpret_cast<__half2 *>(base + L::KE + sw128(16 * u + t, d0)) =
+                __hmul2(kv[t], __floats2half2_rn(S.x, S.y));
+            S.x *= av[t].x;
+            S.y *= av[t].y;
+        }
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- MMAs: A = qh ke^T (whole-chunk form only), dS^T = V^T ke
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
+            if (!exact) {
+                const uint32_t id = umma_idesc_f16(0, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024),
+                             id, ks > 0);
+            }
+            const uint32_t id2 = umma_idesc_f16(1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tmem + 64, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
+                         umma_desc_sw128(aKE + 2048 * ks, 8192, 1024), id2, ks > 0);
+            umma_commit(mbar);
+        }
+
+        // ---- exact form: the score matrix on CUDA cores from the raw operands
+        float pe[32];
+        if (exact) {
+            // thread -> query row t = tid / 2, keys s in [32*(tid&1), +32)
+            const int t = tid >> 1, sb = 32 * (tid & 1);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pe[j] = 0.f;
+            // log2-domain in-chunk prefix of g, two halves of 32 dims, staged
+            // in the raw g region (consumed above)
+            __half *xq = reinterpret_cast<__half *>(base + L::G);          // [64][32]
+            __half *xk = reinterpret_cast<__half *>(base + L::G + 4096);   // [64][32]
+            float *xb = reinterpret_cast<float *>(base + L::G + 8192);     // [64][32]
+            for (int hd = 0; hd < 2; ++hd) {
+                __syncthreads();
+                for (int idx = tid; idx < 64 * 32; idx += 128) {
+                    const int tt = idx >> 5, d = idx & 31;
+                    const int64_t r = sRow[tt];
+                    const int64_t o = (r < 0 ? 0 : r) * 64 + 32 * hd + d;
+                    xq[idx] = r >= 0 ? args.q[o] : __float2half(0.f);
+                    xk[idx] = r >= 0 ? args.k[o] : __float2half(0.f);
+                    xb[idx] = r >= 0 ? args.g[o] * kLog2e : 0.f;
+                }
+                __syncthreads();
+                if (tid < 32) {
+                    float acc = 0.f;
+                    for (int tt = 0; tt < 64; ++tt) {
+                        acc += xb[tt * 32 + tid];
+                        xb[tt * 32 + tid] = acc;
+                    }
+                }
+                __syncthreads();
+                for (int d = 0; d < 32; ++d) {
+                    const float qq = __half2float(xq[t * 32 + d]) * qscale;
+                    const float bt = xb[t * 32 + d];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int s = sb + j;
+                        if (s <= t)
+                            pe[j] = fmaf(qq * __half2float(xk[s * 32 + d]), ex2(bt - xb[s * 32 + d]), pe[j]);
+                    }
+                }
+            }
+        }
+
+        // ---- wait for the MMAs, write the masked scores P (fp16, swizzled)
+        if (!mbar_wait(mbar, 0, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        tc_fence_after();
+        if (!exact) {
+            float a[32];
+            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
+            tc_wait_ld();
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int t = 16 * warp + tr + 8 * hf, s = 8 * n + kc;
+                    const float x0 = s <= t ? a[4 * n + 2 * hf] : 0.f;
+                    const float x1 = s + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, s)) = pack_h2(x0, x1);
+                }
+            }
+        } else {
+            __syncthreads();  // the exact path's staging (in the P / S' region) is consumed
+            const int t = tid >> 1, sb = 32 * (tid & 1);
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+                *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sb + j)) = pack_h2(pe[j], pe[j + 1]);
+        }
+
+        // ---- the state entering the chunk, the chunk summary, publish
+        float Se[KT][4], dS[32];
+        tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16) + 64, dS);
+        tc_wait_ld();
+        int *flags = args.ctrl + 2;
+        if (c > 0) {
+            if (tid == 0) {
+                long long spins = 0;
+                while (ld_acquire(&flags[seq]) < c) {
+                    if (++spins > args.spin_limit) {
+                        atomicOr(args.status, 6u);  // GTR_ERR_TIMEOUT
+                        break;
+                    }
+                    __nanosleep(spins < 64 ? 32 : 256);
+                }
+            }
+            __syncthreads();
+            const float4 *src = reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
+#pragma unroll
+            for (int n = 0; n < KT; ++n) {
+                const float4 x = __ldcg(src + ((warp * KT + n) * 32 + lane));
+                Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
+        }
+        const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
+        if (c + 1 < geo.nc && !hold) {
+            float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
+#pragma unroll
+            for (int n = 0; n < KT; ++n) {
+                const float2 gg = *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
+                float4 x;
+                x.x = fmaf(gg.x, Se[n][0], dS[4 * n + 0]);
+                x.y = fmaf(gg.y, Se[n][1], dS[4 * n + 1]);
+                x.z = fmaf(gg.x, Se[n][2], dS[4 * n + 2]);
+                x.w = fmaf(gg.y, Se[n][3], dS[4 * n + 3]);
+                __stcg(dst + ((warp * KT + n) * 32 + lane), x);
+            }
+            __syncthreads();
+            if (tid == 0) st_release(&flags[seq], c + 1);
+        }
+        // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value columns)
+#pragma unroll
+        for (int n = 0; n < KT; ++n) {
+            const float2 sc = *reinterpret_cast<const float2 *>(vSc + 8 * n + kc);
+            const int dv0 = 16 * warp + tr, dk = 8 * n + kc;
+            *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
+            *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
+        }
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- O = P V + qh S'  (overwrites A's columns; A has been read)
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t aP = base_addr + L::P, aV = base_addr + L::V, aQH = base_addr + L::QH,
+                           aSP = base_addr + L::SP;
+            const uint32_t id_pv = umma_idesc_f16(0, 1), id_qs = umma_idesc_f16(0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tmem, umma_desc_sw128(aP + 32 * ks, 16, 1024), umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
+                         id_pv, ks > 0);
+            if (c > 0) {
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024),
+                             umma_desc_sw128(aSP + 32 * ks, 16, 1024), id_qs, 1);
+            }
+            umma_commit(mbar);
+        }
+        if (!mbar_wait(mbar, 1, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        tc_fence_after();
+
+        // ---- store O: fragments -> swizzled staging (the P / S' region) -> 16-byte rows
+        {
+            float o[32];
+            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), o);
+            tc_wait_ld();
+            unsigned char *st = base + L::G;  // P / S' are consumed by the finished MMA
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+                const int t = 16 * warp + tr, col = 8 * n + kc;
+                *reinterpret_cast<uint32_t *>(st + sw128(t, col)) = pack_h2(o[4 * n], o[4 * n + 1]);
+                *reinterpret_cast<uint32_t *>(st + sw128(t + 8, col)) = pack_h2(o[4 * n + 2], o[4 * n + 3]);
+            }
+            __syncthreads();
+            for (int idx = tid; idx < len * 8; idx += 128) {
+                const int t = idx >> 3, j = idx & 7;
+                *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
+                    *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
+            }
+        }
+    }
+
+    // ---- release tensor memory
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;\n" ::"r"(tmem) : "memory");
+    }
+}
+
+inline cudaError_t launch_umma(const TcArgs &a, cudaStream_t st) {
+    const size_t smem = UmmaLayout::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(gla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)((int64_t)a.geo.nc * a.geo.B * a.geo.heads);
+    gla_umma_kernel<<<grid, 128, smem, st>>>(a);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace gtr

@@ -173,9 +173,11 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
     return a;
 }
 
+bool tcgen05_shape(const Geom &g) { return g.dk == 64 && g.dv == 64 && g.chunk == 64; }
+
 gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const float *g,
                        const Geom &geo, __half *out, cudaStream_t st, int hold_seq = -1,
-                       int hold_chunk = -1, long long spin_limit = kSpinLimit) {
+                       int hold_chunk = -1, long long spin_limit = kSpinLimit, bool tcgen05 = false) {
     void *ws = nullptr;
     gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
     if (s != GTR_OK) return s;
@@ -198,7 +200,10 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     int sms = 0;
     if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
     const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
-    e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
+    if (tcgen05 && tcgen05_shape(geo))
+        e = launch_fused_umma(a, st);
+    else
+        e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 
@@ -246,7 +251,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     bool empty = false;
     gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
     if (s != GTR_OK) return s;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE_SIMT)
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05)
         return fail(GTR_ERR_INVALID_ARG, "bad schedule%s");
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out))
@@ -262,7 +267,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     __half *ho = static_cast<__half *>(out);
     if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
-    return run_fused(hq, hk, hv, g, geo, ho, st);
+    return run_fused(hq, hk, hv, g, geo, ho, st, -1, -1, kSpinLimit, schedule == GTR_SCHED_FUSED_TCGEN05);
 }
 
 }  // namespace
@@ -423,7 +428,7 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k
     Geom geo;
     bool empty = false;
     if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return 0;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_THREE_PHASE_SIMT || empty) return 0;
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05 || empty) return 0;
     if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT)
         return three_phase_ws(geo);
     return fused_ws(geo);

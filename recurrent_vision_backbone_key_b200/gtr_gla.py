@@ -28,7 +28,7 @@ STATUS_NAMES = {
     7: "GTR_ERR_OOM",
 }
 DIRECTIONS = {"l2r": 0, "r2l": 1, "t2b": 2, "b2t": 3}
-SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3}
+SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4}
 
 # Every symbol include/gtr_gla.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p

@@ -15,7 +15,7 @@ from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, s
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["fused", "three_phase", "three_phase_simt"]
+SCHEDULES = ["fused", "fused_tcgen05", "three_phase", "three_phase_simt"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -255,3 +255,33 @@ def test_fused_bounded_wait_times_out_cleanly(oracle_mod):
     torch.cuda.synchronize()
     assert torch.equal(out3, out2)
     assert gtr_gla.gtr_gla_get_last_device_status() == 0
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
+def test_special_gates_d64(oracle_mod, schedule):
+    """d_k = d_v = 64, chunk 64: the shape of the tcgen05 path, whose exact
+    score path takes over when the decay over a chunk is strong."""
+    H, W = 10, 13
+    q, k, v, g = gpu_inputs(2, H, W, 2, 64, 64, seed=17)
+    cases = {
+        "mild": g,
+        "open": torch.zeros_like(g),
+        "closed": torch.full_like(g, -1.0e4),
+        "strong": gpu_inputs(2, H, W, 2, 64, 64, seed=17, gate="strong")[3],
+        "mixed": torch.where(torch.rand_like(g) < 0.97, g, g * 60.0),
+    }
+    for name, gg in cases.items():
+        for direction in (0, 3):
+            out = run_forward(q, k, v, gg, H, W, direction, 64, schedule)
+            compare(out, oracle_full(oracle_mod, q, k, v, gg, H, W, direction))
+
+
+@pytest.mark.parametrize("direction", [0, 2])
+def test_batched_full_size_tcgen05_sampled(oracle_mod, direction):
+    w = WORKLOADS["batched"]
+    q, k, v, g = make_workload_inputs(w, seed=10 + direction, device="cuda")
+    out = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk, "fused_tcgen05")
+    assert torch.isfinite(out).all()
+    _sampled_check(oracle_mod, w, q, k, v, g, out, direction, 6, seed=direction)
+    ref = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk, "fused")
+    assert ((out.float() - ref.float()).abs().max() / ref.float().abs().max()).item() < 2e-3
