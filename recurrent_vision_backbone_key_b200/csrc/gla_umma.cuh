@@ -154,7 +154,7 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
     float *vSc = vGc + 64;
     float *vTot = vSc + 64;  // [4][64]
     int64_t *sRow = reinterpret_cast<int64_t *>(base + L::ROW);
-    int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [1] exact [2] tmem base [3] pad; mbar at +16
+    int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [1] exact [2] tmem base; mbar at +16
     const uint32_t mbar = base_addr + L::MISC + 16;
     const int nseq = geo.B * geo.heads;
 
@@ -364,12 +364,12 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
                 *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sb + j)) = pack_h2(pe[j], pe[j + 1]);
         }
 
-        // ---- the state entering the chunk, the chunk summary, publish
-        float Se[KT][4], dS[32];
-        tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16) + 64, dS);
-        tc_wait_ld();
+        // ---- the state entering the chunk (bounded wait on the predecessor's flag)
+        float Se[KT][4];
         int *flags = args.ctrl + 2;
         if (c > 0) {
+            const float4 *ring_in =
+                reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
             if (tid == 0) {
                 long long spins = 0;
                 while (ld_acquire(&flags[seq]) < c) {
@@ -381,31 +381,14 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
                 }
             }
             __syncthreads();
-            const float4 *src = reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
-                const float4 x = __ldcg(src + ((warp * KT + n) * 32 + lane));
+                const float4 x = __ldcg(ring_in + ((warp * KT + n) * 32 + lane));
                 Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
             }
         } else {
 #pragma unroll
             for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
-        }
-        const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
-        if (c + 1 < geo.nc && !hold) {
-            float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
-#pragma unroll
-            for (int n = 0; n < KT; ++n) {
-                const float2 gg = *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
-                float4 x;
-                x.x = fmaf(gg.x, Se[n][0], dS[4 * n + 0]);
-                x.y = fmaf(gg.y, Se[n][1], dS[4 * n + 1]);
-                x.z = fmaf(gg.x, Se[n][2], dS[4 * n + 2]);
-                x.w = fmaf(gg.y, Se[n][3], dS[4 * n + 3]);
-                __stcg(dst + ((warp * KT + n) * 32 + lane), x);
-            }
-            __syncthreads();
-            if (tid == 0) st_release(&flags[seq], c + 1);
         }
         // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value columns)
 #pragma unroll
@@ -436,6 +419,29 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
                              umma_desc_sw128(aSP + 32 * ks, 16, 1024), id_qs, 1);
             }
             umma_commit(mbar);
+        }
+
+        // ---- publish S_leave = diag(gamma_c) S_enter + dS while the output MMA runs
+        {
+            float dS[32];
+            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16) + 64, dS);
+            tc_wait_ld();
+            const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
+            if (c + 1 < geo.nc && !hold) {
+                float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
+#pragma unroll
+                for (int n = 0; n < KT; ++n) {
+                    const float2 gg = *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
+                    float4 x;
+                    x.x = fmaf(gg.x, Se[n][0], dS[4 * n + 0]);
+                    x.y = fmaf(gg.y, Se[n][1], dS[4 * n + 1]);
+                    x.z = fmaf(gg.x, Se[n][2], dS[4 * n + 2]);
+                    x.w = fmaf(gg.y, Se[n][3], dS[4 * n + 3]);
+                    __stcg(dst + ((warp * KT + n) * 32 + lane), x);
+                }
+                __syncthreads();
+                if (tid == 0) st_release(&flags[seq], c + 1);
+            }
         }
         if (!mbar_wait(mbar, 1, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
         tc_fence_after();

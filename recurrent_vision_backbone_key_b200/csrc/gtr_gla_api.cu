@@ -200,10 +200,34 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     int sms = 0;
     if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
     const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
-    if (tcgen05 && tcgen05_shape(geo))
+    // The tcgen05 kernel does one chunk per tile: use it when sequences are
+    // many (the explicit schedule forces it for its shape).
+    if (tcgen05_shape(geo) && (tcgen05 || !pair))
         e = launch_fused_umma(a, st);
     else
         e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
+}
+
+// The fused schedule on the mma.sync kernels only (one or two chunks per tile).
+gtr_status_t run_fused_mma(const __half *q, const __half *k, const __half *v, const float *g,
+                           const Geom &geo, __half *out, cudaStream_t st) {
+    void *ws = nullptr;
+    gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
+    if (s != GTR_OK) return s;
+    unsigned *status = nullptr;
+    if ((s = status_word(&status)) != GTR_OK) return s;
+    TcArgs a = make_args(q, k, v, g, geo);
+    a.out = out;
+    a.ctrl = static_cast<int *>(ws);
+    a.ring = reinterpret_cast<float *>(static_cast<char *>(ws) + fused_ctrl_bytes(geo));
+    a.status = status;
+    cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
+    if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
+    int sms = 0;
+    if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
+    const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
+    e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 
@@ -267,6 +291,8 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     __half *ho = static_cast<__half *>(out);
     if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
+    // GTR_SCHED_FUSED keeps the mma.sync kernels; AUTO lets run_fused choose.
+    if (schedule == GTR_SCHED_FUSED) return run_fused_mma(hq, hk, hv, g, geo, ho, st);
     return run_fused(hq, hk, hv, g, geo, ho, st, -1, -1, kSpinLimit, schedule == GTR_SCHED_FUSED_TCGEN05);
 }
 

@@ -15,7 +15,7 @@ from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, s
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["fused", "fused_tcgen05", "three_phase", "three_phase_simt"]
+SCHEDULES = ["auto", "fused", "fused_tcgen05", "three_phase", "three_phase_simt"]
 
 
 @pytest.fixture(scope="module", autouse=True)
