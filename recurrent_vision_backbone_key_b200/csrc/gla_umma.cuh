@@ -25,8 +25,8 @@
 // Operands live in shared memory as 64 x 64 fp16 row-major tiles with 128-byte
 // rows in the 128-byte swizzled canonical layout (16-byte chunk j of row r
 // stored at chunk j ^ (r mod 8)), read as K-major or MN-major by the MMA
-// descriptors.  Accumulators: TMEM columns [0,64) hold A and then O, columns
-// [64,128) hold dS^T; with M = 64, row m sits in TMEM lane (m mod 16) + 32 (m / 16),
+// descriptors.  Accumulators: 64 TMEM columns hold A, then dS^T, then O (three
+// MMA rounds); with M = 64, row m sits in TMEM lane (m mod 16) + 32 (m / 16),
 // so warp w reads rows 16w..16w+15 with the 16x256b load, in the m16n8
 // accumulator-fragment layout.
 #pragma once
@@ -139,7 +139,7 @@ struct UmmaLayout {
 };
 
 // ---------------------------------------------------------------- the kernel
-__global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
+__global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
     using L = UmmaLayout;
     constexpr int DK = 64, DV = 64, C = 64, KT = 8;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
 
     // ---- tensor memory first (before the ticket: a CTA waiting for TMEM holds no ticket)
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;\n" ::"r"(base_addr + L::MISC + 8)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;\n" ::"r"(base_addr + L::MISC + 8)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
@@ -276,22 +276,18 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMAs: A = qh ke^T (whole-chunk form only), dS^T = V^T ke
-        if (tid == 0) {
+        // Three MMA rounds through the same 64 TMEM columns: A, then dS^T,
+        // then O.  `phase` is the parity of the next mbarrier completion.
+        uint32_t phase = 0;
+        const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
+        // ---- round 1: A = qh ke^T (whole-chunk form only)
+        if (!exact && tid == 0) {
             tc_fence_after();
-            const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
-            if (!exact) {
-                const uint32_t id = umma_idesc_f16(0, 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024),
-                             id, ks > 0);
-            }
-            const uint32_t id2 = umma_idesc_f16(1, 1);
+            const uint32_t id = umma_idesc_f16(0, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tmem + 64, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
-                         umma_desc_sw128(aKE + 2048 * ks, 8192, 1024), id2, ks > 0);
+                umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024), id,
+                         ks > 0);
             umma_commit(mbar);
         }
 
@@ -339,10 +335,11 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
             }
         }
 
-        // ---- wait for the MMAs, write the masked scores P (fp16, swizzled)
-        if (!mbar_wait(mbar, 0, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
-        tc_fence_after();
+        // ---- write the masked scores P (fp16, swizzled)
         if (!exact) {
+            if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+            phase ^= 1u;
+            tc_fence_after();
             float a[32];
             tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
             tc_wait_ld();
@@ -362,6 +359,20 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
                 *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sb + j)) = pack_h2(pe[j], pe[j + 1]);
+        }
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();  // A read by every warp; P written
+
+        // ---- round 2: dS^T = V^T ke into the same columns, while the boundary state is fetched
+        if (tid == 0) {
+            tc_fence_after();
+            const uint32_t id2 = umma_idesc_f16(1, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                umma_f16(tmem, umma_desc_sw128(aV + 2048 * ks, 8192, 1024), umma_desc_sw128(aKE + 2048 * ks, 8192, 1024),
+                         id2, ks > 0);
+            umma_commit(mbar);
         }
 
         // ---- the state entering the chunk (bounded wait on the predecessor's flag)
@@ -398,15 +409,21 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
         }
+        // ---- the chunk summary dS^T (round 2)
+        float dS[32];
+        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        phase ^= 1u;
+        tc_fence_after();
+        tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), dS);
+        tc_wait_ld();
         fence_async_shared();
         tc_fence_before();
-        __syncthreads();
+        __syncthreads();  // S' written; dS^T read by every warp
 
-        // ---- O = P V + qh S'  (overwrites A's columns; A has been read)
+        // ---- round 3: O = P V + qh S' into the same columns
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t aP = base_addr + L::P, aV = base_addr + L::V, aQH = base_addr + L::QH,
-                           aSP = base_addr + L::SP;
+            const uint32_t aP = base_addr + L::P, aSP = base_addr + L::SP;
             const uint32_t id_pv = umma_idesc_f16(0, 1), id_qs = umma_idesc_f16(0, 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
@@ -423,9 +440,6 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
 
         // ---- publish S_leave = diag(gamma_c) S_enter + dS while the output MMA runs
         {
-            float dS[32];
-            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16) + 64, dS);
-            tc_wait_ld();
             const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
             if (c + 1 < geo.nc && !hold) {
                 float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
@@ -443,7 +457,8 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
                 if (tid == 0) st_release(&flags[seq], c + 1);
             }
         }
-        if (!mbar_wait(mbar, 1, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        phase ^= 1u;
         tc_fence_after();
 
         // ---- store O: fragments -> swizzled staging (the P / S' region) -> 16-byte rows
@@ -472,7 +487,7 @@ __global__ void __launch_bounds__(128, 4) gla_umma_kernel(const TcArgs args) {
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;\n" ::"r"(tmem) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;\n" ::"r"(tmem) : "memory");
     }
 }
 
