@@ -164,10 +164,11 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
+    // the ticket comes from warp 1, so its round trip overlaps the allocation
+    if (tid == 32) misc[0] = atomicAdd(&args.ctrl[0], 1);
     if (tid == 0) {
         mbar_init(mbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        misc[0] = atomicAdd(&args.ctrl[0], 1);
         misc[1] = 0;
     }
     tc_fence_before();
@@ -461,23 +462,26 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
         phase ^= 1u;
         tc_fence_after();
 
-        // ---- store O: fragments -> swizzled staging (the P / S' region) -> 16-byte rows
+        // ---- store O: each warp stages its own 16 rows (swizzled, in the
+        // finished P / S' region) and writes them as 16-byte row pieces
         {
             float o[32];
             tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), o);
             tc_wait_ld();
-            unsigned char *st = base + L::G;  // P / S' are consumed by the finished MMA
+            unsigned char *st = base + L::G;
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
                 const int t = 16 * warp + tr, col = 8 * n + kc;
                 *reinterpret_cast<uint32_t *>(st + sw128(t, col)) = pack_h2(o[4 * n], o[4 * n + 1]);
                 *reinterpret_cast<uint32_t *>(st + sw128(t + 8, col)) = pack_h2(o[4 * n + 2], o[4 * n + 3]);
             }
-            __syncthreads();
-            for (int idx = tid; idx < len * 8; idx += 128) {
-                const int t = idx >> 3, j = idx & 7;
-                *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
-                    *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
+                if (t < len)
+                    *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
+                        *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
             }
         }
     }
