@@ -58,7 +58,7 @@ struct TcArgs {
     float *gamma;          // SUMMARY: [nseq][nc][dk]
     const float *S_enter;  // OUTPUT:  [nseq][nc][dk][dv]
     __half *out;           // OUTPUT / FUSED
-    int *ctrl;             // FUSED: [0] ticket, [1] unused, then nseq flags; zeroed before each launch
+    int *ctrl;             // FUSED: [0] ticket, [1] unused, then 4 flags per sequence; zeroed before each launch
     float *ring;           // FUSED: [nseq][2][dk*dv] fragment-ordered states
     unsigned *status;      // FUSED: device status word (GTR_ERR_TIMEOUT on a give-up)
     long long spin_limit;  // FUSED: polls before a wait gives up

@@ -119,27 +119,40 @@ __device__ __forceinline__ uint32_t sw128(int row, int col) {
     return (uint32_t)(row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + ((col & 7) << 1));
 }
 
+// 16 TMEM lanes x 32 fp32 columns -> 16 registers (four 8-column tiles).
+__device__ __forceinline__ void tmem_ld_16x32(uint32_t taddr, float (&r)[16]) {
+    uint32_t *u = reinterpret_cast<uint32_t *>(r);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+        : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+          "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+        : "r"(taddr));
+}
+
 // ---------------------------------------------------------------- layout
 struct UmmaLayout {
-    // all offsets relative to a 1024-byte aligned base
-    static constexpr uint32_t QH = 0;          // raw q rows, then the qh (or qe) tile in place
-    static constexpr uint32_t KE = 8192;       // raw k rows, then the ke tile in place
-    static constexpr uint32_t RQ = QH;
-    static constexpr uint32_t RK = KE;
+    // all offsets relative to a 1024-byte aligned base; every tile is swizzled
+    static constexpr uint32_t QH = 0;          // raw q, then the qh (or qe) tile in place
+    static constexpr uint32_t KE = 8192;       // raw k, then the ke tile in place; then S'^T
+    static constexpr uint32_t SP = KE;         // (scaled entering state)^T, rows = value columns,
+                                               // written once the summary MMA has read ke
     static constexpr uint32_t V = 16384;       // v tile (also read as MN-major)
-    static constexpr uint32_t G = 24576;       // raw g rows fp32 [64][64] (16 KB); then the exact
-                                               // path's staging; then P + S'; then the output staging
-    static constexpr uint32_t P = G;           // masked scores
-    static constexpr uint32_t SP = G + 8192;   // (scaled entering state)^T, rows = value columns
-    static constexpr uint32_t VEC = 40960;     // gamma_c[64], sc[64], sub-chunk totals [4][64] (fp32)
+    static constexpr uint32_t P = 24576;       // exact path's staging, then the masked scores,
+                                               // then the output staging
+    static constexpr uint32_t VEC = 32768;     // gamma_c[64], sc[64], sub-chunk totals [4][64] (fp32)
     static constexpr uint32_t ROW = VEC + 6 * 64 * 4;  // int64 [64]
-    static constexpr uint32_t MISC = ROW + 64 * 8;     // tile, exact flag, tmem base, mbarrier (8-aligned)
+    static constexpr uint32_t MISC = ROW + 64 * 8;     // tile, tmem base, mbarrier (8-aligned)
     static constexpr uint32_t BYTES = MISC + 64;
     static constexpr uint32_t ALLOC = BYTES + 1024;    // slack for aligning the base
 };
 
 // ---------------------------------------------------------------- the kernel
-__global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
+// Chain of boundary states: warp w owns value rows 16w..16w+15 of S^T (its
+// TMEM lanes), and that slice of S_leave depends only on the same slice of
+// S_enter and of dS.  So each warp waits for, reads and publishes its own
+// slice, with one flag per (sequence, warp): no CTA barrier on the chain.
+__global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     using L = UmmaLayout;
     constexpr int DK = 64, DV = 64, C = 64, KT = 8;
     extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -154,7 +167,7 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
     float *vSc = vGc + 64;
     float *vTot = vSc + 64;  // [4][64]
     int64_t *sRow = reinterpret_cast<int64_t *>(base + L::ROW);
-    int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [1] exact [2] tmem base; mbar at +16
+    int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [2] tmem base; mbar at +16
     const uint32_t mbar = base_addr + L::MISC + 16;
     const int nseq = geo.B * geo.heads;
 
@@ -169,7 +182,6 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
     if (tid == 0) {
         mbar_init(mbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
-        misc[1] = 0;
     }
     tc_fence_before();
     __syncthreads();
@@ -193,45 +205,39 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
                                     : (int64_t)-1;
         __syncthreads();
 
-        // ---- stage q, k, g rows (raw) and v (swizzled operand tile), one cp.async batch
+        // ---- q, k, v rows into swizzled tiles (one cp.async batch)
         for (int idx = tid; idx < C * 8; idx += 128) {
             const int t = idx >> 3, j = idx & 7;
             const int64_t r = sRow[t];
             const int64_t o = (r < 0 ? 0 : r) * 64 + j * 8;
-            cp_async16(base + L::RQ + t * 128 + j * 16, args.q + o, r >= 0);
-            cp_async16(base + L::RK + t * 128 + j * 16, args.k + o, r >= 0);
-            cp_async16(base + L::V + t * 128 + (((j ^ (t & 7)) & 7) << 4), args.v + o, r >= 0);
-        }
-        for (int idx = tid; idx < C * 16; idx += 128) {
-            const int t = idx >> 4, j = idx & 15;
-            const int64_t r = sRow[t];
-            cp_async16(base + L::G + t * 256 + j * 16, args.g + (r < 0 ? 0 : r) * 64 + j * 4, r >= 0);
+            const uint32_t so = t * 128 + (((j ^ (t & 7)) & 7) << 4);
+            cp_async16(base + L::QH + so, args.q + o, r >= 0);
+            cp_async16(base + L::KE + so, args.k + o, r >= 0);
+            cp_async16(base + L::V + so, args.v + o, r >= 0);
         }
         cp_async_commit();
-        cp_async_wait_all();
-        __syncthreads();
 
-        // ---- operand prep: task (dim pair dp, sub-chunk u), 16 tokens each
-        const int dp = tid & 31, u = tid >> 5;
-        const int d0 = 2 * dp;
-        __half2 qv[16], kv[16];
+        // ---- g straight into registers: warp u takes sub-chunk u (tokens
+        // 16u..16u+15), lane dp the key dims (2dp, 2dp+1); one 256-byte row
+        // per warp load.  a_t = exp(g_t); padding rows get g = 0 (a = 1).
+        const int u = warp, d0 = 2 * lane;
         float2 av[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
-            const int row = 16 * u + t;
-            qv[t] = *reinterpret_cast<const __half2 *>(base + L::RQ + row * 128 + d0 * 2);
-            kv[t] = *reinterpret_cast<const __half2 *>(base + L::RK + row * 128 + d0 * 2);
-            const float2 gv = *reinterpret_cast<const float2 *>(base + L::G + row * 256 + d0 * 4);
-            av[t] = make_float2(ex2(gv.x * kLog2e), ex2(gv.y * kLog2e));
+            const int64_t r = sRow[16 * u + t];
+            av[t] = r >= 0 ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * 64 + d0)) : make_float2(0.f, 0.f);
         }
         float2 tot = make_float2(1.f, 1.f);
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
+            av[t] = make_float2(ex2(av[t].x * kLog2e), ex2(av[t].y * kLog2e));
             tot.x *= av[t].x;
             tot.y *= av[t].y;
         }
         *reinterpret_cast<float2 *>(vTot + u * 64 + d0) = tot;
-        __syncthreads();  // sub-chunk totals visible; raw q / k / g all read
+        cp_async_wait_all();
+        __syncthreads();  // sub-chunk totals and the q, k, v tiles visible
+
         float2 Ebase = make_float2(1.f, 1.f), Sbase = make_float2(1.f, 1.f), gam = make_float2(1.f, 1.f);
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
@@ -241,41 +247,41 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
             gam.x *= tw.x;
             gam.y *= tw.y;
         }
+        // Every warp covers all 64 key dims with the same products, so the
+        // vote is the same in every warp.
         const float lo = 3.3546263e-4f;  // e^-kChunkRange
+        const bool gam_ok = __all_sync(0xffffffffu, gam.x >= lo && gam.y >= lo && gam.x <= 1.f / lo &&
+                                                        gam.y <= 1.f / lo);
+        // qh = q~ E_t / gamma_c (whole-chunk form) or qe = q~ E_t, in place
+        const float2 rg = gam_ok ? make_float2(qscale / gam.x, qscale / gam.y) : make_float2(qscale, qscale);
         __half2 qmax = __float2half2_rn(0.f);
+        {
+            float2 E = Ebase;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) qmax = __hmax2(qmax, __habs2(qv[t]));
+            for (int t = 0; t < 16; ++t) {
+                __half2 *p = reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0));
+                const __half2 qv = *p;
+                qmax = __hmax2(qmax, __habs2(qv));
+                E.x *= av[t].x;
+                E.y *= av[t].y;
+                *p = __hmul2(qv, __floats2half2_rn(E.x * rg.x, E.y * rg.y));
+            }
+            float2 S = Sbase;  // decay after token t to the chunk end
+#pragma unroll
+            for (int t = 15; t >= 0; --t) {
+                __half2 *p = reinterpret_cast<__half2 *>(base + L::KE + sw128(16 * u + t, d0));
+                *p = __hmul2(*p, __floats2half2_rn(S.x, S.y));
+                S.x *= av[t].x;
+                S.y *= av[t].y;
+            }
+        }
         const float2 qm = __half22float2(qmax);
-        const bool fast = gam.x >= lo && gam.y >= lo && gam.x <= 1.f / lo && gam.y <= 1.f / lo &&
-                          fmaxf(qm.x, qm.y) * qscale <= 16.f;
-        if (!fast) misc[1] = 1;
-        if (u == 0) {
-            *reinterpret_cast<float2 *>(vGc + d0) = gam;
-        }
-        __syncthreads();
-        const bool exact = misc[1] != 0;
-        // qh = q~ E_t / gamma_c (whole-chunk form) or qe = q~ E_t (exact form)
-        const float2 rg = exact ? make_float2(1.f, 1.f) : make_float2(1.f / gam.x, 1.f / gam.y);
-        if (u == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
-        float2 E = Ebase;
-#pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            E.x *= av[t].x;
-            E.y *= av[t].y;
-            *reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0)) =
-                __hmul2(qv[t], __floats2half2_rn(E.x * rg.x * qscale, E.y * rg.y * qscale));
-        }
-        float2 S = Sbase;  // decay after token t to the chunk end
-#pragma unroll
-        for (int t = 15; t >= 0; --t) {
-            *reinterpret_cast<__half2 *>(base + L::KE + sw128(16 * u + t, d0)) =
-                __hmul2(kv[t], __floats2half2_rn(S.x, S.y));
-            S.x *= av[t].x;
-            S.y *= av[t].y;
-        }
+        if (warp == 0) *reinterpret_cast<float2 *>(vGc + d0) = gam;
         fence_async_shared();
         tc_fence_before();
-        __syncthreads();
+        // the whole-chunk form needs the gate range and |q~| <= 16 (qh then fits fp16)
+        const bool exact = __syncthreads_or(!gam_ok || fmaxf(qm.x, qm.y) * qscale > 16.f) != 0;
+        if (warp == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
 
         // Three MMA rounds through the same 64 TMEM columns: A, then dS^T,
         // then O.  `phase` is the parity of the next mbarrier completion.
@@ -295,42 +301,59 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
         // ---- exact form: the score matrix on CUDA cores from the raw operands
         float pe[32];
         if (exact) {
+            if (gam_ok) {
+                // qh was written with 1 / gamma_c: rewrite qe = q~ E_t from the raw rows
+                float2 E = Ebase;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int64_t r = sRow[16 * u + t];
+                    const float2 gv = r >= 0 ? *reinterpret_cast<const float2 *>(args.g + r * 64 + d0)
+                                             : make_float2(0.f, 0.f);
+                    const __half2 qv = r >= 0 ? *reinterpret_cast<const __half2 *>(args.q + r * 64 + d0)
+                                              : __float2half2_rn(0.f);
+                    E.x *= ex2(gv.x * kLog2e);
+                    E.y *= ex2(gv.y * kLog2e);
+                    *reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0)) =
+                        __hmul2(qv, __floats2half2_rn(E.x * qscale, E.y * qscale));
+                }
+                fence_async_shared();
+            }
             // thread -> query row t = tid / 2, keys s in [32*(tid&1), +32)
             const int t = tid >> 1, sb = 32 * (tid & 1);
 #pragma unroll
             for (int j = 0; j < 32; ++j) pe[j] = 0.f;
-            // log2-domain in-chunk prefix of g, two halves of 32 dims, staged
-            // in the raw g region (consumed above)
-            __half *xq = reinterpret_cast<__half *>(base + L::G);          // [64][32]
-            __half *xk = reinterpret_cast<__half *>(base + L::G + 4096);   // [64][32]
-            float *xb = reinterpret_cast<float *>(base + L::G + 8192);     // [64][32]
-            for (int hd = 0; hd < 2; ++hd) {
+            // log2-domain in-chunk prefix of g, four quarters of 16 dims,
+            // staged in the (not yet used) score region
+            __half *xq = reinterpret_cast<__half *>(base + L::P);          // [64][16]
+            __half *xk = reinterpret_cast<__half *>(base + L::P + 2048);   // [64][16]
+            float *xb = reinterpret_cast<float *>(base + L::P + 4096);     // [64][16]
+            for (int hd = 0; hd < 4; ++hd) {
                 __syncthreads();
-                for (int idx = tid; idx < 64 * 32; idx += 128) {
-                    const int tt = idx >> 5, d = idx & 31;
+                for (int idx = tid; idx < 64 * 16; idx += 128) {
+                    const int tt = idx >> 4, d = idx & 15;
                     const int64_t r = sRow[tt];
-                    const int64_t o = (r < 0 ? 0 : r) * 64 + 32 * hd + d;
+                    const int64_t o = (r < 0 ? 0 : r) * 64 + 16 * hd + d;
                     xq[idx] = r >= 0 ? args.q[o] : __float2half(0.f);
                     xk[idx] = r >= 0 ? args.k[o] : __float2half(0.f);
                     xb[idx] = r >= 0 ? args.g[o] * kLog2e : 0.f;
                 }
                 __syncthreads();
-                if (tid < 32) {
+                if (tid < 16) {
                     float acc = 0.f;
                     for (int tt = 0; tt < 64; ++tt) {
-                        acc += xb[tt * 32 + tid];
-                        xb[tt * 32 + tid] = acc;
+                        acc += xb[tt * 16 + tid];
+                        xb[tt * 16 + tid] = acc;
                     }
                 }
                 __syncthreads();
-                for (int d = 0; d < 32; ++d) {
-                    const float qq = __half2float(xq[t * 32 + d]) * qscale;
-                    const float bt = xb[t * 32 + d];
+                for (int d = 0; d < 16; ++d) {
+                    const float qq = __half2float(xq[t * 16 + d]) * qscale;
+                    const float bt = xb[t * 16 + d];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int s = sb + j;
                         if (s <= t)
-                            pe[j] = fmaf(qq * __half2float(xk[s * 32 + d]), ex2(bt - xb[s * 32 + d]), pe[j]);
+                            pe[j] = fmaf(qq * __half2float(xk[s * 16 + d]), ex2(bt - xb[s * 16 + d]), pe[j]);
                     }
                 }
             }
@@ -355,7 +378,7 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
                 }
             }
         } else {
-            __syncthreads();  // the exact path's staging (in the P / S' region) is consumed
+            __syncthreads();  // the exact path's staging (in the score region) is consumed
             const int t = tid >> 1, sb = 32 * (tid & 1);
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
@@ -376,15 +399,16 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
             umma_commit(mbar);
         }
 
-        // ---- the state entering the chunk (bounded wait on the predecessor's flag)
+        // ---- this warp's slice of the state entering the chunk (bounded
+        // wait on the predecessor's flag for the same slice)
         float Se[KT][4];
-        int *flags = args.ctrl + 2;
+        int *flag = args.ctrl + 2 + (int64_t)seq * 4 + warp;
         if (c > 0) {
             const float4 *ring_in =
                 reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
-            if (tid == 0) {
+            if (lane == 0) {
                 long long spins = 0;
-                while (ld_acquire(&flags[seq]) < c) {
+                while (ld_acquire(flag) < c) {
                     if (++spins > args.spin_limit) {
                         atomicOr(args.status, 6u);  // GTR_ERR_TIMEOUT
                         break;
@@ -392,7 +416,7 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
                     __nanosleep(spins < 64 ? 32 : 256);
                 }
             }
-            __syncthreads();
+            __syncwarp();
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
                 const float4 x = __ldcg(ring_in + ((warp * KT + n) * 32 + lane));
@@ -402,7 +426,41 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
         }
-        // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value columns)
+        // ---- the chunk summary dS^T (round 2); publish this warp's slice of
+        // S_leave = diag(gamma_c) S_enter + dS, half the columns at a time
+        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        phase ^= 1u;
+        tc_fence_after();
+        {
+            const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
+            const bool publish = c + 1 < geo.nc && !hold;
+            float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                float dS[16];
+                tmem_ld_16x32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * hf, dS);
+                tc_wait_ld();
+                if (publish) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        const int n = 4 * hf + m;
+                        const float2 gg = *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
+                        float4 x;
+                        x.x = fmaf(gg.x, Se[n][0], dS[4 * m + 0]);
+                        x.y = fmaf(gg.y, Se[n][1], dS[4 * m + 1]);
+                        x.z = fmaf(gg.x, Se[n][2], dS[4 * m + 2]);
+                        x.w = fmaf(gg.y, Se[n][3], dS[4 * m + 3]);
+                        __stcg(dst + ((warp * KT + n) * 32 + lane), x);
+                    }
+                }
+            }
+            if (publish) {
+                __syncwarp();
+                if (lane == 0) st_release(flag, c + 1);
+            }
+        }
+        // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value
+        // columns), over ke (the summary MMA is complete)
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
             const float2 sc = *reinterpret_cast<const float2 *>(vSc + 8 * n + kc);
@@ -410,13 +468,6 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
         }
-        // ---- the chunk summary dS^T (round 2)
-        float dS[32];
-        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
-        phase ^= 1u;
-        tc_fence_after();
-        tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), dS);
-        tc_wait_ld();
         fence_async_shared();
         tc_fence_before();
         __syncthreads();  // S' written; dS^T read by every warp
@@ -438,37 +489,17 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
             }
             umma_commit(mbar);
         }
-
-        // ---- publish S_leave = diag(gamma_c) S_enter + dS while the output MMA runs
-        {
-            const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
-            if (c + 1 < geo.nc && !hold) {
-                float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
-#pragma unroll
-                for (int n = 0; n < KT; ++n) {
-                    const float2 gg = *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
-                    float4 x;
-                    x.x = fmaf(gg.x, Se[n][0], dS[4 * n + 0]);
-                    x.y = fmaf(gg.y, Se[n][1], dS[4 * n + 1]);
-                    x.z = fmaf(gg.x, Se[n][2], dS[4 * n + 2]);
-                    x.w = fmaf(gg.y, Se[n][3], dS[4 * n + 3]);
-                    __stcg(dst + ((warp * KT + n) * 32 + lane), x);
-                }
-                __syncthreads();
-                if (tid == 0) st_release(&flags[seq], c + 1);
-            }
-        }
         if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
         phase ^= 1u;
         tc_fence_after();
 
         // ---- store O: each warp stages its own 16 rows (swizzled, in the
-        // finished P / S' region) and writes them as 16-byte row pieces
+        // finished score region) and writes them as 16-byte row pieces
         {
             float o[32];
             tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), o);
             tc_wait_ld();
-            unsigned char *st = base + L::G;
+            unsigned char *st = base + L::P;
 #pragma unroll
             for (int n = 0; n < 8; ++n) {
                 const int t = 16 * warp + tr, col = 8 * n + kc;
@@ -498,6 +529,9 @@ __global__ void __launch_bounds__(128, 5) gla_umma_kernel(const TcArgs args) {
 inline cudaError_t launch_umma(const TcArgs &a, cudaStream_t st) {
     const size_t smem = UmmaLayout::ALLOC;
     cudaError_t e = cudaFuncSetAttribute(gla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    // six CTAs of ~36 KB per SM: ask for the largest shared-memory carveout
+    e = cudaFuncSetAttribute(gla_umma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     const unsigned grid = (unsigned)((int64_t)a.geo.nc * a.geo.B * a.geo.heads);
     gla_umma_kernel<<<grid, 128, smem, st>>>(a);

@@ -129,9 +129,10 @@ size_t three_phase_ws(const Geom &g) {
            align256(nseq * g.nc * g.dk * sizeof(float));
 }
 
-// Fused kernel: control words (ticket, exit count, one flag per sequence)
+// Fused kernels: control words (ticket, unused, four flags per sequence: the
+// mma.sync kernel uses one per sequence, the tcgen05 kernel one per warp)
 // then a two-slot ring of boundary states per sequence.
-size_t fused_ctrl_bytes(const Geom &g) { return align256(((size_t)g.B * g.heads + 2) * sizeof(int)); }
+size_t fused_ctrl_bytes(const Geom &g) { return align256(((size_t)g.B * g.heads * 4 + 2) * sizeof(int)); }
 size_t fused_ws(const Geom &g) {
     return fused_ctrl_bytes(g) + (size_t)g.B * g.heads * 2 * g.dk * g.dv * sizeof(float);
 }
