@@ -50,16 +50,41 @@ def measured_peaks():
         return 6650.0, 1590.0, "fallback"
 
 
-def profiled_traffic(w, schedule):
-    """DRAM bytes per launch of the fused kernel from the committed ncu summary,
+# Committed ncu summaries: (file, kernel sources hashed into it) per kernel.
+PROFILE_SUMMARIES = {
+    "gla_umma_kernel": ("gla_umma_fused_d64_batched.md", ("gla_umma.cuh", "gla_tc.cuh", "gla_common.cuh")),
+    "gla_tc_kernel<64,64,FUSED,1>": ("gla_tc_fused_d64_batched.md", ("gla_tc.cuh", "gla_common.cuh")),
+}
+
+
+def fused_kernel_name(w, schedule):
+    """The kernel the fused schedules launch for this workload (the library's
+    dispatch: tcgen05 for d_k = d_v = 64 and chunk 64 when sequences are at
+    least twice the SM count, or when asked for; else the mma.sync kernel, one
+    or two chunks per tile)."""
+    nseq = w.B * w.heads
+    sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    pair = nseq < 2 * sms
+    tc5_shape = w.d_k == 64 and w.d_v == 64 and w.chunk == 64
+    if schedule == "fused_tcgen05" or (schedule == "auto" and tc5_shape and not pair):
+        return "gla_umma_kernel"
+    mode = "FUSED_PAIR" if pair else "FUSED"
+    return f"gla_tc_kernel<{w.d_k},{w.d_v},{mode},{2 if pair else 1}>"
+
+
+def profiled_traffic(w, kernel):
+    """DRAM bytes per launch of the given kernel from the committed ncu summary,
     if that summary was taken on this workload from the current kernel source."""
     import hashlib
-    prof = os.path.join(ROOT, "profiles", "gla_tc_fused_d64_batched.md")
-    if w.name != "batched" or schedule not in ("auto", "fused") or not os.path.exists(prof):
+    if w.name != "batched" or kernel not in PROFILE_SUMMARIES:
+        return None
+    fname, sources = PROFILE_SUMMARIES[kernel]
+    prof = os.path.join(ROOT, "profiles", fname)
+    if not os.path.exists(prof):
         return None
     src = os.path.join(ROOT, "recurrent_vision_backbone_key_b200", "csrc")
     h = hashlib.sha256()
-    for f in ("gla_tc.cuh", "gla_common.cuh"):
+    for f in sources:
         with open(os.path.join(src, f), "rb") as fh:
             h.update(fh.read())
     fields = {}
@@ -277,7 +302,7 @@ def main():
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     alg_bytes = w.algorithmic_bytes()
     per_launch_ms = ms / args.steps
-    dominant = "forward step"
+    dominant = fused_kernel_name(w, args.schedule) if sched in (0, 1, 4) else "forward step"
     phase_ms = None
     if sched == 2:
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
@@ -287,7 +312,7 @@ def main():
     achieved = alg_bytes / (per_launch_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved / hbm_peak,
-                "traffic": profiled_traffic(w, args.schedule) if phase_ms is None else None,
+                "traffic": profiled_traffic(w, dominant) if phase_ms is None else None,
                 "kernel": dominant, "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
                 "algorithmic_bytes_per_launch": alg_bytes,
                 "tensor_flops_per_step": w.algorithmic_flops(),
