@@ -19,15 +19,16 @@
 //   the boundary readout.
 // qh grows like exp(chunk decay); the whole-chunk form is used when the decay
 // over the chunk is at most kChunkRange nats in every key dimension.  Other
-// chunks keep the three MMAs with the safe operands qe_t = q~_t E_t (<= |q~|)
+// chunks keep the other MMAs with the safe operands qe_t = q~_t E_t (<= |q~|)
 // and compute the score matrix exactly on CUDA cores.
 //
 // Operands live in shared memory as 64 x 64 fp16 row-major tiles with 128-byte
 // rows in the 128-byte swizzled canonical layout (16-byte chunk j of row r
 // stored at chunk j ^ (r mod 8)), read as K-major or MN-major by the MMA
-// descriptors.  Accumulators: 64 TMEM columns hold A, then dS^T, then O (three
-// MMA rounds); with M = 64, row m sits in TMEM lane (m mod 16) + 32 (m / 16),
-// so warp w reads rows 16w..16w+15 with the 16x256b load, in the m16n8
+// descriptors.  Accumulators: with M = 64, row m of an accumulator sits in TMEM
+// lane (m mod 16) + 32 (m / 16) + base, base 0 or 16, so two of them share 64
+// columns: A (base 0) and dS^T (base 16) in one MMA round, then O over A.
+// Warp w reads rows 16w..16w+15 of either with the 16x256b load, in the m16n8
 // accumulator-fragment layout.
 #pragma once
 
@@ -199,15 +200,19 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     const float qscale = rsqrtf((float)DK);
 
     if (ok_tile) {
-        // ---- row table
-        if (tid < C)
-            sRow[tid] = (tid < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + tid, geo.H, geo.W, geo.N)) * geo.heads + h
-                                    : (int64_t)-1;
-        __syncthreads();
+        // ---- row table: each warp its own 16 rows (tokens 16w..16w+15),
+        // which are the only rows it loads, preps and stores (the exact
+        // path, which reads all rows, starts with a CTA barrier)
+        if (lane < 16) {
+            const int t = 16 * warp + lane;
+            sRow[t] = (t < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
+                                : (int64_t)-1;
+        }
+        __syncwarp();
 
-        // ---- q, k, v rows into swizzled tiles (one cp.async batch)
-        for (int idx = tid; idx < C * 8; idx += 128) {
-            const int t = idx >> 3, j = idx & 7;
+        // ---- q, k, v rows into swizzled tiles (one cp.async batch per warp)
+        for (int idx = lane; idx < 16 * 8; idx += 32) {
+            const int t = 16 * warp + (idx >> 3), j = idx & 7;
             const int64_t r = sRow[t];
             const int64_t o = (r < 0 ? 0 : r) * 64 + j * 8;
             const uint32_t so = t * 128 + (((j ^ (t & 7)) & 7) << 4);
@@ -283,18 +288,28 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         const bool exact = __syncthreads_or(!gam_ok || fmaxf(qm.x, qm.y) * qscale > 16.f) != 0;
         if (warp == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
 
-        // Three MMA rounds through the same 64 TMEM columns: A, then dS^T,
-        // then O.  `phase` is the parity of the next mbarrier completion.
+        // Two MMA rounds through the same 64 TMEM columns.  Round 1: A = qh ke^T
+        // (whole-chunk form only) in TMEM lanes 0-15 of each 32-lane group and
+        // dS^T = V^T ke in lanes 16-31 (an M = 64 accumulator uses half of each
+        // group).  Round 2: O = P V + qh S' over A.  `phase` is the parity of the
+        // next mbarrier completion.
         uint32_t phase = 0;
         const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
-        // ---- round 1: A = qh ke^T (whole-chunk form only)
-        if (!exact && tid == 0) {
+        constexpr uint32_t kDsLanes = 16u << 16;
+        if (tid == 0) {
             tc_fence_after();
-            const uint32_t id = umma_idesc_f16(0, 0);
+            if (!exact) {
+                const uint32_t id = umma_idesc_f16(0, 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024),
+                             id, ks > 0);
+            }
+            const uint32_t id2 = umma_idesc_f16(1, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024), id,
-                         ks > 0);
+                umma_f16(tmem + kDsLanes, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
+                         umma_desc_sw128(aKE + 2048 * ks, 8192, 1024), id2, ks > 0);
             umma_commit(mbar);
         }
 
@@ -357,50 +372,15 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                     }
                 }
             }
-        }
-
-        // ---- write the masked scores P (fp16, swizzled)
-        if (!exact) {
-            if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
-            phase ^= 1u;
-            tc_fence_after();
-            float a[32];
-            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
-            tc_wait_ld();
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int t = 16 * warp + tr + 8 * hf, s = 8 * n + kc;
-                    const float x0 = s <= t ? a[4 * n + 2 * hf] : 0.f;
-                    const float x1 = s + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
-                    *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, s)) = pack_h2(x0, x1);
-                }
-            }
-        } else {
             __syncthreads();  // the exact path's staging (in the score region) is consumed
-            const int t = tid >> 1, sb = 32 * (tid & 1);
+            const int t2 = tid >> 1, sb2 = 32 * (tid & 1);
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-                *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sb + j)) = pack_h2(pe[j], pe[j + 1]);
-        }
-        fence_async_shared();
-        tc_fence_before();
-        __syncthreads();  // A read by every warp; P written
-
-        // ---- round 2: dS^T = V^T ke into the same columns, while the boundary state is fetched
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t id2 = umma_idesc_f16(1, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tmem, umma_desc_sw128(aV + 2048 * ks, 8192, 1024), umma_desc_sw128(aKE + 2048 * ks, 8192, 1024),
-                         id2, ks > 0);
-            umma_commit(mbar);
+                *reinterpret_cast<uint32_t *>(base + L::P + sw128(t2, sb2 + j)) = pack_h2(pe[j], pe[j + 1]);
         }
 
         // ---- this warp's slice of the state entering the chunk (bounded
-        // wait on the predecessor's flag for the same slice)
+        // wait on the predecessor's flag for the same slice), while round 1 runs
         float Se[KT][4];
         int *flag = args.ctrl + 2 + (int64_t)seq * 4 + warp;
         if (c > 0) {
@@ -426,11 +406,28 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
         }
-        // ---- the chunk summary dS^T (round 2); publish this warp's slice of
-        // S_leave = diag(gamma_c) S_enter + dS, half the columns at a time
+
         if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
         phase ^= 1u;
         tc_fence_after();
+        // ---- the masked scores P (fp16, swizzled), this warp's 16 query rows
+        if (!exact) {
+            float a[32];
+            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
+            tc_wait_ld();
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int t = 16 * warp + tr + 8 * hf, s = 8 * n + kc;
+                    const float x0 = s <= t ? a[4 * n + 2 * hf] : 0.f;
+                    const float x1 = s + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, s)) = pack_h2(x0, x1);
+                }
+            }
+        }
+        // ---- publish this warp's slice of S_leave = diag(gamma_c) S_enter + dS,
+        // half the columns at a time
         {
             const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
             const bool publish = c + 1 < geo.nc && !hold;
@@ -438,7 +435,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
                 float dS[16];
-                tmem_ld_16x32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * hf, dS);
+                tmem_ld_16x32(tmem + kDsLanes + ((uint32_t)(32 * warp) << 16) + 32 * hf, dS);
                 tc_wait_ld();
                 if (publish) {
 #pragma unroll
@@ -460,7 +457,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             }
         }
         // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value
-        // columns), over ke (the summary MMA is complete)
+        // columns), over ke (round 1 is complete)
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
             const float2 sc = *reinterpret_cast<const float2 *>(vSc + 8 * n + kc);
@@ -470,9 +467,9 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         }
         fence_async_shared();
         tc_fence_before();
-        __syncthreads();  // S' written; dS^T read by every warp
+        __syncthreads();  // P and S' written; A and dS^T read by every warp
 
-        // ---- round 3: O = P V + qh S' into the same columns
+        // ---- round 2: O = P V + qh S' over A
         if (tid == 0) {
             tc_fence_after();
             const uint32_t aP = base_addr + L::P, aSP = base_addr + L::SP;
