@@ -410,24 +410,9 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
         phase ^= 1u;
         tc_fence_after();
-        // ---- the masked scores P (fp16, swizzled), this warp's 16 query rows
-        if (!exact) {
-            float a[32];
-            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
-            tc_wait_ld();
-#pragma unroll
-            for (int n = 0; n < 8; ++n) {
-#pragma unroll
-                for (int hf = 0; hf < 2; ++hf) {
-                    const int t = 16 * warp + tr + 8 * hf, s = 8 * n + kc;
-                    const float x0 = s <= t ? a[4 * n + 2 * hf] : 0.f;
-                    const float x1 = s + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
-                    *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, s)) = pack_h2(x0, x1);
-                }
-            }
-        }
         // ---- publish this warp's slice of S_leave = diag(gamma_c) S_enter + dS,
-        // half the columns at a time
+        // half the columns at a time, as soon as round 1 is done: the chain of
+        // boundary states waits on this release
         {
             const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
             const bool publish = c + 1 < geo.nc && !hold;
@@ -454,6 +439,22 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             if (publish) {
                 __syncwarp();
                 if (lane == 0) st_release(flag, c + 1);
+            }
+        }
+        // ---- the masked scores P (fp16, swizzled), this warp's 16 query rows
+        if (!exact) {
+            float a[32];
+            tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), a);
+            tc_wait_ld();
+#pragma unroll
+            for (int n = 0; n < 8; ++n) {
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int t = 16 * warp + tr + 8 * hf, s = 8 * n + kc;
+                    const float x0 = s <= t ? a[4 * n + 2 * hf] : 0.f;
+                    const float x1 = s + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
+                    *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, s)) = pack_h2(x0, x1);
+                }
             }
         }
         // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value
