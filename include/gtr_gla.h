@@ -186,17 +186,19 @@ size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k
  * inside a kernel gave up since the last query. */
 gtr_status_t gtr_gla_get_last_device_status(void *stream);
 
-/* Test hook for the bounded wait of the fused schedule: runs
- * gtr_gla_forward_ex(..., GTR_SCHED_FUSED, ...) except that the tile of
- * sequence hold_seq (= b*heads + h), chunk hold_chunk never publishes its
- * boundary state, and each wait gives up after spin_limit polls (> 0).  The
- * successor tile then times out, records GTR_ERR_TIMEOUT in the device status
- * word (read it with gtr_gla_get_last_device_status) and the kernel still
- * finishes; its output is not meaningful.  hold_seq = -1 disables the hold. */
+/* Test hook for the bounded wait of the fused schedules: runs
+ * gtr_gla_forward_ex(..., schedule, ...) for schedule GTR_SCHED_AUTO,
+ * GTR_SCHED_FUSED or GTR_SCHED_FUSED_TCGEN05 (others: GTR_ERR_INVALID_ARG),
+ * except that the tile of sequence hold_seq (= b*heads + h), chunk hold_chunk
+ * never publishes its boundary state, and each wait gives up after spin_limit
+ * polls (> 0).  The successor tile then times out, records GTR_ERR_TIMEOUT in
+ * the device status word (read it with gtr_gla_get_last_device_status) and
+ * the kernel still finishes; its output is not meaningful.  hold_seq = -1
+ * disables the hold. */
 gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const void *v, const float *g,
                                          int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
-                                         int direction, int chunk, int hold_seq, int hold_chunk,
-                                         long long spin_limit, void *out, void *stream);
+                                         int direction, int chunk, int schedule, int hold_seq,
+                                         int hold_chunk, long long spin_limit, void *out, void *stream);
 
 /* Frees every internal workspace of every device (synchronises each device
  * that has one).  Later calls allocate again on demand. */

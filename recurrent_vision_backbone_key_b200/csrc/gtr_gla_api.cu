@@ -176,9 +176,12 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
 
 bool tcgen05_shape(const Geom &g) { return g.dk == 64 && g.dv == 64 && g.chunk == 64; }
 
+// Which kernel a fused schedule launches.
+enum FusedKernel { FK_AUTO = 0, FK_MMA = 1, FK_TCGEN05 = 2 };
+
 gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const float *g,
-                       const Geom &geo, __half *out, cudaStream_t st, int hold_seq = -1,
-                       int hold_chunk = -1, long long spin_limit = kSpinLimit, bool tcgen05 = false) {
+                       const Geom &geo, __half *out, cudaStream_t st, FusedKernel which,
+                       int hold_seq = -1, int hold_chunk = -1, long long spin_limit = kSpinLimit) {
     void *ws = nullptr;
     gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
     if (s != GTR_OK) return s;
@@ -201,35 +204,18 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     int sms = 0;
     if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
     const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
-    // The tcgen05 kernel does one chunk per tile: use it when sequences are
-    // many (the explicit schedule forces it for its shape).
-    if (tcgen05_shape(geo) && (tcgen05 || !pair))
+    // The tcgen05 kernel does one chunk per tile: the library uses it when
+    // sequences are many; FK_TCGEN05 forces it for its shape.
+    const bool tc5 = tcgen05_shape(geo) && (which == FK_TCGEN05 || (which == FK_AUTO && !pair));
+    if (tc5)
         e = launch_fused_umma(a, st);
     else
         e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 
-// The fused schedule on the mma.sync kernels only (one or two chunks per tile).
-gtr_status_t run_fused_mma(const __half *q, const __half *k, const __half *v, const float *g,
-                           const Geom &geo, __half *out, cudaStream_t st) {
-    void *ws = nullptr;
-    gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
-    if (s != GTR_OK) return s;
-    unsigned *status = nullptr;
-    if ((s = status_word(&status)) != GTR_OK) return s;
-    TcArgs a = make_args(q, k, v, g, geo);
-    a.out = out;
-    a.ctrl = static_cast<int *>(ws);
-    a.ring = reinterpret_cast<float *>(static_cast<char *>(ws) + fused_ctrl_bytes(geo));
-    a.status = status;
-    cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
-    if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
-    int sms = 0;
-    if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
-    const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
-    e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
-    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
+FusedKernel fused_kernel_for(int schedule) {
+    return schedule == GTR_SCHED_FUSED ? FK_MMA : (schedule == GTR_SCHED_FUSED_TCGEN05 ? FK_TCGEN05 : FK_AUTO);
 }
 
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
@@ -293,8 +279,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
     // GTR_SCHED_FUSED keeps the mma.sync kernels; AUTO lets run_fused choose.
-    if (schedule == GTR_SCHED_FUSED) return run_fused_mma(hq, hk, hv, g, geo, ho, st);
-    return run_fused(hq, hk, hv, g, geo, ho, st, -1, -1, kSpinLimit, schedule == GTR_SCHED_FUSED_TCGEN05);
+    return run_fused(hq, hk, hv, g, geo, ho, st, fused_kernel_for(schedule));
 }
 
 }  // namespace
@@ -480,8 +465,8 @@ gtr_status_t gtr_gla_get_last_device_status(void *stream) {
 
 gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const void *v, const float *g,
                                          int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
-                                         int direction, int chunk, int hold_seq, int hold_chunk,
-                                         long long spin_limit, void *out, void *stream) {
+                                         int direction, int chunk, int schedule, int hold_seq,
+                                         int hold_chunk, long long spin_limit, void *out, void *stream) {
     t_err[0] = '\0';
     Geom geo;
     bool empty = false;
@@ -489,10 +474,13 @@ gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const voi
     if (s != GTR_OK) return s;
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (spin_limit < 1) return fail(GTR_ERR_INVALID_ARG, "spin_limit must be positive%s");
+    if (schedule != GTR_SCHED_AUTO && schedule != GTR_SCHED_FUSED && schedule != GTR_SCHED_FUSED_TCGEN05)
+        return fail(GTR_ERR_INVALID_ARG, "schedule must be AUTO, FUSED or FUSED_TCGEN05%s");
     if (empty) return GTR_OK;
     return run_fused(static_cast<const __half *>(q), static_cast<const __half *>(k),
                      static_cast<const __half *>(v), g, geo, static_cast<__half *>(out),
-                     static_cast<cudaStream_t>(stream), hold_seq, hold_chunk, spin_limit);
+                     static_cast<cudaStream_t>(stream), fused_kernel_for(schedule), hold_seq, hold_chunk,
+                     spin_limit);
 }
 
 gtr_status_t gtr_gla_release_workspace(void) {
@@ -529,6 +517,6 @@ const char *gtr_gla_last_error(void) { return t_err; }
 
 uint64_t gtr_gla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-int gtr_gla_version(void) { return 100; }
+int gtr_gla_version(void) { return 200; }
 
 }  // extern "C"

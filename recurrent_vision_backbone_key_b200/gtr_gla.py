@@ -43,7 +43,7 @@ SIGNATURES = {
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gtr_gla_get_last_device_status": (_I, [_P]),
-    "gtr_gla_debug_forward_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+    "gtr_gla_debug_forward_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                          ctypes.c_longlong, _P, _P]),
     "gtr_gla_release_workspace": (_I, []),
     "gtr_gla_status_string": (ctypes.c_char_p, [_I]),
@@ -164,10 +164,11 @@ def gtr_gla_get_last_device_status(stream=None) -> int:
 
 
 def gtr_gla_debug_forward_fused(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
-                                hold_seq, hold_chunk, spin_limit, out, stream=None) -> int:
+                                schedule, hold_seq, hold_chunk, spin_limit, out, stream=None) -> int:
+    sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
     return load().gtr_gla_debug_forward_fused(_addr(q), _addr(k), _addr(v), _addr(g), B, heads,
                                               grid_h, grid_w, d_k, d_v, _dir(direction), chunk,
-                                              hold_seq, hold_chunk, spin_limit, _addr(out),
+                                              sched, hold_seq, hold_chunk, spin_limit, _addr(out),
                                               _stream(stream))
 
 

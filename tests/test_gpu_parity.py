@@ -234,23 +234,25 @@ def test_fused_repeated_calls_reset_control_words(oracle_mod):
     assert gtr_gla.gtr_gla_get_last_device_status() == 0
 
 
-def test_fused_bounded_wait_times_out_cleanly(oracle_mod):
+@pytest.mark.parametrize("schedule,d,chunk,H,W", [("fused", 64, 16, 8, 8), ("fused_tcgen05", 64, 64, 16, 16)])
+def test_fused_bounded_wait_times_out_cleanly(oracle_mod, schedule, d, chunk, H, W):
     """A tile that never publishes its state: the successor's wait gives up
     after the spin limit, the status word reports GTR_ERR_TIMEOUT, the
-    kernel finishes, and the next call is correct again."""
-    H, W, heads = 8, 8, 2
-    q, k, v, g = gpu_inputs(1, H, W, heads, 64, 64, seed=9)
+    kernel finishes, and the next call is correct again.  Run on the mma.sync
+    kernel and on the tcgen05 kernel (per-warp waits)."""
+    heads = 2
+    q, k, v, g = gpu_inputs(1, H, W, heads, d, d, seed=9)
     out = torch.zeros_like(v)
-    st = gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, 64, 64, 0, 16,
+    st = gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, d, d, 0, chunk, schedule,
                                              1, 1, 2000, out)
     assert st == 0
     assert gtr_gla.gtr_gla_get_last_device_status() == 6  # GTR_ERR_TIMEOUT
     assert gtr_gla.gtr_gla_get_last_device_status() == 0  # cleared by the read
-    out2 = run_forward(q, k, v, g, H, W, 0, 16, "fused")
+    out2 = run_forward(q, k, v, g, H, W, 0, chunk, schedule)
     compare(out2, oracle_full(oracle_mod, q, k, v, g, H, W, 0))
     # the hook with no hold changes nothing
     out3 = torch.zeros_like(v)
-    assert gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, 64, 64, 0, 16,
+    assert gtr_gla.gtr_gla_debug_forward_fused(q, k, v, g, 1, heads, H, W, d, d, 0, chunk, schedule,
                                                -1, -1, 1 << 22, out3) == 0
     torch.cuda.synchronize()
     assert torch.equal(out3, out2)
@@ -271,9 +273,17 @@ def test_special_gates_d64(oracle_mod, schedule):
         "mixed": torch.where(torch.rand_like(g) < 0.97, g, g * 60.0),
     }
     for name, gg in cases.items():
-        for direction in (0, 3):
+        for direction in range(4):
             out = run_forward(q, k, v, gg, H, W, direction, 64, schedule)
             compare(out, oracle_full(oracle_mod, q, k, v, gg, H, W, direction))
+    # |q~| above 16 in a few tokens with mild gates: the tcgen05 kernel
+    # rewrites those chunks' query operand without the 1/gamma_c factor
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    big = torch.rand(q.shape[:3], device="cuda", generator=gen) < 0.05
+    qb = torch.where(big[..., None], q.float() * 300.0, q.float()).half()
+    for direction in (0, 2):
+        out = run_forward(qb, k, v, g, H, W, direction, 64, schedule)
+        compare(out, oracle_full(oracle_mod, qb, k, v, g, H, W, direction))
 
 
 @pytest.mark.parametrize("direction", [0, 2])
