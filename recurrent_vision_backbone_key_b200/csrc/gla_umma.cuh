@@ -258,10 +258,11 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         const bool gam_ok = __all_sync(0xffffffffu, gam.x >= lo && gam.y >= lo && gam.x <= 1.f / lo &&
                                                         gam.y <= 1.f / lo);
         // qh = q~ E_t / gamma_c (whole-chunk form) or qe = q~ E_t, in place
-        const float2 rg = gam_ok ? make_float2(qscale / gam.x, qscale / gam.y) : make_float2(qscale, qscale);
         __half2 qmax = __float2half2_rn(0.f);
         {
-            float2 E = Ebase;
+            // E_t / gamma_c * qscale (or E_t * qscale), carried as one product
+            float2 E = gam_ok ? make_float2(Ebase.x * (qscale / gam.x), Ebase.y * (qscale / gam.y))
+                              : make_float2(Ebase.x * qscale, Ebase.y * qscale);
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
                 __half2 *p = reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0));
@@ -269,7 +270,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                 qmax = __hmax2(qmax, __habs2(qv));
                 E.x *= av[t].x;
                 E.y *= av[t].y;
-                *p = __hmul2(qv, __floats2half2_rn(E.x * rg.x, E.y * rg.y));
+                *p = __hmul2(qv, __floats2half2_rn(E.x, E.y));
             }
             float2 S = Sbase;  // decay after token t to the chunk end
 #pragma unroll
