@@ -110,10 +110,15 @@ gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, con
                                 int direction, int chunk, int schedule, void *out, void *stream);
 
 /* End-to-end call on HOST buffers: copies q, k, v, g (host) to the device,
- * runs gtr_gla_forward on `stream`, copies the result into out (host) and
- * synchronises `stream` before returning.  Layouts as gtr_gla_forward.
- * Device staging buffers come from the internal workspace.  Page-locked host
- * buffers give the fastest copies; pageable ones work too. */
+ * runs the forward (GTR_SCHED_AUTO), copies the result into out (host) and
+ * returns once out is complete.  Layouts as gtr_gla_forward.  The batch is
+ * cut into up to 8 slices of whole batch items (problems under 8 MiB of
+ * traffic run as one); each slice's upload, forward and download run on three
+ * internal streams of this (device, stream) pair, so uploads overlap the
+ * forward and the downloads of earlier slices.  Those streams start after the
+ * work queued on `stream` before the call.  Device staging buffers come from
+ * the internal workspace.  Page-locked host buffers give the fastest copies
+ * and the overlap; pageable ones work too. */
 gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, const float *g,
                                   int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                   int direction, int chunk, void *out, void *stream);

@@ -2,6 +2,7 @@
 // internal workspace, and dispatch to the kernels.  Host code only.
 #include "gtr_gla.h"
 
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -303,6 +304,37 @@ gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, con
                         schedule, out, stream);
 }
 
+// Copy/compute pipeline of the host-buffer entry point.  Every batch item is
+// one contiguous byte range of every tensor, so the batch is cut into up to
+// kHostSlices slices; slice i's upload, forward and download run on three
+// streams of their own, and the uploads of later slices overlap the forward
+// and the download of earlier ones (PCIe carries both directions at once).
+constexpr int kHostSlices = 8;
+constexpr size_t kHostSliceMinBytes = 8u << 20;  // smaller problems run as one slice
+struct HostPipe {
+    cudaStream_t up = nullptr, run = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, up_done[kHostSlices] = {}, run_done[kHostSlices] = {};
+};
+std::map<WsKey, HostPipe> g_pipes;  // (device, caller's stream); guarded by g_ws_mu
+
+cudaError_t host_pipe(int dev, cudaStream_t st, HostPipe **out) {
+    HostPipe &hp = g_pipes[WsKey{dev, st, WS_STAGING}];
+    cudaError_t e = cudaSuccess;
+    if (!hp.up) {
+        if ((e = cudaStreamCreateWithFlags(&hp.up, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&hp.run, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&hp.down, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaEventCreateWithFlags(&hp.start, cudaEventDisableTiming)) != cudaSuccess)
+            return e;
+        for (int i = 0; i < kHostSlices; ++i)
+            if ((e = cudaEventCreateWithFlags(&hp.up_done[i], cudaEventDisableTiming)) != cudaSuccess ||
+                (e = cudaEventCreateWithFlags(&hp.run_done[i], cudaEventDisableTiming)) != cudaSuccess)
+                return e;
+    }
+    *out = &hp;
+    return e;
+}
+
 gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, const float *g,
                                   int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                   int direction, int chunk, void *out, void *stream) {
@@ -314,15 +346,16 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (empty) return GTR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t bq = align256(tok_bytes(geo, d_k, 2)), bv = align256(tok_bytes(geo, d_v, 2));
-    const size_t bg = align256(tok_bytes(geo, d_k, 4));
-    // Staging for inputs and output lives in the workspace of a private
-    // key (the stream's workspace is used by the forward call itself).
+    const size_t nq = tok_bytes(geo, d_k, 2), nv = tok_bytes(geo, d_v, 2), ng = tok_bytes(geo, d_k, 4);
+    const size_t bq = align256(nq), bv = align256(nv), bg = align256(ng);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    // Staging for inputs and output lives in the workspace of a private key
+    // (the stream's workspace is used by the forward call itself).
     void *stage = nullptr;
+    HostPipe *hp = nullptr;
     {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
         size_t need = 2 * bq + 2 * bv + bg;
         std::lock_guard<std::mutex> lk(g_ws_mu);
         Workspace &w = g_ws[WsKey{dev, st, WS_STAGING}];
@@ -343,21 +376,40 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
             w.bytes = need;
         }
         stage = w.ptr;
+        if ((e = host_pipe(dev, st, &hp)) != cudaSuccess) return cuda_fail(e, "pipeline streams");
     }
     char *p = static_cast<char *>(stage);
-    void *dq = p, *dk_ = p + bq, *dv_ = p + 2 * bq, *dg = p + 2 * bq + bv, *dout = p + 2 * bq + bv + bg;
-    cudaError_t e;
-    if ((e = cudaMemcpyAsync(dq, q, tok_bytes(geo, d_k, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(dk_, k, tok_bytes(geo, d_k, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(dv_, v, tok_bytes(geo, d_v, 2), cudaMemcpyHostToDevice, st)) != cudaSuccess ||
-        (e = cudaMemcpyAsync(dg, g, tok_bytes(geo, d_k, 4), cudaMemcpyHostToDevice, st)) != cudaSuccess)
-        return cuda_fail(e, "host-to-device copy");
-    s = forward_impl(dq, dk_, dv_, static_cast<const float *>(dg), B, heads, grid_h, grid_w, d_k, d_v,
-                     direction, chunk, GTR_SCHED_AUTO, dout, stream);
-    if (s != GTR_OK) return s;
-    if ((e = cudaMemcpyAsync(out, dout, tok_bytes(geo, d_v, 2), cudaMemcpyDeviceToHost, st)) != cudaSuccess)
-        return cuda_fail(e, "device-to-host copy");
-    if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    char *dq = p, *dk_ = p + bq, *dv_ = p + 2 * bq, *dg = p + 2 * bq + bv, *dout = p + 2 * bq + bv + bg;
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k);
+    const char *hv = static_cast<const char *>(v), *hg = reinterpret_cast<const char *>(g);
+    char *hout = static_cast<char *>(out);
+    // slices of whole batch items, none below kHostSliceMinBytes of traffic
+    const size_t total = 2 * nq + 2 * nv + ng;
+    int S = (int)std::min<size_t>(std::min<size_t>((size_t)B, kHostSlices), std::max<size_t>(1, total / kHostSliceMinBytes));
+    // the uploads start after the work already queued on the caller's stream
+    if ((e = cudaEventRecord(hp->start, st)) != cudaSuccess || (e = cudaStreamWaitEvent(hp->up, hp->start, 0)) != cudaSuccess)
+        return cuda_fail(e, "pipeline start");
+    for (int i = 0; i < S; ++i) {
+        const int b0 = (int)((int64_t)B * i / S), b1 = (int)((int64_t)B * (i + 1) / S), nb = b1 - b0;
+        const size_t per_b = (size_t)geo.N * heads;  // token-heads per batch item
+        const size_t oq = (size_t)b0 * per_b * d_k * 2, ov = (size_t)b0 * per_b * d_v * 2, og = (size_t)b0 * per_b * d_k * 4;
+        const size_t sq = (size_t)nb * per_b * d_k * 2, sv = (size_t)nb * per_b * d_v * 2, sg = (size_t)nb * per_b * d_k * 4;
+        if ((e = cudaMemcpyAsync(dq + oq, hq + oq, sq, cudaMemcpyHostToDevice, hp->up)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(dk_ + oq, hk + oq, sq, cudaMemcpyHostToDevice, hp->up)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(dv_ + ov, hv + ov, sv, cudaMemcpyHostToDevice, hp->up)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(dg + og, hg + og, sg, cudaMemcpyHostToDevice, hp->up)) != cudaSuccess ||
+            (e = cudaEventRecord(hp->up_done[i], hp->up)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(hp->run, hp->up_done[i], 0)) != cudaSuccess)
+            return cuda_fail(e, "host-to-device copy");
+        s = forward_impl(dq + oq, dk_ + oq, dv_ + ov, reinterpret_cast<const float *>(dg + og), nb, heads, grid_h,
+                         grid_w, d_k, d_v, direction, chunk, GTR_SCHED_AUTO, dout + ov, hp->run);
+        if (s != GTR_OK) return s;
+        if ((e = cudaEventRecord(hp->run_done[i], hp->run)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(hp->down, hp->run_done[i], 0)) != cudaSuccess ||
+            (e = cudaMemcpyAsync(hout + ov, dout + ov, sv, cudaMemcpyDeviceToHost, hp->down)) != cudaSuccess)
+            return cuda_fail(e, "device-to-host copy");
+    }
+    if ((e = cudaStreamSynchronize(hp->down)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
     return GTR_OK;
 }
 
@@ -495,6 +547,21 @@ gtr_status_t gtr_gla_release_workspace(void) {
         }
     }
     g_ws.clear();
+    for (auto &kv : g_pipes) {
+        HostPipe &hp = kv.second;
+        cudaSetDevice(kv.first.dev);
+        if (hp.up) {
+            cudaStreamDestroy(hp.up);
+            cudaStreamDestroy(hp.run);
+            cudaStreamDestroy(hp.down);
+            cudaEventDestroy(hp.start);
+            for (int i = 0; i < kHostSlices; ++i) {
+                cudaEventDestroy(hp.up_done[i]);
+                cudaEventDestroy(hp.run_done[i]);
+            }
+        }
+    }
+    g_pipes.clear();
     cudaSetDevice(cur);
     return GTR_OK;
 }
