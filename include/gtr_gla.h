@@ -221,6 +221,22 @@ uint64_t gtr_gla_launch_count(void);
 /* ABI version: major*10000 + minor*100 + patch. */
 int gtr_gla_version(void);
 
+/* 1 if this library is the bounds-checked debug build, else 0.  The checked
+ * build (libgtr_gla_checked.so, compiled with GTR_BOUNDS_CHECK) tests every
+ * global-memory index a kernel computes at run time against its buffer's
+ * extent before the access; an index out of range is counted, the first one
+ * recorded, and the access skipped instead of made.  It is slower, and meant
+ * for tests. */
+int gtr_gla_bounds_checked(void);
+
+/* Checked build only: waits for the device (cudaDeviceSynchronize), then
+ * returns in *count the accesses skipped since the last clear, and for the
+ * first of them its site code (*site), index (*index) and the extent it broke
+ * (*limit); all zero when none.  clear != 0 resets the report.  The normal
+ * build returns GTR_ERR_INVALID_ARG with everything zero. */
+gtr_status_t gtr_gla_debug_bounds_report(unsigned long long *count, int *site, long long *index,
+                                         long long *limit, int clear);
+
 #ifdef __cplusplus
 }
 #endif

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gla_check.cuh"
+
 namespace gtr {
 
 // Problem geometry shared by every kernel.  Token layout [B][N][heads][d],

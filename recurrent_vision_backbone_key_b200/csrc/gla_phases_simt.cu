@@ -25,7 +25,8 @@ __device__ void load_rows_h(const __half *src, const Geom &g, int b, int h, int 
         float x = 0.f;
         if (t < len) {
             int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
-            x = __half2float(src[tok_offset(g, b, p, h, d) + i]);
+            const int64_t o = tok_offset(g, b, p, h, d) + i;
+            if (GTR_INB(o, (int64_t)g.B * g.N * g.heads * d, BS_SIMT_LOAD)) x = __half2float(src[o]);
         }
         dst[t * ld + i] = x;
     }
@@ -38,7 +39,8 @@ __device__ void load_rows_f(const float *src, const Geom &g, int b, int h, int t
         float x = 0.f;
         if (t < len) {
             int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
-            x = src[tok_offset(g, b, p, h, d) + i];
+            const int64_t o = tok_offset(g, b, p, h, d) + i;
+            if (GTR_INB(o, (int64_t)g.B * g.N * g.heads * d, BS_SIMT_LOAD)) x = src[o];
         }
         dst[t * ld + i] = x;
     }
@@ -77,6 +79,7 @@ __global__ void __launch_bounds__(kThreads) summary_simt_kernel(
     prefix_rows(bs, ldk, len, dk);
     __syncthreads();
     const int64_t seq = (int64_t)b * g.heads + h;
+    if (!GTR_INB(seq * g.nc + c, (int64_t)g.B * g.heads * g.nc, BS_SIMT_SUMMARY)) return;
     for (int idx = threadIdx.x; idx < len * dk; idx += blockDim.x) {
         int t = idx / dk, i = idx - t * dk;
         kw[t * ldk + i] *= expf(bs[(len - 1) * ldk + i] - bs[t * ldk + i]);
@@ -97,11 +100,12 @@ __global__ void __launch_bounds__(kThreads) summary_simt_kernel(
 // threads own consecutive elements, so every step is one coalesced sweep.
 // In place is allowed: element e of chunk c is read before it is written.
 __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
-    const float *dS, const float *__restrict__ gamma, int nc, int dk, int dv, float *S_enter) {
+    const float *dS, const float *__restrict__ gamma, int nseq, int nc, int dk, int dv, float *S_enter) {
     const int per_seq = (dk * dv + blockDim.x - 1) / blockDim.x;
     const int64_t seq = blockIdx.x / per_seq;
     const int e = (blockIdx.x % per_seq) * blockDim.x + threadIdx.x;
     if (e >= dk * dv) return;
+    if (!GTR_INB(seq, nseq, BS_SIMT_SCAN)) return;
     const int i = e / dv;
     const int64_t stride = (int64_t)dk * dv;
     const float *src = dS + seq * nc * stride + e;
@@ -141,8 +145,9 @@ __global__ void __launch_bounds__(kThreads) output_simt_kernel(
     load_rows_f(gl, g, b, h, t0, len, dk, bs, ldk);
     load_rows_h(v, g, b, h, t0, len, dv, vv, dv);
     const int64_t seq = (int64_t)b * g.heads + h;
-    const float *Sg = S_enter + (seq * g.nc + c) * (int64_t)dk * dv;
-    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[e] = Sg[e];
+    const bool s_ok = GTR_INB(seq * g.nc + c, (int64_t)g.B * g.heads * g.nc, BS_SIMT_SENTER);
+    const float *Sg = S_enter + (s_ok ? seq * g.nc + c : 0) * (int64_t)dk * dv;
+    for (int e = threadIdx.x; e < dk * dv; e += blockDim.x) S[e] = s_ok ? Sg[e] : 0.f;
     __syncthreads();
     prefix_rows(bs, ldk, len, dk);
     for (int idx = threadIdx.x; idx < C * dk; idx += blockDim.x) {
@@ -171,7 +176,8 @@ __global__ void __launch_bounds__(kThreads) output_simt_kernel(
         for (int i = 0; i < dk; ++i) acc = fmaf(qs[t * ldk + i], S[i * dv + j], acc);
         for (int s = 0; s <= t; ++s) acc = fmaf(A[t * C + s], vv[s * dv + j], acc);
         int p = scan_pos(g.dir, t0 + t, g.H, g.W, g.N);
-        out[tok_offset(g, b, p, h, dv) + j] = __float2half_rn(acc);
+        const int64_t o = tok_offset(g, b, p, h, dv) + j;
+        if (GTR_INB(o, (int64_t)g.B * g.N * g.heads * dv, BS_SIMT_OUT)) out[o] = __float2half_rn(acc);
     }
 }
 
@@ -197,7 +203,7 @@ cudaError_t launch_summary_v0(const __half *k, const __half *v, const float *g, 
 cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
                            float *S_enter, cudaStream_t st) {
     dim3 grid((unsigned)((int64_t)((dk * dv + kThreads - 1) / kThreads) * nseq));
-    scan_simt_kernel<<<grid, kThreads, 0, st>>>(dS, gamma, nc, dk, dv, S_enter);
+    scan_simt_kernel<<<grid, kThreads, 0, st>>>(dS, gamma, nseq, nc, dk, dv, S_enter);
     count_launch();
     return cudaGetLastError();
 }

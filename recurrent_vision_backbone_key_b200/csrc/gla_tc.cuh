@@ -206,6 +206,7 @@ gla_tc_kernel(const TcArgs args) {
 
     // ------------------------------------------------ which tile
     const int nseq = geo.B * geo.heads;
+    const int64_t rows = (int64_t)geo.B * geo.N * geo.heads;  // token-head rows of every tensor
     if (tid < 4 * NCH) Fl_(tid >> 2)[tid & 3] = 0;
     int tile;
     if (MODE == TC_FUSED) {
@@ -245,9 +246,11 @@ gla_tc_kernel(const TcArgs args) {
     for (int idx = tid; idx < NCH * C; idx += NT) {
         const int i = part_of(idx, C), t = idx - i * C;
         const int cc = c0 + i;
-        Row_(i)[t] = (t < chunk_len(i))
-                         ? ((int64_t)b * geo.N + scan_pos(geo.dir, cc * C + t, geo.H, geo.W, geo.N)) * geo.heads + h
-                         : (int64_t)-1;
+        int64_t r = (t < chunk_len(i))
+                        ? ((int64_t)b * geo.N + scan_pos(geo.dir, cc * C + t, geo.H, geo.W, geo.N)) * geo.heads + h
+                        : (int64_t)-1;
+        if (r >= 0 && !GTR_INB(r, rows, BS_TC_ROW)) r = -1;
+        Row_(i)[t] = r;
     }
     __syncthreads();
 
@@ -262,22 +265,24 @@ gla_tc_kernel(const TcArgs args) {
             const int i = part_of(idx, C * VCH), rem = idx - i * (C * VCH);
             const int t = rem / VCH, j = rem - t * VCH;
             const int64_t r = Row_(i)[t];
-            cp_async16(V_(i) + t * LDV + j * 8, args.v + (r < 0 ? 0 : r) * DV + j * 8, r >= 0);
+            const bool ok = r >= 0 && GTR_INB(r * DV + j * 8 + 7, rows * DV, BS_TC_LOAD);
+            cp_async16(V_(i) + t * LDV + j * 8, args.v + (ok ? r * DV + j * 8 : 0), ok);
         }
         for (int idx = tid; idx < NCH * C * QCH; idx += NT) {
             const int i = part_of(idx, C * QCH), rem = idx - i * (C * QCH);
             const int t = rem / QCH, j = rem - t * QCH;
             const int64_t r = Row_(i)[t];
-            const int64_t o = (r < 0 ? 0 : r) * DK + j * 8;
-            if (MODE != TC_SUMMARY) cp_async16(Q_(i) + t * LDK + j * 8, args.q + o, r >= 0);
-            cp_async16(K_(i) + t * LDK + j * 8, args.k + o, r >= 0);
+            const bool ok = r >= 0 && GTR_INB(r * DK + j * 8 + 7, rows * DK, BS_TC_LOAD);
+            const int64_t o = ok ? r * DK + j * 8 : 0;
+            if (MODE != TC_SUMMARY) cp_async16(Q_(i) + t * LDK + j * 8, args.q + o, ok);
+            cp_async16(K_(i) + t * LDK + j * 8, args.k + o, ok);
         }
         for (int idx = tid; idx < NCH * C * GCH; idx += NT) {
             const int i = part_of(idx, C * GCH), rem = idx - i * (C * GCH);
             const int t = rem / GCH, j = rem - t * GCH;
             const int64_t r = Row_(i)[t];
-            cp_async16(reinterpret_cast<float *>(Scr_(i)) + t * DK + j * 4, args.g + (r < 0 ? 0 : r) * DK + j * 4,
-                       r >= 0);
+            const bool ok = r >= 0 && GTR_INB(r * DK + j * 4 + 3, rows * DK, BS_TC_LOAD);
+            cp_async16(reinterpret_cast<float *>(Scr_(i)) + t * DK + j * 4, args.g + (ok ? r * DK + j * 4 : 0), ok);
         }
         cp_async_commit();
         cp_async_wait_all();
@@ -407,9 +412,10 @@ gla_tc_kernel(const TcArgs args) {
                     const int t = idx / DK, d = idx - t * DK;
                     const int64_t r = sRow[16 * u + t];
                     const int64_t o = (r < 0 ? 0 : r) * DK + d;
-                    xq[idx] = r >= 0 ? args.q[o] : __float2half(0.f);
-                    xk[idx] = r >= 0 ? args.k[o] : __float2half(0.f);
-                    xb[idx] = r >= 0 ? args.g[o] * kLog2e : 0.f;
+                    const bool ok = r >= 0 && GTR_INB(o, rows * DK, BS_TC_EXACT);
+                    xq[idx] = ok ? args.q[o] : __float2half(0.f);
+                    xk[idx] = ok ? args.k[o] : __float2half(0.f);
+                    xb[idx] = ok ? args.g[o] * kLog2e : 0.f;
                 }
                 __syncthreads();
                 for (int d = tid; d < DK; d += NT) {
@@ -503,6 +509,7 @@ gla_tc_kernel(const TcArgs args) {
     const int64_t sdx = ((int64_t)seq * geo.nc + c);
     if (MODE == TC_SUMMARY) {
         // dS_c[dk][dv] = L^T transposed; gamma_c
+        if (!GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SUMMARY)) return;
         float *dst = args.dS + sdx * DK * DV;
         const int vr = v0 + (lane >> 2);
 #pragma unroll
@@ -521,7 +528,7 @@ gla_tc_kernel(const TcArgs args) {
     float Se[KT][4];
     bool have_state = c > 0;
     if (MODE == TC_OUTPUT) {
-        const float *src = args.S_enter + sdx * DK * DV;
+        const float *src = args.S_enter + (GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SENTER) ? sdx : 0) * DK * DV;
         const int vr = v0 + (lane >> 2);
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
@@ -539,8 +546,10 @@ gla_tc_kernel(const TcArgs args) {
         // two, since the tile reads it before it writes it)
         const int slot_in = NCH == 1 ? ((c0 - 1) & 1) : 0;
         const int slot_out = NCH == 1 ? (c0 & 1) : 0;
+        // seq < nseq indexes the flags and both ring slots
+        const bool seq_ok = GTR_INB(seq, nseq, BS_TC_FLAG) && GTR_INB((int64_t)seq * 2 + 1, (int64_t)nseq * 2, BS_TC_RING);
         if (c0 > 0) {
-            if (tid == 0) {
+            if (tid == 0 && seq_ok) {
                 long long spins = 0;
                 while (ld_acquire(&flags[seq]) < c0) {
                     if (++spins > args.spin_limit) {
@@ -551,7 +560,7 @@ gla_tc_kernel(const TcArgs args) {
                 }
             }
             __syncthreads();
-            if (ch == 0) {
+            if (ch == 0 && seq_ok) {
                 const float4 *src = reinterpret_cast<const float4 *>(
                     args.ring + ((int64_t)seq * 2 + slot_in) * (DK * DV));
 #pragma unroll
@@ -589,7 +598,7 @@ gla_tc_kernel(const TcArgs args) {
         }
         // the tile's last chunk publishes diag(gamma_c) S_enter + L for the next tile
         const bool hold = (seq == args.hold_seq && args.hold_chunk >= c0 && args.hold_chunk < c0 + NCH);
-        if (c0 + NCH < geo.nc && !hold) {
+        if (c0 + NCH < geo.nc && !hold && seq_ok) {
             if (ch == NCH - 1) {
                 float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + slot_out) * (DK * DV));
 #pragma unroll
@@ -656,8 +665,9 @@ gla_tc_kernel(const TcArgs args) {
             const int64_t *sRow = Row_(i);
             for (int idx = tid; idx < len * VCH; idx += NT) {
                 const int t = idx / VCH, j = idx - t * VCH;
-                *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
-                    *reinterpret_cast<const int4 *>(so + t * LDV + j * 8);
+                if (sRow[t] >= 0 && GTR_INB(sRow[t] * DV + j * 8 + 7, rows * DV, BS_TC_OUT))
+                    *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
+                        *reinterpret_cast<const int4 *>(so + t * LDV + j * 8);
             }
         }
     }

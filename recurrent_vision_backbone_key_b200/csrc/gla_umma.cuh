@@ -171,6 +171,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [2] tmem base; mbar at +16
     const uint32_t mbar = base_addr + L::MISC + 16;
     const int nseq = geo.B * geo.heads;
+    const int64_t rows = (int64_t)geo.B * geo.N * geo.heads;  // token-head rows of every tensor
 
     // ---- tensor memory first (before the ticket: a CTA waiting for TMEM holds no ticket)
     if (warp == 0) {
@@ -205,8 +206,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         // path, which reads all rows, starts with a CTA barrier)
         if (lane < 16) {
             const int t = 16 * warp + lane;
-            sRow[t] = (t < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
-                                : (int64_t)-1;
+            int64_t r = (t < len) ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
+                                  : (int64_t)-1;
+            if (r >= 0 && !GTR_INB(r, rows, BS_UMMA_ROW)) r = -1;
+            sRow[t] = r;
         }
         __syncwarp();
 
@@ -214,11 +217,12 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         for (int idx = lane; idx < 16 * 8; idx += 32) {
             const int t = 16 * warp + (idx >> 3), j = idx & 7;
             const int64_t r = sRow[t];
-            const int64_t o = (r < 0 ? 0 : r) * 64 + j * 8;
+            const bool ok = r >= 0 && GTR_INB(r * 64 + j * 8 + 7, rows * 64, BS_UMMA_QKV);
+            const int64_t o = ok ? r * 64 + j * 8 : 0;
             const uint32_t so = t * 128 + (((j ^ (t & 7)) & 7) << 4);
-            cp_async16(base + L::QH + so, args.q + o, r >= 0);
-            cp_async16(base + L::KE + so, args.k + o, r >= 0);
-            cp_async16(base + L::V + so, args.v + o, r >= 0);
+            cp_async16(base + L::QH + so, args.q + o, ok);
+            cp_async16(base + L::KE + so, args.k + o, ok);
+            cp_async16(base + L::V + so, args.v + o, ok);
         }
         cp_async_commit();
 
@@ -230,7 +234,9 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
             const int64_t r = sRow[16 * u + t];
-            av[t] = r >= 0 ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * 64 + d0)) : make_float2(0.f, 0.f);
+            av[t] = (r >= 0 && GTR_INB(r * 64 + d0 + 1, rows * 64, BS_UMMA_G))
+                        ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * 64 + d0))
+                        : make_float2(0.f, 0.f);
         }
         float2 tot = make_float2(1.f, 1.f);
 #pragma unroll
@@ -323,10 +329,11 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     const int64_t r = sRow[16 * u + t];
-                    const float2 gv = r >= 0 ? *reinterpret_cast<const float2 *>(args.g + r * 64 + d0)
-                                             : make_float2(0.f, 0.f);
-                    const __half2 qv = r >= 0 ? *reinterpret_cast<const __half2 *>(args.q + r * 64 + d0)
-                                              : __float2half2_rn(0.f);
+                    const bool ok = r >= 0 && GTR_INB(r * 64 + d0 + 1, rows * 64, BS_UMMA_EXACT);
+                    const float2 gv = ok ? *reinterpret_cast<const float2 *>(args.g + r * 64 + d0)
+                                         : make_float2(0.f, 0.f);
+                    const __half2 qv = ok ? *reinterpret_cast<const __half2 *>(args.q + r * 64 + d0)
+                                          : __float2half2_rn(0.f);
                     E.x *= ex2(gv.x * kLog2e);
                     E.y *= ex2(gv.y * kLog2e);
                     *reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0)) =
@@ -349,9 +356,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                     const int tt = idx >> 4, d = idx & 15;
                     const int64_t r = sRow[tt];
                     const int64_t o = (r < 0 ? 0 : r) * 64 + 16 * hd + d;
-                    xq[idx] = r >= 0 ? args.q[o] : __float2half(0.f);
-                    xk[idx] = r >= 0 ? args.k[o] : __float2half(0.f);
-                    xb[idx] = r >= 0 ? args.g[o] * kLog2e : 0.f;
+                    const bool ok = r >= 0 && GTR_INB(o, rows * 64, BS_UMMA_EXACT);
+                    xq[idx] = ok ? args.q[o] : __float2half(0.f);
+                    xk[idx] = ok ? args.k[o] : __float2half(0.f);
+                    xb[idx] = ok ? args.g[o] * kLog2e : 0.f;
                 }
                 __syncthreads();
                 if (tid < 16) {
@@ -387,7 +395,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         if (c > 0) {
             const float4 *ring_in =
                 reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
-            if (lane == 0) {
+            if (lane == 0 && GTR_INB(2 + (int64_t)seq * 4 + warp, 2 + (int64_t)nseq * 4, BS_UMMA_FLAG)) {
                 long long spins = 0;
                 while (ld_acquire(flag) < c) {
                     if (++spins > args.spin_limit) {
@@ -400,7 +408,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             __syncwarp();
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
-                const float4 x = __ldcg(ring_in + ((warp * KT + n) * 32 + lane));
+                const int64_t e = ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV) + ((warp * KT + n) * 32 + lane) * 4;
+                const float4 x = GTR_INB(e + 3, (int64_t)nseq * 2 * DK * DV, BS_UMMA_RING)
+                                     ? __ldcg(ring_in + ((warp * KT + n) * 32 + lane))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
                 Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
             }
         } else {
@@ -433,13 +444,16 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                         x.y = fmaf(gg.y, Se[n][1], dS[4 * m + 1]);
                         x.z = fmaf(gg.x, Se[n][2], dS[4 * m + 2]);
                         x.w = fmaf(gg.y, Se[n][3], dS[4 * m + 3]);
-                        __stcg(dst + ((warp * KT + n) * 32 + lane), x);
+                        const int64_t e = ((int64_t)seq * 2 + (c & 1)) * (DK * DV) + ((warp * KT + n) * 32 + lane) * 4;
+                        if (GTR_INB(e + 3, (int64_t)nseq * 2 * DK * DV, BS_UMMA_RING))
+                            __stcg(dst + ((warp * KT + n) * 32 + lane), x);
                     }
                 }
             }
             if (publish) {
                 __syncwarp();
-                if (lane == 0) st_release(flag, c + 1);
+                if (lane == 0 && GTR_INB(2 + (int64_t)seq * 4 + warp, 2 + (int64_t)nseq * 4, BS_UMMA_FLAG))
+                    st_release(flag, c + 1);
             }
         }
         // ---- the masked scores P (fp16, swizzled), this warp's 16 query rows
@@ -509,7 +523,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
-                if (t < len)
+                if (t < len && sRow[t] >= 0 && GTR_INB(sRow[t] * DV + j * 8 + 7, rows * DV, BS_UMMA_OUT))
                     *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
                         *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
             }

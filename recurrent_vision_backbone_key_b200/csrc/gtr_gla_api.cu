@@ -9,6 +9,7 @@
 #include <map>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "gla_common.cuh"
 #include "gla_tc.cuh"
@@ -17,6 +18,22 @@ namespace gtr {
 
 static std::atomic<uint64_t> g_launches{0};
 void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// Readers of the per-translation-unit bounds reports (checked builds only
+// register any); function-local statics, so registration at load time does
+// not depend on the order in which translation units initialise.
+std::mutex &bounds_readers_mu() {
+    static std::mutex mu;
+    return mu;
+}
+std::vector<BoundsReader> &bounds_readers() {
+    static std::vector<BoundsReader> readers;
+    return readers;
+}
+void register_bounds_reader(BoundsReader reader) {
+    std::lock_guard<std::mutex> lk(bounds_readers_mu());
+    bounds_readers().push_back(reader);
+}
 
 namespace {
 
@@ -585,5 +602,35 @@ const char *gtr_gla_last_error(void) { return t_err; }
 uint64_t gtr_gla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int gtr_gla_version(void) { return 200; }
+
+int gtr_gla_bounds_checked(void) {
+#ifdef GTR_BOUNDS_CHECK
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+gtr_status_t gtr_gla_debug_bounds_report(unsigned long long *count, int *site, long long *index,
+                                         long long *limit, int clear) {
+    t_err[0] = '\0';
+    if (!count || !site || !index || !limit) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    *count = 0;
+    *site = 0;
+    *index = 0;
+    *limit = 0;
+    if (!gtr_gla_bounds_checked()) return fail(GTR_ERR_INVALID_ARG, "library built without bounds checks%s");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    gtr::BoundsReport sum = {};
+    std::lock_guard<std::mutex> lk(gtr::bounds_readers_mu());
+    for (gtr::BoundsReader r : gtr::bounds_readers())
+        if (r(&sum, clear) != 0) return fail(GTR_ERR_CUDA, "reading a bounds report failed%s");
+    *count = sum.count;
+    *site = sum.site;
+    *index = sum.index;
+    *limit = sum.limit;
+    return GTR_OK;
+}
 
 }  // extern "C"

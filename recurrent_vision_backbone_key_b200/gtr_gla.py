@@ -20,6 +20,7 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libgtr_gla.so")
+CHECKED_LIB_PATH = os.path.join(_PKG, "libgtr_gla_checked.so")  # bounds-checked debug build
 
 GTR_OK = 0
 STATUS_NAMES = {
@@ -50,6 +51,10 @@ SIGNATURES = {
     "gtr_gla_last_error": (ctypes.c_char_p, []),
     "gtr_gla_launch_count": (ctypes.c_uint64, []),
     "gtr_gla_version": (_I, []),
+    "gtr_gla_bounds_checked": (_I, []),
+    "gtr_gla_debug_bounds_report": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_int),
+                                         ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong),
+                                         _I]),
 }
 
 _lib = None
@@ -61,21 +66,46 @@ class GtrError(RuntimeError):
         super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
 
 
+def _open(path: str) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m recurrent_vision_backbone_key_b200.build`"
+            " (no CPU fallback exists)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     """Load the CUDA library (once).  Raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(path):
-            raise RuntimeError(
-                f"{path} is missing: build it with `python -m recurrent_vision_backbone_key_b200.build`"
-                " (no CPU fallback exists)")
-        lib = ctypes.CDLL(path)
-        for name, (res, args) in SIGNATURES.items():
-            fn = getattr(lib, name)
-            fn.restype = res
-            fn.argtypes = args
-        _lib = lib
+        _lib = _open(path)
     return _lib
+
+
+_lib_checked = None
+
+
+def load_checked(path: str = CHECKED_LIB_PATH) -> ctypes.CDLL:
+    """Load the bounds-checked debug build (once), a separate library with the
+    same C ABI.  Raises if it has not been built."""
+    global _lib_checked
+    if _lib_checked is None:
+        _lib_checked = _open(path)
+    return _lib_checked
+
+
+def bounds_report(lib: ctypes.CDLL, clear: bool = True):
+    """(count, site, index, limit) of the accesses a checked build skipped."""
+    cnt, site = ctypes.c_ulonglong(0), ctypes.c_int(0)
+    idx, lim = ctypes.c_longlong(0), ctypes.c_longlong(0)
+    check(lib.gtr_gla_debug_bounds_report(ctypes.byref(cnt), ctypes.byref(site), ctypes.byref(idx),
+                                          ctypes.byref(lim), int(clear)))
+    return cnt.value, site.value, idx.value, lim.value
 
 
 def _addr(x):

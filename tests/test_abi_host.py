@@ -38,6 +38,22 @@ def test_exports_every_declared_symbol(lib):
     assert names <= set(lib.SIGNATURES), names - set(lib.SIGNATURES)
 
 
+def test_bounds_checked_build_loads_and_exports(lib):
+    """The bounds-checked debug build has the same C ABI; it says it is the
+    checked one, and the normal build refuses the report call."""
+    libbuild.build(checked=True)
+    checked = lib.load_checked()
+    for n in sorted(declared_functions()):
+        assert hasattr(checked, n), n
+    assert checked.gtr_gla_bounds_checked() == 1
+    assert lib.load().gtr_gla_bounds_checked() == 0
+    cnt, site = ctypes.c_ulonglong(7), ctypes.c_int(7)
+    idx, lim = ctypes.c_longlong(7), ctypes.c_longlong(7)
+    st = lib.load().gtr_gla_debug_bounds_report(ctypes.byref(cnt), ctypes.byref(site), ctypes.byref(idx),
+                                                ctypes.byref(lim), 0)
+    assert st == 1 and cnt.value == 0 and site.value == 0
+
+
 def test_version_and_status_strings(lib):
     assert lib.gtr_gla_version() >= 100
     assert lib.gtr_gla_status_string(0) == "ok"
