@@ -97,6 +97,37 @@ def profiled_traffic(w, kernel):
     return int(fields["traffic_bytes_per_launch"])
 
 
+def graph_replay_ms(call, dirs, replays=50):
+    """Median CUDA-event milliseconds of one forward replayed from a CUDA graph
+    (one graph per direction, replayed in turn)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for d in dirs:  # the workspaces of this stream exist before the capture
+            call(d, side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graphs = []
+    for d in dirs:
+        gph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gph, stream=side):
+            call(d, side)
+        graphs.append(gph)
+    for i in range(3 * len(graphs)):
+        graphs[i % len(graphs)].replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    torch.cuda.synchronize()
+    for i, (a, b) in enumerate(ev):
+        a.record()
+        graphs[i % len(graphs)].replay()
+        b.record()
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) for a, b in ev)
+    del graphs
+    return {"median_ms_per_forward": t[len(t) // 2], "min_ms": t[0], "replays": replays,
+            "note": "CUDA-graph replay, one forward per graph, CUDA events around each replay"}
+
+
 def describe(w):
     dirs = "+".join(DIR_NAMES[d] for d in w.directions)
     return (f"{w.name}: B{w.B} {w.grid_h}x{w.grid_w} grid ({w.N} tokens), {w.heads} heads, "
@@ -235,16 +266,27 @@ def run_reference(args, w):
     return 0
 
 
-def time_steps(fn, steps, stream):
-    """Runs fn(i) for i in range(steps) between two events on `stream`; ms."""
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(steps):
+def time_steps(fn, steps, stream, flush=None):
+    """Runs fn(i) for i in range(steps) on `stream`; ms.  Without `flush`, one
+    pair of events brackets all steps.  With it, flush() runs before every
+    step (outside the timing) and the per-step event times are summed."""
+    if flush is None:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(steps):
+            fn(i)
+        end.record(stream)
+        end.synchronize()
+        return start.elapsed_time(end)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i, (a, b) in enumerate(ev):
+        flush()
+        a.record(stream)
         fn(i)
-    end.record(stream)
-    end.synchronize()
-    return start.elapsed_time(end)
+        b.record(stream)
+    ev[-1][1].synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev)
 
 
 def main():
@@ -258,6 +300,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = WORKLOADS[args.workload]
@@ -281,6 +324,13 @@ def main():
                                                  w.d_k, w.d_v, dirs[i % len(dirs)], w.chunk, sched,
                                                  out, stream))
 
+    # Inputs smaller than twice L2 would be read from L2 by the next step:
+    # then L2 is flushed (a write larger than L2) before every timed step.
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None
+    if alg_bytes_total(w) < 2 * l2:
+        scrub = torch.empty(2 * l2, dtype=torch.uint8, device=f"cuda:{dev}")
+        flush = lambda: scrub.fill_(1)
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
@@ -288,7 +338,7 @@ def main():
     l0 = gtr_gla.gtr_gla_launch_count()
     with ClockSampler(dev) as clocks:
         torch.cuda.synchronize()
-        ms = time_steps(step, args.steps, stream)
+        ms = time_steps(step, args.steps, stream, flush)
         torch.cuda.synchronize()
     launches = gtr_gla.gtr_gla_launch_count() - l0
     rdist.barrier()
@@ -319,6 +369,13 @@ def main():
                 "tensor_frac_of_bf16_peak": w.algorithmic_flops() / (ms / args.steps * 1e-3) / 1e12 / tc_peak}
     if phase_ms:
         roofline["phase_ms"] = phase_ms
+
+    # The pages' latency protocol: median CUDA-event time of one forward
+    # replayed from a CUDA graph (outside the timed region above).
+    graph = None
+    if not args.no_graph:
+        graph = graph_replay_ms(lambda d, st: gtr_gla.check(gtr_gla.gtr_gla_forward_ex(
+            q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d, w.chunk, sched, out, st)), dirs)
 
     # End to end through the host-buffer entry point: pinned host inputs in,
     # host output back, every step.
@@ -360,8 +417,11 @@ def main():
             "config": {"workload": describe(w), "B": w.B, "grid": [w.grid_h, w.grid_w],
                        "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk,
                        "schedule": args.schedule, "parallelism": f"dp{world} (independent batches)",
-                       "l2": f"inputs larger than L2 ({alg_bytes_total(w) / 1e6:.0f} MB per step), no flush"},
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                       "l2": (f"inputs larger than L2 ({alg_bytes_total(w) / 1e6:.0f} MB per step), no flush"
+                              if flush is None else
+                              f"L2 flushed before every timed step ({2 * l2 / 1e6:.0f} MB write, outside the "
+                              f"per-step CUDA events); {alg_bytes_total(w) / 1e6:.1f} MB per step")},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": int(launches), "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -98,7 +98,9 @@ typedef enum {
  * out must not overlap q, k, v or g (GTR_ERR_ALIAS).  Uses an internal
  * per-device, per-stream workspace that grows on demand (GTR_ERR_OOM if it
  * cannot); a call that has to grow it synchronises the device, so make the
- * first call of the largest size outside any stream capture. */
+ * first call of the largest size on that stream outside any stream capture.
+ * After that, calls on the stream can be captured into a CUDA graph and
+ * replayed (the fused schedules reset their control words inside the graph). */
 gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const float *g,
                              int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                              int direction, int chunk, void *out, void *stream);

@@ -313,3 +313,39 @@ def test_batched_full_size_tcgen05_sampled(oracle_mod, direction):
     _sampled_check(oracle_mod, w, q, k, v, g, out, direction, 6, seed=direction)
     ref = run_forward(q, k, v, g, w.grid_h, w.grid_w, direction, w.chunk, "fused")
     assert ((out.float() - ref.float()).abs().max() / ref.float().abs().max()).item() < 2e-3
+
+
+@pytest.mark.parametrize("B,heads", [(1, 6), (4, 40)])
+def test_cuda_graph_twelve_call_stack(B, heads):
+    """A stack of 12 forward calls cycling the four directions (the high-res
+    block stack), captured once into a CUDA graph and replayed: every replay
+    gives the outputs of the eager calls bit for bit.  (1, 6) runs the
+    mma.sync kernel with two chunks per tile, (4, 40) the tcgen05 kernel."""
+    H = W = 24
+    xs = [gpu_inputs(B, H, W, heads, 64, 64, seed=400 + i) for i in range(12)]
+    outs = [torch.empty_like(x[2]) for x in xs]
+
+    def stack():
+        st = torch.cuda.current_stream()
+        for i, (q, k, v, g) in enumerate(xs):
+            gtr_gla.forward(q, k, v, g, H, W, direction=i % 4, chunk=64, out=outs[i], stream=st)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        stack()  # eager: allocates the workspaces before the capture
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    eager = [o.clone() for o in outs]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):  # the stream whose workspace exists
+        stack()
+    for rep in range(3):
+        for o in outs:
+            o.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        for o, e in zip(outs, eager):
+            assert torch.equal(o, e), rep
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0
+    del graph
