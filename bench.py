@@ -60,11 +60,11 @@ PROFILE_SUMMARIES = {
 def fused_kernel_name(w, schedule):
     """The kernel the fused schedules launch for this workload (the library's
     dispatch: tcgen05 for d_k = d_v = 64 and chunk 64 when sequences are at
-    least twice the SM count, or when asked for; else the mma.sync kernel, one
-    or two chunks per tile)."""
+    least twice the SM count, or when asked for; else the mma.sync kernel, two
+    chunks per tile for few sequences when d_v <= 64, else one)."""
     nseq = w.B * w.heads
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    pair = nseq < 2 * sms
+    pair = nseq < 2 * sms and w.d_v <= 64  # two-chunk tiles exist for d_v <= 64
     tc5_shape = w.d_k == 64 and w.d_v == 64 and w.chunk == 64
     if schedule == "fused_tcgen05" or (schedule == "auto" and tc5_shape and not pair):
         return "gla_umma_kernel"
