@@ -98,7 +98,11 @@ __global__ void __launch_bounds__(kThreads) summary_simt_kernel(
 
 // Phase 2: one thread per state element, serial over chunks; consecutive
 // threads own consecutive elements, so every step is one coalesced sweep.
-// In place is allowed: element e of chunk c is read before it is written.
+// The loads do not depend on the running state, so they are issued kAhead
+// chunks ahead of their use and only the fma chain is serial.  In place is
+// allowed: element e of chunk c is read (kAhead steps early) before step c
+// writes it, and no step writes an element a later prefetch reads.
+constexpr int kAhead = 8;
 __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
     const float *dS, const float *__restrict__ gamma, int nseq, int nc, int dk, int dv, float *S_enter) {
     const int per_seq = (dk * dv + blockDim.x - 1) / blockDim.x;
@@ -111,12 +115,27 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
     const float *src = dS + seq * nc * stride + e;
     const float *gm = gamma + seq * nc * dk + i;
     float *dst = S_enter + seq * nc * stride + e;
+    float xs[kAhead], as[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+        xs[u] = u < nc ? src[u * stride] : 0.f;
+        as[u] = u < nc ? gm[(int64_t)u * dk] : 0.f;
+    }
     float S = 0.f;
-    for (int c = 0; c < nc; ++c) {
-        float x = src[c * stride];
-        float a = gm[(int64_t)c * dk];
-        dst[c * stride] = S;
-        S = fmaf(a, S, x);
+    for (int c0 = 0; c0 < nc; c0 += kAhead) {
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int c = c0 + u;
+            if (c < nc) {
+                const float x = xs[u], a = as[u];
+                if (c + kAhead < nc) {  // chunk c + kAhead, read before anything writes it
+                    xs[u] = src[(c + kAhead) * stride];
+                    as[u] = gm[(int64_t)(c + kAhead) * dk];
+                }
+                dst[c * stride] = S;
+                S = fmaf(a, S, x);
+            }
+        }
     }
 }
 

@@ -164,6 +164,9 @@ gtr_status_t status_word(unsigned **out) {
 }
 
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
+// At most this many (batch, head) sequences: GTR_SCHED_AUTO runs the
+// three-phase schedule (the fused chain is the bottleneck then).
+constexpr int64_t kFewSequences = 16;
 
 // Streaming multiprocessors of the current device (cached per device).
 cudaError_t sm_count(int *out) {
@@ -296,6 +299,12 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     __half *ho = static_cast<__half *>(out);
     if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
+    // With few sequences the fused kernels wait on the chain of boundary
+    // states (one L2 hand-over per chunk step); the three-phase schedule has
+    // no such chain (its scan is a pipelined sweep) and its state traffic is
+    // small then, so AUTO takes it.
+    if (schedule == GTR_SCHED_AUTO && (int64_t)geo.B * geo.heads <= kFewSequences)
+        return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
     // GTR_SCHED_FUSED keeps the mma.sync kernels; AUTO lets run_fused choose.
     return run_fused(hq, hk, hv, g, geo, ho, st, fused_kernel_for(schedule));
 }
