@@ -352,9 +352,11 @@ def main():
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     alg_bytes = w.algorithmic_bytes()
     per_launch_ms = ms / args.steps
-    dominant = fused_kernel_name(w, args.schedule) if sched in (0, 1, 4) else "forward step"
+    # AUTO runs the three-phase schedule for at most 16 sequences (the library's rule)
+    three_phase = sched == 2 or (sched == 0 and w.B * w.heads <= 16)
+    dominant = fused_kernel_name(w, args.schedule) if sched in (0, 1, 4) and not three_phase else "forward step"
     phase_ms = None
-    if sched == 2:
+    if three_phase:
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
         dominant = max(phase_ms, key=phase_ms.get)
         per_launch_ms = phase_ms[dominant]

@@ -79,8 +79,10 @@ typedef enum {
 } gtr_status_t;
 
 typedef enum {
-    GTR_SCHED_AUTO = 0,             /* library choice: GTR_SCHED_FUSED_TCGEN05 for its shape when
-                                       there are at least 2 sequences per SM, else GTR_SCHED_FUSED */
+    GTR_SCHED_AUTO = 0,             /* library choice: GTR_SCHED_THREE_PHASE for at most 16
+                                       sequences (B*heads); else GTR_SCHED_FUSED_TCGEN05 for its
+                                       shape when there are at least 2 sequences per SM, else
+                                       GTR_SCHED_FUSED */
     GTR_SCHED_FUSED = 1,            /* one kernel (mma.sync tensor cores): summaries, chained
                                        boundary states, outputs */
     GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output (tensor cores) */
