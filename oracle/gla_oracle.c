@@ -28,7 +28,7 @@
  *     with S_t a d_k x d_v matrix, g_t the per-key-dimension log-gate.
  *     The readout uses S_t *including* token t.
  *
- * Readings taken where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   - tensor layout [B][N][heads][d], tokens in row-major spatial order;
  *   - R->L is the reversed row-major order, T->B is column-major order
  *     (t = col*H + row), B->T is the reversed column-major order;

@@ -27,7 +27,7 @@
 // stored at chunk j ^ (r mod 8)), read as K-major or MN-major by the MMA
 // descriptors.  Accumulators: with M = 64, row m of an accumulator sits in TMEM
 // lane (m mod 16) + 32 (m / 16) + base, base 0 or 16, so two of them share 64
-// columns: A (base 0) and dS^T (base 16) in one MMA round, then O over A.
+// columns: A (base 0) and dS^T (base 16) in one MMA pass, then O over A.
 // Warp w reads rows 16w..16w+15 of either with the 16x256b load, in the m16n8
 // accumulator-fragment layout.
 #pragma once
@@ -295,10 +295,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         const bool exact = __syncthreads_or(!gam_ok || fmaxf(qm.x, qm.y) * qscale > 16.f) != 0;
         if (warp == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
 
-        // Two MMA rounds through the same 64 TMEM columns.  Round 1: A = qh ke^T
+        // Two MMA passes through the same 64 TMEM columns.  Pass 1: A = qh ke^T
         // (whole-chunk form only) in TMEM lanes 0-15 of each 32-lane group and
         // dS^T = V^T ke in lanes 16-31 (an M = 64 accumulator uses half of each
-        // group).  Round 2: O = P V + qh S' over A.  `phase` is the parity of the
+        // group).  Pass 2: O = P V + qh S' over A.  `phase` is the parity of the
         // next mbarrier completion.
         uint32_t phase = 0;
         const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         }
 
         // ---- this warp's slice of the state entering the chunk (bounded
-        // wait on the predecessor's flag for the same slice), while round 1 runs
+        // wait on the predecessor's flag for the same slice), while pass 1 runs
         float Se[KT][4];
         int *flag = args.ctrl + 2 + (int64_t)seq * 4 + warp;
         if (c > 0) {
@@ -423,7 +423,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         phase ^= 1u;
         tc_fence_after();
         // ---- publish this warp's slice of S_leave = diag(gamma_c) S_enter + dS,
-        // half the columns at a time, as soon as round 1 is done: the chain of
+        // half the columns at a time, as soon as pass 1 is done: the chain of
         // boundary states waits on this release
         {
             const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
@@ -473,7 +473,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             }
         }
         // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value
-        // columns), over ke (round 1 is complete)
+        // columns), over ke (pass 1 is complete)
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
             const float2 sc = *reinterpret_cast<const float2 *>(vSc + 8 * n + kc);
@@ -485,7 +485,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         tc_fence_before();
         __syncthreads();  // P and S' written; A and dS^T read by every warp
 
-        // ---- round 2: O = P V + qh S' over A
+        // ---- pass 2: O = P V + qh S' over A
         if (tid == 0) {
             tc_fence_after();
             const uint32_t aP = base_addr + L::P, aSP = base_addr + L::SP;
