@@ -2,8 +2,8 @@
 direction on tiny and odd shapes (7 x 9 grid, one or three heads) through
 libgtr_gla_checked.so, where every global index computed at run time is
 tested against its buffer before the access.  The outputs must match the
-oracle and the build must report no skipped access.  This stands in for
-compute-sanitizer, which is closed on the pool."""
+oracle and the build must report no skipped access.  This stands in for a
+run under a memory-checking tool."""
 import ctypes
 
 import pytest
