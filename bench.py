@@ -57,19 +57,15 @@ PROFILE_SUMMARIES = {
 }
 
 
-def fused_kernel_name(w, schedule):
-    """The kernel the fused schedules launch for this workload (the library's
-    dispatch: tcgen05 for d_k = d_v = 64 and chunk 64 when sequences are at
-    least twice the SM count, or when asked for; else the mma.sync kernel, two
-    chunks per tile for few sequences when d_v <= 64, else one)."""
-    nseq = w.B * w.heads
+def planned_kernel(w, schedule):
+    """(plan code, kernel name) of what the library launches for this workload
+    and schedule on this device (the library's own dispatch, gtr_gla_plan)."""
     sms = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
-    pair = nseq < 2 * sms and w.d_v <= 64  # two-chunk tiles exist for d_v <= 64
-    tc5_shape = w.d_k == 64 and w.d_v == 64 and w.chunk == 64
-    if schedule == "fused_tcgen05" or (schedule == "auto" and tc5_shape and not pair):
-        return "gla_umma_kernel"
-    mode = "FUSED_PAIR" if pair else "FUSED"
-    return f"gla_tc_kernel<{w.d_k},{w.d_v},{mode},{2 if pair else 1}>"
+    plan = gtr_gla.gtr_gla_plan(w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, w.chunk, schedule, sms)
+    names = {0: "three-phase (summary, scan, output)", 1: "three-phase on CUDA cores",
+             2: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,1>", 3: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,2>",
+             4: "gla_umma_kernel"}
+    return plan, names.get(plan, "unknown")
 
 
 def profiled_traffic(w, kernel):
@@ -352,11 +348,9 @@ def main():
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     alg_bytes = w.algorithmic_bytes()
     per_launch_ms = ms / args.steps
-    # AUTO runs the three-phase schedule for at most 16 sequences (the library's rule)
-    three_phase = sched == 2 or (sched == 0 and w.B * w.heads <= 16)
-    dominant = fused_kernel_name(w, args.schedule) if sched in (0, 1, 4) and not three_phase else "forward step"
+    plan, dominant = planned_kernel(w, args.schedule)
     phase_ms = None
-    if three_phase:
+    if plan == 0:  # the three-phase schedule: time its phases one by one
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
         dominant = max(phase_ms, key=phase_ms.get)
         per_launch_ms = phase_ms[dominant]

@@ -92,6 +92,15 @@ typedef enum {
                                        other shapes run GTR_SCHED_FUSED) */
 } gtr_schedule_t;
 
+/* The kernels a schedule launches (gtr_gla_plan). */
+typedef enum {
+    GTR_PLAN_THREE_PHASE = 0,       /* chunk summaries, boundary scan, chunk outputs (tensor cores) */
+    GTR_PLAN_THREE_PHASE_SIMT = 1,  /* the same three phases on CUDA cores */
+    GTR_PLAN_FUSED_MMA = 2,         /* fused mma.sync kernel, one chunk per tile */
+    GTR_PLAN_FUSED_MMA_PAIR = 3,    /* fused mma.sync kernel, two chunks per tile (d_v <= 64) */
+    GTR_PLAN_FUSED_TCGEN05 = 4      /* fused tcgen05 kernel (d_k = d_v = 64, chunk 64) */
+} gtr_plan_t;
+
 /* The GLA forward over all B*heads sequences (see the operation above).
  *   q, k (device, fp16) [B][N][heads][d_k]; v (device, fp16) [B][N][heads][d_v];
  *   g (device, fp32) [B][N][heads][d_k] log-gates; out (device, fp16)
@@ -224,6 +233,16 @@ uint64_t gtr_gla_launch_count(void);
 
 /* ABI version: major*10000 + minor*100 + patch. */
 int gtr_gla_version(void);
+
+/* Which kernels gtr_gla_forward_ex(..., schedule, ...) launches for this
+ * problem on a device with sm_count streaming multiprocessors: a gtr_plan_t,
+ * or -1 for invalid arguments.  Host-only; needs no device.  AUTO takes the
+ * three-phase schedule for at most 16 sequences (B*heads), the tcgen05
+ * kernel for its shape when sequences are at least 2*sm_count, else the
+ * mma.sync kernel with two chunks per tile below 2*sm_count sequences when
+ * d_v <= 64, one chunk per tile otherwise. */
+int gtr_gla_plan(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int chunk, int schedule,
+                 int sm_count);
 
 /* 1 if this library is the bounds-checked debug build, else 0.  The checked
  * build (libgtr_gla_checked.so, compiled with GTR_BOUNDS_CHECK) tests every

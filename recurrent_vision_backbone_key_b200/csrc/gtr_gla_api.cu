@@ -197,11 +197,31 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
 
 bool tcgen05_shape(const Geom &g) { return g.dk == 64 && g.dv == 64 && g.chunk == 64; }
 
-// Which kernel a fused schedule launches.
-enum FusedKernel { FK_AUTO = 0, FK_MMA = 1, FK_TCGEN05 = 2 };
+// The kernels a schedule launches for a problem: a host-only decision, so
+// it can be asked without a device (gtr_gla_plan).  With three_phase_ok
+// false (the bounded-wait test hook) AUTO keeps to the fused kernels.
+gtr_plan_t plan_for(const Geom &geo, int schedule, int sms, bool three_phase_ok = true) {
+    const int64_t nseq = (int64_t)geo.B * geo.heads;
+    if (schedule == GTR_SCHED_THREE_PHASE) return GTR_PLAN_THREE_PHASE;
+    if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return GTR_PLAN_THREE_PHASE_SIMT;
+    // With few sequences the fused kernels wait on the chain of boundary
+    // states (one L2 hand-over per chunk step); the three-phase schedule has
+    // no such chain (its scan is a pipelined sweep) and its state traffic is
+    // small then, so AUTO takes it.
+    if (schedule == GTR_SCHED_AUTO && three_phase_ok && nseq <= kFewSequences) return GTR_PLAN_THREE_PHASE;
+    // Few sequences leave the chain of boundary states as the critical path:
+    // then two chunks per tile halve its length (d_v <= 64).  Many sequences
+    // keep every SM busy anyway: then one chunk per tile gives more resident
+    // CTAs.  The tcgen05 kernel does one chunk per tile: AUTO uses it when
+    // sequences are many; GTR_SCHED_FUSED_TCGEN05 forces it for its shape.
+    const bool pair = nseq < 2 * (int64_t)sms;
+    if (tcgen05_shape(geo) && (schedule == GTR_SCHED_FUSED_TCGEN05 || (schedule == GTR_SCHED_AUTO && !pair)))
+        return GTR_PLAN_FUSED_TCGEN05;
+    return (pair && geo.dv <= 64) ? GTR_PLAN_FUSED_MMA_PAIR : GTR_PLAN_FUSED_MMA;
+}
 
 gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const float *g,
-                       const Geom &geo, __half *out, cudaStream_t st, FusedKernel which,
+                       const Geom &geo, __half *out, cudaStream_t st, gtr_plan_t plan,
                        int hold_seq = -1, int hold_chunk = -1, long long spin_limit = kSpinLimit) {
     void *ws = nullptr;
     gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
@@ -219,24 +239,11 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     // Ticket and flags start from zero for every launch.
     cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
     if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
-    // Few sequences leave the chain of boundary states as the critical path:
-    // then two chunks per tile halve its length.  Many sequences keep every
-    // SM busy anyway: then one chunk per tile gives more resident CTAs.
-    int sms = 0;
-    if ((e = sm_count(&sms)) != cudaSuccess) return cuda_fail(e, "device query");
-    const bool pair = (int64_t)geo.B * geo.heads < 2 * (int64_t)sms;
-    // The tcgen05 kernel does one chunk per tile: the library uses it when
-    // sequences are many; FK_TCGEN05 forces it for its shape.
-    const bool tc5 = tcgen05_shape(geo) && (which == FK_TCGEN05 || (which == FK_AUTO && !pair));
-    if (tc5)
+    if (plan == GTR_PLAN_FUSED_TCGEN05)
         e = launch_fused_umma(a, st);
     else
-        e = launch_tc(a, pair ? TC_FUSED_PAIR : TC_FUSED, st);
+        e = launch_tc(a, plan == GTR_PLAN_FUSED_MMA_PAIR ? TC_FUSED_PAIR : TC_FUSED, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
-}
-
-FusedKernel fused_kernel_for(int schedule) {
-    return schedule == GTR_SCHED_FUSED ? FK_MMA : (schedule == GTR_SCHED_FUSED_TCGEN05 ? FK_TCGEN05 : FK_AUTO);
 }
 
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
@@ -297,16 +304,13 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     const __half *hq = static_cast<const __half *>(q), *hk = static_cast<const __half *>(k);
     const __half *hv = static_cast<const __half *>(v);
     __half *ho = static_cast<__half *>(out);
-    if (schedule == GTR_SCHED_THREE_PHASE) return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
-    if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return run_three_phase(hq, hk, hv, g, geo, ho, st, true);
-    // With few sequences the fused kernels wait on the chain of boundary
-    // states (one L2 hand-over per chunk step); the three-phase schedule has
-    // no such chain (its scan is a pipelined sweep) and its state traffic is
-    // small then, so AUTO takes it.
-    if (schedule == GTR_SCHED_AUTO && (int64_t)geo.B * geo.heads <= kFewSequences)
-        return run_three_phase(hq, hk, hv, g, geo, ho, st, false);
-    // GTR_SCHED_FUSED keeps the mma.sync kernels; AUTO lets run_fused choose.
-    return run_fused(hq, hk, hv, g, geo, ho, st, fused_kernel_for(schedule));
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
+    const gtr_plan_t plan = plan_for(geo, schedule, sms);
+    if (plan == GTR_PLAN_THREE_PHASE || plan == GTR_PLAN_THREE_PHASE_SIMT)
+        return run_three_phase(hq, hk, hv, g, geo, ho, st, plan == GTR_PLAN_THREE_PHASE_SIMT);
+    return run_fused(hq, hk, hv, g, geo, ho, st, plan);
 }
 
 }  // namespace
@@ -555,10 +559,13 @@ gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const voi
     if (schedule != GTR_SCHED_AUTO && schedule != GTR_SCHED_FUSED && schedule != GTR_SCHED_FUSED_TCGEN05)
         return fail(GTR_ERR_INVALID_ARG, "schedule must be AUTO, FUSED or FUSED_TCGEN05%s");
     if (empty) return GTR_OK;
+    int sms = 0;
+    cudaError_t e = sm_count(&sms);
+    if (e != cudaSuccess) return cuda_fail(e, "device query");
     return run_fused(static_cast<const __half *>(q), static_cast<const __half *>(k),
                      static_cast<const __half *>(v), g, geo, static_cast<__half *>(out),
-                     static_cast<cudaStream_t>(stream), fused_kernel_for(schedule), hold_seq, hold_chunk,
-                     spin_limit);
+                     static_cast<cudaStream_t>(stream), plan_for(geo, schedule, sms, false), hold_seq,
+                     hold_chunk, spin_limit);
 }
 
 gtr_status_t gtr_gla_release_workspace(void) {
@@ -611,6 +618,15 @@ const char *gtr_gla_last_error(void) { return t_err; }
 uint64_t gtr_gla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int gtr_gla_version(void) { return 200; }
+
+int gtr_gla_plan(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int chunk, int schedule,
+                 int sm_count) {
+    Geom geo;
+    bool empty = false;
+    if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return -1;
+    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05 || sm_count < 1) return -1;
+    return (int)plan_for(geo, schedule, sm_count);
+}
 
 int gtr_gla_bounds_checked(void) {
 #ifdef GTR_BOUNDS_CHECK

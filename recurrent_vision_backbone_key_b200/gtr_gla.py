@@ -51,6 +51,7 @@ SIGNATURES = {
     "gtr_gla_last_error": (ctypes.c_char_p, []),
     "gtr_gla_launch_count": (ctypes.c_uint64, []),
     "gtr_gla_version": (_I, []),
+    "gtr_gla_plan": (_I, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
     "gtr_gla_bounds_checked": (_I, []),
     "gtr_gla_debug_bounds_report": (_I, [ctypes.POINTER(ctypes.c_ulonglong), ctypes.POINTER(ctypes.c_int),
                                          ctypes.POINTER(ctypes.c_longlong), ctypes.POINTER(ctypes.c_longlong),
@@ -212,6 +213,14 @@ def gtr_gla_status_string(status: int) -> str:
 
 def gtr_gla_launch_count() -> int:
     return int(load().gtr_gla_launch_count())
+
+
+PLANS = {0: "three_phase", 1: "three_phase_simt", 2: "fused_mma", 3: "fused_mma_pair", 4: "fused_tcgen05"}
+
+
+def gtr_gla_plan(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule, sm_count) -> int:
+    sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    return int(load().gtr_gla_plan(B, heads, grid_h, grid_w, d_k, d_v, chunk, sched, sm_count))
 
 
 def gtr_gla_version() -> int:

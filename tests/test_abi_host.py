@@ -113,3 +113,29 @@ def test_workspace_bytes(lib):
     nc = (100 + 15) // 16
     assert n >= 6 * nc * 32 * 64 * 4 + 6 * nc * 32 * 4
     assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 24, 16, 16, 2) == 0
+
+
+def test_dispatch_plan(lib):
+    """The kernels each schedule launches (host-only decision, 148 SMs)."""
+    plan = lambda B, heads, H, W, dk, dv, C, sched: lib.gtr_gla_plan(B, heads, H, W, dk, dv, C, sched, 148)
+    # batched: many sequences at d = 64, chunk 64 -> the tcgen05 kernel
+    assert plan(32, 12, 40, 40, 64, 64, 64, "auto") == 4
+    # latency configs and the B1 sweep: at most 16 sequences -> three phases
+    assert plan(1, 6, 40, 40, 64, 64, 64, "auto") == 0
+    assert plan(1, 6, 80, 80, 64, 64, 64, "auto") == 0
+    assert plan(1, 8, 256, 256, 128, 128, 64, "auto") == 0
+    assert plan(2, 8, 40, 40, 64, 64, 64, "auto") == 0
+    # B8 sweep: 64 sequences, d_v = 128 -> mma.sync, one chunk per tile
+    assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 2
+    # 64 sequences at d = 64: fewer than 2 per SM -> mma.sync with two chunks per tile
+    assert plan(8, 8, 64, 64, 64, 64, 64, "auto") == 3
+    assert plan(8, 8, 64, 64, 64, 64, 64, "fused_tcgen05") == 4
+    assert plan(8, 8, 64, 64, 32, 64, 64, "fused_tcgen05") == 3  # not its shape
+    assert plan(32, 12, 40, 40, 64, 64, 64, "fused") == 2
+    assert plan(32, 12, 40, 40, 64, 64, 32, "auto") == 2  # chunk 32: not the tcgen05 shape
+    assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase") == 0
+    assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase_simt") == 1
+    # invalid arguments
+    assert lib.gtr_gla_plan(1, 1, 8, 8, 16, 16, 16, 9, 148) == -1
+    assert lib.gtr_gla_plan(1, 1, 8, 8, 24, 16, 16, 0, 148) == -1
+    assert lib.gtr_gla_plan(1, 1, 8, 8, 16, 16, 16, 0, 0) == -1
