@@ -51,5 +51,11 @@ cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc
                            float *S_enter, cudaStream_t st);
 cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, const float *g,
                              const float *S_enter, const Geom &geo, __half *out, cudaStream_t st);
+// The boundary scan in two passes over segments of chunks (more parallel
+// work for long chains and few state elements); agg holds scan_agg_bytes.
+int scan_segments(int64_t nseq, int nc, int dk, int dv);
+size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv);
+cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                                  float *S_enter, float *agg, cudaStream_t st);
 void count_launch(int n = 1);
 }  // namespace gtr

@@ -8,6 +8,8 @@
 // exp() of a difference of in-chunk prefix sums, so it is safe for any gate
 // values.  It is the straightforward schedule the tensor-core kernels are
 // checked and timed against.
+#include <algorithm>
+
 #include "gla_common.cuh"
 
 namespace gtr {
@@ -139,6 +141,75 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
     }
 }
 
+// The same scan in two passes over segments of each sequence's chunks, with
+// four state elements (one float4, one key row) per thread: more independent
+// work for problems with few state elements and long chains.
+//   pass 1 (APPLY = false): the aggregate of segment s, the state leaving it
+//     from zero and the product of its gates, D_s and Gam_s;
+//   pass 2 (APPLY = true): the state entering segment s from the aggregates
+//     of segments 0..s-1, then the segment's chunks again, writing S_enter.
+// Pass 1 only reads dS; pass 2 reads each element before it writes it, so
+// S_enter may be dS.  Aggregates: [seq][nseg - 1][d_k*d_v (D) + d_k (Gam)].
+template <bool APPLY>
+__global__ void __launch_bounds__(kThreads) scan_seg_kernel(const float *dS, const float *__restrict__ gamma,
+                                                            int nseq, int nc, int dk, int dv, int L, int nseg,
+                                                            float *agg, float *S_enter) {
+    const int n4 = dk * dv / 4;
+    const int per = (n4 + blockDim.x - 1) / blockDim.x;
+    const int segs = APPLY ? nseg : nseg - 1;
+    const int64_t ss = blockIdx.x / per;
+    const int e4 = (int)(blockIdx.x % per) * blockDim.x + threadIdx.x;
+    if (e4 >= n4) return;
+    const int64_t seq = ss / segs;
+    const int seg = (int)(ss - seq * segs);
+    if (!GTR_INB(seq, nseq, BS_SIMT_SCAN)) return;
+    const int i = (4 * e4) / dv;  // the key row of the four elements
+    const int64_t aggstride = (int64_t)dk * dv + dk;
+    const int c0 = seg * L, c1 = min(nc, c0 + L);
+    float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (APPLY) {
+        const float *ab = agg + seq * (nseg - 1) * aggstride;
+        for (int s = 0; s < seg; ++s) {
+            const float4 D = reinterpret_cast<const float4 *>(ab + s * aggstride)[e4];
+            const float G = ab[s * aggstride + (int64_t)dk * dv + i];
+            S = make_float4(fmaf(G, S.x, D.x), fmaf(G, S.y, D.y), fmaf(G, S.z, D.z), fmaf(G, S.w, D.w));
+        }
+    }
+    const float4 *src = reinterpret_cast<const float4 *>(dS) + seq * nc * (int64_t)n4 + e4;
+    float4 *dst = reinterpret_cast<float4 *>(S_enter) + seq * nc * (int64_t)n4 + e4;
+    const float *gm = gamma + seq * nc * dk + i;
+    float4 xs[kAhead];
+    float as[kAhead];
+#pragma unroll
+    for (int u = 0; u < kAhead; ++u) {
+        xs[u] = c0 + u < c1 ? src[(int64_t)(c0 + u) * n4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        as[u] = c0 + u < c1 ? gm[(int64_t)(c0 + u) * dk] : 0.f;
+    }
+    float G = 1.f;
+    for (int b = c0; b < c1; b += kAhead) {
+#pragma unroll
+        for (int u = 0; u < kAhead; ++u) {
+            const int c = b + u;
+            if (c < c1) {
+                const float4 x = xs[u];
+                const float a = as[u];
+                if (c + kAhead < c1) {  // chunk c + kAhead, read before anything writes it
+                    xs[u] = src[(int64_t)(c + kAhead) * n4];
+                    as[u] = gm[(int64_t)(c + kAhead) * dk];
+                }
+                if (APPLY) dst[(int64_t)c * n4] = S;
+                S = make_float4(fmaf(a, S.x, x.x), fmaf(a, S.y, x.y), fmaf(a, S.z, x.z), fmaf(a, S.w, x.w));
+                if (!APPLY) G *= a;
+            }
+        }
+    }
+    if (!APPLY) {
+        float *ab = agg + (seq * (nseg - 1) + seg) * aggstride;
+        reinterpret_cast<float4 *>(ab)[e4] = S;
+        if ((4 * e4) % dv == 0) ab[(int64_t)dk * dv + i] = G;
+    }
+}
+
 // Phase 3: intra-chunk scores A[t][s] = sum_i q~_t[i] k_s[i] exp(b_t[i]-b_s[i])
 // for s <= t, then o_t = (q~_t * exp(b_t)) S_enter + sum_s A[t][s] v_s.
 __global__ void __launch_bounds__(kThreads) output_simt_kernel(
@@ -223,6 +294,38 @@ cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc
                            float *S_enter, cudaStream_t st) {
     dim3 grid((unsigned)((int64_t)((dk * dv + kThreads - 1) / kThreads) * nseq));
     scan_simt_kernel<<<grid, kThreads, 0, st>>>(dS, gamma, nseq, nc, dk, dv, S_enter);
+    count_launch();
+    return cudaGetLastError();
+}
+
+int scan_segments(int64_t nseq, int nc, int dk, int dv) {
+    // as many segments as keep every thread (four elements each) resident at
+    // once on a B200 (about 105k threads at this kernel's register count),
+    // each segment at least 8 chunks long
+    const int64_t threads = nseq * (int64_t)dk * dv / 4;
+    int64_t nseg = threads > 0 ? 105000 / threads : 1;
+    nseg = std::min<int64_t>(nseg, std::max(1, nc / 8));
+    return (int)std::max<int64_t>(1, nseg);
+}
+
+size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv) {
+    return (size_t)nseq * (scan_segments(nseq, nc, dk, dv) - 1) * ((size_t)dk * dv + dk) * sizeof(float);
+}
+
+cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                                  float *S_enter, float *agg, cudaStream_t st) {
+    const int nseg = scan_segments(nseq, nc, dk, dv);
+    const int L = (nc + nseg - 1) / nseg;
+    const int64_t per = ((int64_t)dk * dv / 4 + kThreads - 1) / kThreads;
+    if (nseg > 1) {
+        scan_seg_kernel<false><<<(unsigned)(nseq * (int64_t)(nseg - 1) * per), kThreads, 0, st>>>(
+            dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
+        count_launch();
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    scan_seg_kernel<true><<<(unsigned)(nseq * (int64_t)nseg * per), kThreads, 0, st>>>(dS, gamma, nseq, nc, dk, dv, L,
+                                                                                      nseg, agg, S_enter);
     count_launch();
     return cudaGetLastError();
 }

@@ -92,7 +92,7 @@ size_t tok_bytes(const Geom &g, int d, size_t elem) {
 // Internal workspaces: one grow-only, zero-initialised device buffer per
 // (device, stream, kind).  Kinds keep the schedules apart: the fused
 // kernel's control words must never be overwritten by another schedule.
-enum WsKind { WS_THREE_PHASE = 0, WS_FUSED = 1, WS_STAGING = 2, WS_STATUS = 3 };
+enum WsKind { WS_THREE_PHASE = 0, WS_FUSED = 1, WS_STAGING = 2, WS_STATUS = 3, WS_SCAN = 4 };
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
@@ -144,7 +144,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 size_t three_phase_ws(const Geom &g) {
     size_t nseq = (size_t)g.B * g.heads;
     return align256(nseq * g.nc * g.dk * g.dv * sizeof(float)) +
-           align256(nseq * g.nc * g.dk * sizeof(float));
+           align256(nseq * g.nc * g.dk * sizeof(float)) + align256(scan_agg_bytes((int64_t)nseq, g.nc, g.dk, g.dv));
 }
 
 // Fused kernels: control words (ticket, unused, four flags per sequence: the
@@ -275,7 +275,9 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
                          : summary_tc(k, v, g, geo, dS, gamma, st);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
-    e = launch_scan_v0(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, st);
+    float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
+                                           align256(nseq * geo.nc * geo.dk * sizeof(float)));
+    e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
     e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
@@ -485,8 +487,15 @@ gtr_status_t gtr_gla_boundary_scan(const float *dS, const float *gamma, int B, i
     if (overlap(rs, span(gamma, (size_t)nseq * n_chunks * d_k * 4)))
         return fail(GTR_ERR_ALIAS, "S_enter overlaps gamma%s");
     if (nseq == 0 || n_chunks == 0) return GTR_OK;
-    cudaError_t e = launch_scan_v0(dS, gamma, (int)nseq, n_chunks, d_k, d_v, S_enter,
-                                   static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *agg = nullptr;
+    const size_t ab = scan_agg_bytes(nseq, n_chunks, d_k, d_v);
+    if (ab > 0) {  // segment aggregates in an internal workspace
+        gtr_status_t s = get_workspace(ab, st, &agg, WS_SCAN);
+        if (s != GTR_OK) return s;
+    }
+    cudaError_t e = launch_scan_segmented(dS, gamma, (int)nseq, n_chunks, d_k, d_v, S_enter,
+                                          static_cast<float *>(agg), st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "boundary scan launch");
 }
 
