@@ -301,8 +301,10 @@ cudaError_t launch_scan_v0(const float *dS, const float *gamma, int nseq, int nc
 int scan_segments(int64_t nseq, int nc, int dk, int dv) {
     // as many segments as keep every thread (four elements each) resident at
     // once on a B200 (about 105k threads at this kernel's register count),
-    // each segment at least 8 chunks long
+    // each segment at least 8 chunks long; chains under 32 chunks are not
+    // worth the second launch
     const int64_t threads = nseq * (int64_t)dk * dv / 4;
+    if (nc < 32) return 1;
     int64_t nseg = threads > 0 ? 105000 / threads : 1;
     nseg = std::min<int64_t>(nseg, std::max(1, nc / 8));
     return (int)std::max<int64_t>(1, nseg);
