@@ -178,7 +178,10 @@ gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g,
  * dS, gamma (device, fp32) as written by gtr_gla_chunk_summary with
  * n_chunks chunks; S_enter (device, fp32) [B][heads][n_chunks][d_k][d_v].
  * S_enter may be the same buffer as dS (in place); any other overlap with
- * the inputs is GTR_ERR_ALIAS. */
+ * the inputs is GTR_ERR_ALIAS.  Long chains with few state elements run in
+ * two passes over segments of chunks; their segment aggregates live in an
+ * internal per-device, per-stream workspace (GTR_ERR_OOM if it cannot grow;
+ * make the first call of the largest size outside any stream capture). */
 gtr_status_t gtr_gla_boundary_scan(const float *dS, const float *gamma, int B, int heads,
                                    int n_chunks, int d_k, int d_v, float *S_enter, void *stream);
 
