@@ -417,6 +417,7 @@ def main():
                               if flush is None else
                               f"L2 flushed before every timed step ({2 * l2 / 1e6:.0f} MB write, outside the "
                               f"per-step CUDA events); {alg_bytes_total(w) / 1e6:.1f} MB per step")},
+            "token_heads_per_s": value * w.heads,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": int(launches), "clocks": clocks.summary(),
         }
