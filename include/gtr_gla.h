@@ -79,7 +79,7 @@ typedef enum {
 } gtr_status_t;
 
 typedef enum {
-    GTR_SCHED_AUTO = 0,             /* library choice: GTR_SCHED_THREE_PHASE for at most 16
+    GTR_SCHED_AUTO = 0,             /* library choice: GTR_SCHED_THREE_PHASE for at most 24
                                        sequences (B*heads); else GTR_SCHED_FUSED_TCGEN05 for its
                                        shape when there are at least 2 sequences per SM, else
                                        GTR_SCHED_FUSED */
@@ -240,7 +240,7 @@ int gtr_gla_version(void);
 /* Which kernels gtr_gla_forward_ex(..., schedule, ...) launches for this
  * problem on a device with sm_count streaming multiprocessors: a gtr_plan_t,
  * or -1 for invalid arguments.  Host-only; needs no device.  AUTO takes the
- * three-phase schedule for at most 16 sequences (B*heads), the tcgen05
+ * three-phase schedule for at most 24 sequences (B*heads), the tcgen05
  * kernel for its shape when sequences are at least 2*sm_count, else the
  * mma.sync kernel with two chunks per tile below 2*sm_count sequences when
  * d_v <= 64, one chunk per tile otherwise. */

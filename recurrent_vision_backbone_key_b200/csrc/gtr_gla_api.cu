@@ -165,8 +165,10 @@ gtr_status_t status_word(unsigned **out) {
 
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
 // At most this many (batch, head) sequences: GTR_SCHED_AUTO runs the
-// three-phase schedule (the fused chain is the bottleneck then).
-constexpr int64_t kFewSequences = 16;
+// three-phase schedule (the fused chain is the bottleneck then).  Measured at
+// 40x40, d = 64: three phases win at 24 sequences, the two-chunk fused
+// kernel from 48.
+constexpr int64_t kFewSequences = 24;
 
 // Streaming multiprocessors of the current device (cached per device).
 cudaError_t sm_count(int *out) {

@@ -120,11 +120,13 @@ def test_dispatch_plan(lib):
     plan = lambda B, heads, H, W, dk, dv, C, sched: lib.gtr_gla_plan(B, heads, H, W, dk, dv, C, sched, 148)
     # batched: many sequences at d = 64, chunk 64 -> the tcgen05 kernel
     assert plan(32, 12, 40, 40, 64, 64, 64, "auto") == 4
-    # latency configs and the B1 sweep: at most 16 sequences -> three phases
+    # latency configs and the B1 sweep: at most 24 sequences -> three phases
     assert plan(1, 6, 40, 40, 64, 64, 64, "auto") == 0
     assert plan(1, 6, 80, 80, 64, 64, 64, "auto") == 0
     assert plan(1, 8, 256, 256, 128, 128, 64, "auto") == 0
     assert plan(2, 8, 40, 40, 64, 64, 64, "auto") == 0
+    assert plan(2, 12, 40, 40, 64, 64, 64, "auto") == 0   # 24 sequences
+    assert plan(5, 5, 40, 40, 64, 64, 64, "auto") == 3    # 25: the two-chunk fused kernel
     # B8 sweep: 64 sequences, d_v = 128 -> mma.sync, one chunk per tile
     assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 2
     # 64 sequences at d = 64: fewer than 2 per SM -> mma.sync with two chunks per tile
