@@ -141,7 +141,7 @@ struct UmmaLayout {
     static constexpr uint32_t V = 16384;       // v tile (also read as MN-major)
     static constexpr uint32_t P = 24576;       // exact path's staging, then the masked scores,
                                                // then the output staging
-    static constexpr uint32_t VEC = 32768;     // gamma_c[64], sc[64], sub-chunk totals [4][64] (fp32)
+    static constexpr uint32_t VEC = 32768;     // gamma_c[64], unused[64], sub-chunk totals [4][64] (fp32)
     static constexpr uint32_t ROW = VEC + 6 * 64 * 4;  // int64 [64]
     static constexpr uint32_t MISC = ROW + 64 * 8;     // tile, tmem base, mbarrier (8-aligned)
     static constexpr uint32_t BYTES = MISC + 64;
@@ -165,8 +165,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tr = lane >> 2, kc = 2 * (lane & 3);
     float *vGc = reinterpret_cast<float *>(base + L::VEC);
-    float *vSc = vGc + 64;
-    float *vTot = vSc + 64;  // [4][64]
+    float *vTot = vGc + 128;  // [4][64]
     int64_t *sRow = reinterpret_cast<int64_t *>(base + L::ROW);
     int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [2] tmem base; mbar at +16
     const uint32_t mbar = base_addr + L::MISC + 16;
@@ -293,7 +292,6 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         tc_fence_before();
         // the whole-chunk form needs the gate range and |q~| <= 16 (qh then fits fp16)
         const bool exact = __syncthreads_or(!gam_ok || fmaxf(qm.x, qm.y) * qscale > 16.f) != 0;
-        if (warp == 0) *reinterpret_cast<float2 *>(vSc + d0) = exact ? make_float2(1.f, 1.f) : gam;
 
         // Two MMA passes through the same 64 TMEM columns.  Pass 1: A = qh ke^T
         // (whole-chunk form only) in TMEM lanes 0-15 of each 32-lane group and
@@ -473,10 +471,11 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             }
         }
         // S'^T = (sc . S_enter)^T as the K-major B operand (rows: value
-        // columns), over ke (pass 1 is complete)
+        // columns), over ke (pass 1 is complete); sc = gamma_c (written before
+        // the barrier that decided `exact`) or 1 in the exact form
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
-            const float2 sc = *reinterpret_cast<const float2 *>(vSc + 8 * n + kc);
+            const float2 sc = exact ? make_float2(1.f, 1.f) : *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
             const int dv0 = 16 * warp + tr, dk = 8 * n + kc;
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
             *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
