@@ -107,11 +107,12 @@ typedef enum {
  *   [B][N][heads][d_v], written in full (every token, every head);
  *   direction: gtr_dir_t; chunk: tokens per chunk of the chunkwise schedule.
  * out must not overlap q, k, v or g (GTR_ERR_ALIAS).  Uses an internal
- * per-device, per-stream workspace that grows on demand (GTR_ERR_OOM if it
- * cannot); a call that has to grow it synchronises the device, so make the
- * first call of the largest size on that stream outside any stream capture.
- * After that, calls on the stream can be captured into a CUDA graph and
- * replayed (the fused schedules reset their control words inside the graph). */
+ * per-device, per-stream workspace that grows on demand, in stream order on
+ * `stream` (cudaFreeAsync / cudaMallocAsync / cudaMemsetAsync; GTR_ERR_OOM if
+ * it cannot).  Growing cannot be captured: a call that needs to grow it
+ * inside a stream capture returns GTR_ERR_INVALID_ARG, so make the first call
+ * of the largest size on that stream outside any capture.  After that, calls
+ * on the stream can be captured into a CUDA graph and replayed. */
 gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const float *g,
                              int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                              int direction, int chunk, void *out, void *stream);
@@ -131,29 +132,38 @@ gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, con
  * forward and the downloads of earlier slices.  Those streams start after the
  * work queued on `stream` before the call.  Device staging buffers come from
  * the internal workspace.  Page-locked host buffers give the fastest copies
- * and the overlap; pageable ones work too. */
+ * and the overlap; pageable ones work too.  out must not overlap q, k, v or g
+ * (GTR_ERR_ALIAS).  Returns GTR_ERR_TIMEOUT if a bounded wait inside the
+ * forward gave up.  On any error, the internal streams are drained before
+ * the call returns: no copy touches the caller's buffers afterwards. */
 gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, const float *g,
                                   int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                   int direction, int chunk, void *out, void *stream);
 
 /* gtr_gla_forward without any device allocation.  The GTR pages have no
  * counterpart to this call; it exists for callers that cannot let a library
- * call cudaMalloc while they run: hosts that own every byte of device memory
- * through their own allocator or a fixed budget (engine plugins, serving
- * runtimes) and real-time loops that forbid allocation after start-up.
- * Same arguments, layouts, checks and result as gtr_gla_forward (three-phase
- * schedule).  Its scratch is a 16 MiB array in the library's own device
- * memory, which every GPU that loads the library holds until the process
- * exits.  Problems needing more, i.e. B*heads*ceil(N/chunk)*d_k*(d_v+1)*4
- * bytes above 16 MiB (after 256-byte rounding of the two parts), are
- * rejected with GTR_ERR_UNSUPPORTED_SHAPE and nothing is launched.
- * The first call on a device looks up that device's scratch address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * All calls on a device share the one scratch array: calls whose kernels may
- * overlap on the GPU (different streams without ordering between them)
- * race and give wrong results; order them on one stream or with events.
- * The scratch keeps the last call's contents; every entry a call reads is
- * first written by the same call, so nothing needs clearing. */
+ * allocate device memory while they run: hosts that own every byte of device
+ * memory through their own allocator or a fixed budget (engine plugins,
+ * serving runtimes) and real-time loops that forbid allocation after
+ * start-up.  Arguments, layouts and error statuses as gtr_gla_forward (its
+ * own argument checks, the same codes; the failure text is set as for every
+ * other entry point).  It runs the CUDA-core versions of the three phases
+ * (chunk summaries, boundary scan, chunk outputs), so its result matches
+ * gtr_gla_forward within the forward's tolerance (max |difference| <=
+ * 2e-3 * max |output|), not bit for bit.  Its scratch is a 16 MiB array in
+ * the library's own device memory, which every GPU that loads the library
+ * holds until the process exits.  Problems needing more, i.e.
+ * B*heads*ceil(N/chunk)*d_k*(d_v+1)*4 bytes above 16 MiB (after 256-byte
+ * rounding of the two parts), are rejected with GTR_ERR_UNSUPPORTED_SHAPE and
+ * nothing is launched.  The first call on a device (and the first after the
+ * device's context was recreated, e.g. by cudaDeviceReset) looks up that
+ * device's scratch address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  All calls on a device share the one scratch
+ * array: calls whose kernels may overlap on the GPU (different streams
+ * without ordering between them) race and give wrong results; order them on
+ * one stream or with events.  The scratch keeps the last call's contents;
+ * every entry a call reads is first written by the same call, so nothing
+ * needs clearing. */
 gtr_status_t gtr_gla_forward_noalloc(const void *q, const void *k, const void *v, const float *g,
                                      int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                      int direction, int chunk, void *out, void *stream);
@@ -197,24 +207,35 @@ gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, c
                                   int d_k, int d_v, int direction, int chunk, void *out,
                                   void *stream);
 
-/* Bytes of internal device workspace one gtr_gla_forward_ex call of this
- * size and schedule uses (informational; 0 for invalid arguments). */
+/* Bytes of internal device workspace (per device and stream) that a
+ * gtr_gla_forward call of this size may use: the larger of what its
+ * schedules need, plus the stream's status word (informational; 0 for
+ * invalid arguments or an empty problem). */
 size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
-                               int chunk, int schedule);
+                               int chunk);
+
+/* The same for gtr_gla_forward_ex(..., schedule, ...) (gtr_schedule_t). */
+size_t gtr_gla_workspace_bytes_ex(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                  int chunk, int schedule);
 
 /* Synchronises `stream`, then returns and clears the device-side status
- * word of the current device: GTR_OK, or GTR_ERR_TIMEOUT if a bounded wait
- * inside a kernel gave up since the last query. */
+ * word of (current device, stream): GTR_OK, or GTR_ERR_TIMEOUT if a bounded
+ * wait inside a kernel enqueued on `stream` gave up since the last query.
+ * Each stream has its own word, so a query never sees or clears another
+ * stream's report. */
 gtr_status_t gtr_gla_get_last_device_status(void *stream);
 
 /* Test hook for the bounded wait of the fused schedules: runs
  * gtr_gla_forward_ex(..., schedule, ...) for schedule GTR_SCHED_AUTO,
  * GTR_SCHED_FUSED or GTR_SCHED_FUSED_TCGEN05 (others: GTR_ERR_INVALID_ARG),
  * except that the tile of sequence hold_seq (= b*heads + h), chunk hold_chunk
- * never publishes its boundary state, and each wait gives up after spin_limit
- * polls (> 0).  The successor tile then times out, records GTR_ERR_TIMEOUT in
- * the device status word (read it with gtr_gla_get_last_device_status) and
- * the kernel still finishes; its output is not meaningful.  hold_seq = -1
+ * never publishes its boundary state, and the wait for a predecessor's
+ * boundary state gives up after spin_limit polls (> 0, else
+ * GTR_ERR_INVALID_ARG).  spin_limit bounds only that wait: a CTA's waits for
+ * its own tensor-core work keep a fixed bound of about one second.  The
+ * successor tile then times out, records GTR_ERR_TIMEOUT in the stream's
+ * device status word (read it with gtr_gla_get_last_device_status) and the
+ * kernel still finishes; its output is not meaningful.  hold_seq = -1
  * disables the hold. */
 gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const void *v, const float *g,
                                          int B, int heads, int grid_h, int grid_w, int d_k, int d_v,

@@ -58,4 +58,8 @@ size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv);
 cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
                                   float *S_enter, float *agg, cudaStream_t st);
 void count_launch(int n = 1);
+// Records the calling thread's failure text (returned by gtr_gla_last_error)
+// and returns s; clear_last_error empties it at the start of a call.
+int set_last_error(int s, const char *msg);
+void clear_last_error();
 }  // namespace gtr

@@ -98,9 +98,24 @@ __device__ __forceinline__ void tmem_ld_16x64(uint32_t taddr, float (&r)[32]) {
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(mbar), "r"(count) : "memory");
 }
-// Bounded wait for the given phase parity; returns false if it gave up.
-__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long long limit) {
-    for (long long i = 0; i < limit; ++i) {
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+
+// Bound of a wait for tensor-core work this CTA issued itself: about one
+// second of wall time.  Fixed, so that no caller-tunable limit can make a
+// CTA give up on MMAs that are still in flight.
+constexpr uint64_t kMmaWaitNs = 1000000000ull;
+
+// Wait for the given phase parity of an mbarrier that tensor-core commits
+// complete; returns false only if the fixed bound ran out (an error is
+// recorded by the caller; the CTA keeps its program order, so its TMEM
+// deallocation still follows its last commit).
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -110,8 +125,14 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long l
             : "r"(mbar), "r"(parity)
             : "memory");
         if (done) return true;
+        if ((i & 63u) == 0) {
+            const uint64_t t = global_ns();
+            if (i == 0)
+                t0 = t;
+            else if (t - t0 > kMmaWaitNs)
+                return false;
+        }
     }
-    return false;
 }
 
 // Byte offset of element (row, col) in a 64 x 64 fp16 tile with 128-byte rows,
@@ -417,7 +438,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             for (int n = 0; n < KT; ++n) Se[n][0] = Se[n][1] = Se[n][2] = Se[n][3] = 0.f;
         }
 
-        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        if (!mbar_wait(mbar, phase) && tid == 0) atomicOr(args.status, 6u);
         phase ^= 1u;
         tc_fence_after();
         // ---- publish this warp's slice of S_leave = diag(gamma_c) S_enter + dS,
@@ -501,7 +522,7 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             }
             umma_commit(mbar);
         }
-        if (!mbar_wait(mbar, phase, args.spin_limit * 64) && tid == 0) atomicOr(args.status, 6u);
+        if (!mbar_wait(mbar, phase) && tid == 0) atomicOr(args.status, 6u);
         phase ^= 1u;
         tc_fence_after();
 

@@ -115,24 +115,33 @@ gtr_status_t get_workspace(size_t bytes, cudaStream_t st, void **out, int kind =
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(g_ws_mu);
-    Workspace &w = g_ws[WsKey{dev, kind == WS_STATUS ? nullptr : st, kind}];
+    Workspace &w = g_ws[WsKey{dev, st, kind}];
     if (w.bytes < bytes) {
+        // Growing is stream-ordered on `st` (the only stream that uses this
+        // workspace): the old buffer is freed after the work already queued
+        // on it, the new one is allocated and zeroed in stream order.  An
+        // allocation cannot be recorded into a stream capture.
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        if ((e = cudaStreamIsCapturing(st, &cap)) != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+        if (cap != cudaStreamCaptureStatusNone)
+            return fail(GTR_ERR_INVALID_ARG,
+                        "the internal workspace must grow, which cannot happen inside a stream capture; "
+                        "make a first call of this size on this stream before capturing%s");
         if (w.ptr) {
-            e = cudaStreamSynchronize(st);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-            cudaFree(w.ptr);
+            e = cudaFreeAsync(w.ptr, st);
             w.ptr = nullptr;
             w.bytes = 0;
+            if (e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
         }
         size_t want = (bytes + 0xFFFFF) & ~(size_t)0xFFFFF;  // round up to 1 MiB
-        e = cudaMalloc(&w.ptr, want);
+        e = cudaMallocAsync(&w.ptr, want, st);
         if (e != cudaSuccess) {
             w.ptr = nullptr;
             cudaGetLastError();
             return fail(GTR_ERR_OOM, "workspace allocation failed%s");
         }
-        e = cudaMemset(w.ptr, 0, want);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset");
+        e = cudaMemsetAsync(w.ptr, 0, want, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
         w.bytes = want;
     }
     *out = w.ptr;
@@ -155,14 +164,16 @@ size_t fused_ws(const Geom &g) {
     return fused_ctrl_bytes(g) + (size_t)g.B * g.heads * 2 * g.dk * g.dv * sizeof(float);
 }
 
-// Device status word of the current device (zeroed at creation).
-gtr_status_t status_word(unsigned **out) {
+// Device status word of (current device, stream), zeroed at creation: the
+// kernels a call enqueues on `st` record a bounded wait that gave up here.
+gtr_status_t status_word(cudaStream_t st, unsigned **out) {
     void *p = nullptr;
-    gtr_status_t s = get_workspace(256, nullptr, &p, WS_STATUS);
+    gtr_status_t s = get_workspace(256, st, &p, WS_STATUS);
     *out = static_cast<unsigned *>(p);
     return s;
 }
 
+constexpr int kSchedLast = GTR_SCHED_FUSED_TCGEN05;  // largest gtr_schedule_t value
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
 // At most this many (batch, head) sequences: GTR_SCHED_AUTO runs the
 // three-phase schedule (the fused chain is the bottleneck then).  Measured at
@@ -229,7 +240,7 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     gtr_status_t s = get_workspace(fused_ws(geo), st, &ws, WS_FUSED);
     if (s != GTR_OK) return s;
     unsigned *status = nullptr;
-    if ((s = status_word(&status)) != GTR_OK) return s;
+    if ((s = status_word(st, &status)) != GTR_OK) return s;
     TcArgs a = make_args(q, k, v, g, geo);
     a.out = out;
     a.ctrl = static_cast<int *>(ws);
@@ -294,7 +305,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     bool empty = false;
     gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
     if (s != GTR_OK) return s;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05)
+    if (schedule < GTR_SCHED_AUTO || schedule > kSchedLast)
         return fail(GTR_ERR_INVALID_ARG, "bad schedule%s");
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out))
@@ -318,6 +329,15 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
 }
 
 }  // namespace
+
+// The calling thread's failure text, for entry points in other translation
+// units (gtr_gla_last_error returns it).
+int set_last_error(int s, const char *msg) {
+    std::snprintf(t_err, sizeof t_err, "%s", msg);
+    return s;
+}
+void clear_last_error() { t_err[0] = '\0'; }
+
 }  // namespace gtr
 
 using namespace gtr;
@@ -378,9 +398,15 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
     gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
     if (s != GTR_OK) return s;
     if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    const size_t nq = tok_bytes(geo, d_k, 2), nv = tok_bytes(geo, d_v, 2), ng = tok_bytes(geo, d_k, 4);
+    {
+        const Range ro = span(out, nv);
+        if (overlap(ro, span(q, nq)) || overlap(ro, span(k, nq)) || overlap(ro, span(v, nv)) ||
+            overlap(ro, span(g, ng)))
+            return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
+    }
     if (empty) return GTR_OK;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const size_t nq = tok_bytes(geo, d_k, 2), nv = tok_bytes(geo, d_v, 2), ng = tok_bytes(geo, d_k, 4);
     const size_t bq = align256(nq), bv = align256(nv), bg = align256(ng);
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -420,9 +446,18 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
     // slices of whole batch items, none below kHostSliceMinBytes of traffic
     const size_t total = 2 * nq + 2 * nv + ng;
     int S = (int)std::min<size_t>(std::min<size_t>((size_t)B, kHostSlices), std::max<size_t>(1, total / kHostSliceMinBytes));
+    // On an error part-way, wait for what was already queued on the internal
+    // streams before returning: no copy may still touch the caller's host
+    // buffers after this call returns.
+    auto drain = [&](gtr_status_t r) {
+        cudaStreamSynchronize(hp->up);
+        cudaStreamSynchronize(hp->run);
+        cudaStreamSynchronize(hp->down);
+        return r;
+    };
     // the uploads start after the work already queued on the caller's stream
     if ((e = cudaEventRecord(hp->start, st)) != cudaSuccess || (e = cudaStreamWaitEvent(hp->up, hp->start, 0)) != cudaSuccess)
-        return cuda_fail(e, "pipeline start");
+        return drain(cuda_fail(e, "pipeline start"));
     for (int i = 0; i < S; ++i) {
         const int b0 = (int)((int64_t)B * i / S), b1 = (int)((int64_t)B * (i + 1) / S), nb = b1 - b0;
         const size_t per_b = (size_t)geo.N * heads;  // token-heads per batch item
@@ -434,17 +469,18 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
             (e = cudaMemcpyAsync(dg + og, hg + og, sg, cudaMemcpyHostToDevice, hp->up)) != cudaSuccess ||
             (e = cudaEventRecord(hp->up_done[i], hp->up)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(hp->run, hp->up_done[i], 0)) != cudaSuccess)
-            return cuda_fail(e, "host-to-device copy");
+            return drain(cuda_fail(e, "host-to-device copy"));
         s = forward_impl(dq + oq, dk_ + oq, dv_ + ov, reinterpret_cast<const float *>(dg + og), nb, heads, grid_h,
                          grid_w, d_k, d_v, direction, chunk, GTR_SCHED_AUTO, dout + ov, hp->run);
-        if (s != GTR_OK) return s;
+        if (s != GTR_OK) return drain(s);
         if ((e = cudaEventRecord(hp->run_done[i], hp->run)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(hp->down, hp->run_done[i], 0)) != cudaSuccess ||
             (e = cudaMemcpyAsync(hout + ov, dout + ov, sv, cudaMemcpyDeviceToHost, hp->down)) != cudaSuccess)
-            return cuda_fail(e, "device-to-host copy");
+            return drain(cuda_fail(e, "device-to-host copy"));
     }
-    if ((e = cudaStreamSynchronize(hp->down)) != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-    return GTR_OK;
+    if ((e = cudaStreamSynchronize(hp->down)) != cudaSuccess) return drain(cuda_fail(e, "cudaStreamSynchronize"));
+    // the forward ran on the internal compute stream: report its bounded waits here
+    return gtr_gla_get_last_device_status(hp->run);
 }
 
 gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g, int B, int heads,
@@ -528,29 +564,45 @@ gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, c
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk output launch");
 }
 
-size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
-                               int chunk, int schedule) {
+size_t gtr_gla_workspace_bytes_ex(int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
+                                  int chunk, int schedule) {
     Geom geo;
     bool empty = false;
     if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return 0;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05 || empty) return 0;
+    if (schedule < GTR_SCHED_AUTO || schedule > kSchedLast || empty) return 0;
+    const size_t status = 256;  // the stream's device status word
     if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT)
-        return three_phase_ws(geo);
-    return fused_ws(geo);
+        return three_phase_ws(geo) + status;
+    if (schedule == GTR_SCHED_AUTO) return std::max(three_phase_ws(geo), fused_ws(geo)) + status;
+    return fused_ws(geo) + status;
+}
+
+size_t gtr_gla_workspace_bytes(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int chunk) {
+    return gtr_gla_workspace_bytes_ex(B, heads, grid_h, grid_w, d_k, d_v, chunk, GTR_SCHED_AUTO);
 }
 
 gtr_status_t gtr_gla_get_last_device_status(void *stream) {
     t_err[0] = '\0';
-    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     unsigned *word = nullptr;
-    gtr_status_t s = status_word(&word);
-    if (s != GTR_OK) return s;
+    {
+        std::lock_guard<std::mutex> lk(g_ws_mu);
+        auto it = g_ws.find(WsKey{dev, st, WS_STATUS});
+        if (it != g_ws.end()) word = static_cast<unsigned *>(it->second.ptr);
+    }
+    if (!word) return GTR_OK;  // nothing that reports has run on this stream
     unsigned v = 0;
-    if ((e = cudaMemcpy(&v, word, sizeof v, cudaMemcpyDeviceToHost)) != cudaSuccess)
+    if ((e = cudaMemcpyAsync(&v, word, sizeof v, cudaMemcpyDeviceToHost, st)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(st)) != cudaSuccess)
         return cuda_fail(e, "status read");
     if (v != 0) {
-        if ((e = cudaMemset(word, 0, sizeof v)) != cudaSuccess) return cuda_fail(e, "status reset");
+        if ((e = cudaMemsetAsync(word, 0, sizeof v, st)) != cudaSuccess ||
+            (e = cudaStreamSynchronize(st)) != cudaSuccess)
+            return cuda_fail(e, "status reset");
         return fail(GTR_ERR_TIMEOUT, "a bounded device wait gave up%s");
     }
     return GTR_OK;
@@ -635,7 +687,7 @@ int gtr_gla_plan(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int
     Geom geo;
     bool empty = false;
     if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return -1;
-    if (schedule < GTR_SCHED_AUTO || schedule > GTR_SCHED_FUSED_TCGEN05 || sm_count < 1) return -1;
+    if (schedule < GTR_SCHED_AUTO || schedule > kSchedLast || sm_count < 1) return -1;
     return (int)plan_for(geo, schedule, sm_count);
 }
 

@@ -42,7 +42,8 @@ SIGNATURES = {
     "gtr_gla_chunk_summary": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gtr_gla_boundary_scan": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
-    "gtr_gla_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "gtr_gla_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I]),
+    "gtr_gla_workspace_bytes_ex": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "gtr_gla_get_last_device_status": (_I, [_P]),
     "gtr_gla_debug_forward_fused": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                          ctypes.c_longlong, _P, _P]),
@@ -186,8 +187,13 @@ def gtr_gla_chunk_output(q, k, v, g, S_enter, B, heads, grid_h, grid_w, d_k, d_v
                                        _addr(out), _stream(stream))
 
 
-def gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule=0) -> int:
-    return int(load().gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule))
+def gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk) -> int:
+    return int(load().gtr_gla_workspace_bytes(B, heads, grid_h, grid_w, d_k, d_v, chunk))
+
+
+def gtr_gla_workspace_bytes_ex(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule) -> int:
+    sched = SCHEDULES[schedule] if isinstance(schedule, str) else int(schedule)
+    return int(load().gtr_gla_workspace_bytes_ex(B, heads, grid_h, grid_w, d_k, d_v, chunk, sched))
 
 
 def gtr_gla_get_last_device_status(stream=None) -> int:

@@ -109,10 +109,15 @@ def test_phase_entry_points_validate(lib):
 
 def test_workspace_bytes(lib):
     # three-phase: dS (nseq*nc*dk*dv fp32) + gamma (nseq*nc*dk fp32), 256-byte aligned
-    n = lib.gtr_gla_workspace_bytes(2, 3, 10, 10, 32, 64, 16, 2)
+    n = lib.gtr_gla_workspace_bytes_ex(2, 3, 10, 10, 32, 64, 16, "three_phase")
     nc = (100 + 15) // 16
     assert n >= 6 * nc * 32 * 64 * 4 + 6 * nc * 32 * 4
-    assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 24, 16, 16, 2) == 0
+    assert lib.gtr_gla_workspace_bytes_ex(1, 1, 4, 4, 24, 16, 16, "three_phase") == 0
+    # the seven-argument form is the bound over the schedules AUTO may take
+    n7 = lib.gtr_gla_workspace_bytes(2, 3, 10, 10, 32, 64, 16)
+    assert n7 >= n and n7 >= lib.gtr_gla_workspace_bytes_ex(2, 3, 10, 10, 32, 64, 16, "fused")
+    assert lib.gtr_gla_workspace_bytes(0, 3, 10, 10, 32, 64, 16) == 0
+    assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 24, 16, 16) == 0
 
 
 def test_dispatch_plan(lib):
@@ -141,3 +146,45 @@ def test_dispatch_plan(lib):
     assert lib.gtr_gla_plan(1, 1, 8, 8, 16, 16, 16, 9, 148) == -1
     assert lib.gtr_gla_plan(1, 1, 8, 8, 24, 16, 16, 0, 148) == -1
     assert lib.gtr_gla_plan(1, 1, 8, 8, 16, 16, 16, 0, 0) == -1
+
+
+def test_debug_hook_validates_spin_limit(lib):
+    """The test hook's spin limit bounds only the wait for a predecessor's
+    boundary state and must be positive; waits for a CTA's own tensor-core
+    work have a fixed bound the caller cannot lower."""
+    cdll = lib.load()
+    args = [A, 2 * A, 3 * A, 4 * A, 1, 2, 16, 16, 64, 64, 0, 64, 4, 1, 1]
+    for bad in (0, -1):
+        assert cdll.gtr_gla_debug_forward_fused(*args, bad, 5 * A, 0) == 1
+        assert "spin_limit" in lib.last_error()
+    assert cdll.gtr_gla_debug_forward_fused(*args[:12], 2, 1, 1, 100, 5 * A, 0) == 1  # schedule
+
+
+def test_noalloc_error_paths_set_text(lib):
+    """Every refusal of the no-allocation entry point names its reason."""
+    cases = [
+        (dict(q=None), 1, "null"),
+        (dict(direction=7), 1, "direction"),
+        (dict(B=-1), 1, "negative"),
+        (dict(d_k=48), 2, "d_k"),
+        (dict(chunk=128), 2, "chunk"),
+        (dict(q=A + 8), 3, "aligned"),
+        (dict(out=A + 512), 4, "overlaps"),
+        (dict(B=64, heads=64, grid_h=64, grid_w=64, d_k=128, d_v=128, out=1 << 40), 2, "16 MiB"),
+    ]
+    for kw, want, text in cases:
+        args = dict(q=A, k=2 * A, v=3 * A, g=4 * A, B=1, heads=2, grid_h=4, grid_w=4, d_k=16,
+                    d_v=16, direction=0, chunk=16, out=5 * A, stream=0)
+        args.update(kw)
+        assert lib.gtr_gla_forward_noalloc(**args) == want, kw
+        assert text in lib.last_error(), (kw, lib.last_error())
+
+
+def test_host_entry_alias_check(lib):
+    """The host-buffer entry point refuses an output that overlaps an input
+    before it touches the device."""
+    import torch
+    q = torch.zeros((1, 16, 2, 16), dtype=torch.float16)
+    g = torch.zeros((1, 16, 2, 16), dtype=torch.float32)
+    st = lib.gtr_gla_forward_host(q, q, q, g, 1, 2, 4, 4, 16, 16, 0, 16, q, 0)
+    assert st == 4 and "overlaps" in lib.last_error()

@@ -2,12 +2,15 @@
 library allocate device memory while they run (hosts that own all device
 memory through their own allocator or budget, real-time loops that forbid
 allocation after start-up).  Its scratch is a fixed 16 MiB array inside the
-library, so the test checks, through the C ABI, that two calls in a row give
-the same result as gtr_gla_forward within the parity tolerance, and that a
-problem too large for the fixed scratch is refused without a launch.
+library that every call reuses, so the tests call it through the C ABI
+several times in a row, on problems of different sizes, and check every
+result against gtr_gla_forward and against the fp64 oracle within the
+forward's tolerance; a problem too large for the fixed scratch is refused
+without a launch.
 
 This file is collected last on purpose and works in a fresh process too.
 """
+import numpy as np
 import pytest
 import torch
 
@@ -29,22 +32,41 @@ def _lib():
 
 
 def _rel(a, b):
-    return ((a.float() - b.float()).abs().max() / b.float().abs().max().clamp_min(1e-30)).item()
+    a = a.float().cpu().numpy().astype(np.float64) if hasattr(a, "cpu") else np.asarray(a)
+    b = b.float().cpu().numpy().astype(np.float64) if hasattr(b, "cpu") else np.asarray(b)
+    return float(np.abs(a - b).max() / max(np.abs(b).max(), 1e-30))
 
 
-def test_noalloc_matches_forward_on_two_calls():
-    # GTR-S-like 640x640 grid (40x40 tokens, 6 heads, d=64) fits the scratch.
-    H, W, heads, d = 40, 40, 6, 64
-    for call, (seed, direction) in enumerate([(1, 0), (2, 2)]):
-        q, k, v, g = (x.cuda() for x in make_inputs(1, H, W, heads, d, d, seed=seed))
-        ref = torch.empty_like(v)
-        gtr_gla.check(gtr_gla.gtr_gla_forward(q, k, v, g, 1, heads, H, W, d, d, direction, 64, ref))
-        out = torch.full_like(v, float("nan"))
-        st = gtr_gla.gtr_gla_forward_noalloc(q, k, v, g, 1, heads, H, W, d, d, direction, 64, out)
-        assert st == 0, gtr_gla.gtr_gla_status_string(st)
-        torch.cuda.synchronize()
+def _noalloc(q, k, v, g, B, heads, H, W, dk, dv, direction, chunk):
+    out = torch.full_like(v, float("nan"))
+    st = gtr_gla.gtr_gla_forward_noalloc(q, k, v, g, B, heads, H, W, dk, dv, direction, chunk, out)
+    assert st == 0, (gtr_gla.gtr_gla_status_string(st), gtr_gla.last_error())
+    torch.cuda.synchronize()
+    return out
+
+
+def test_noalloc_matches_forward_and_oracle_on_consecutive_calls(oracle_mod):
+    """Four calls in a row: the GTR-S-like 40x40 grid (6 heads, d=64) twice
+    with other inputs and directions, then a d_k=d_v=128 problem (the widest
+    shared-memory layout of the CUDA-core output kernel), then a smaller grid
+    again, so leftover scratch contents of a larger call are never read."""
+    cases = [
+        (1, 40, 40, 6, 64, 64, 0, 1),
+        (1, 40, 40, 6, 64, 64, 2, 2),
+        (1, 32, 32, 2, 128, 128, 3, 3),
+        (2, 9, 13, 3, 32, 64, 1, 4),
+    ]
+    for call, (B, H, W, heads, dk, dv, direction, seed) in enumerate(cases):
+        qc, kc, vc, gc = make_inputs(B, H, W, heads, dk, dv, seed=seed)
+        q, k, v, g = (x.cuda() for x in (qc, kc, vc, gc))
+        out = _noalloc(q, k, v, g, B, heads, H, W, dk, dv, direction, 64)
         assert torch.isfinite(out).all(), f"call {call}"
-        assert _rel(out, ref) <= REL_TOL, f"call {call}"
+        ref = torch.empty_like(v)
+        gtr_gla.check(gtr_gla.gtr_gla_forward(q, k, v, g, B, heads, H, W, dk, dv, direction, 64, ref))
+        torch.cuda.synchronize()
+        assert _rel(out, ref) <= REL_TOL, f"call {call} against gtr_gla_forward"
+        exact = oracle_mod.gla_serial(qc, kc, vc, gc, H, W, direction)
+        assert _rel(out, exact) <= REL_TOL, f"call {call} against the oracle"
 
 
 def test_noalloc_refuses_oversized_problem():
@@ -55,4 +77,5 @@ def test_noalloc_refuses_oversized_problem():
     before = gtr_gla.gtr_gla_launch_count()
     st = gtr_gla.gtr_gla_forward_noalloc(q, q, q, g, 32, 12, 40, 40, 64, 64, 0, 64, out)
     assert st == 2  # GTR_ERR_UNSUPPORTED_SHAPE
+    assert "16 MiB" in gtr_gla.last_error()
     assert gtr_gla.gtr_gla_launch_count() == before
