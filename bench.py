@@ -64,7 +64,7 @@ def planned_kernel(w, schedule):
     plan = gtr_gla.gtr_gla_plan(w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, w.chunk, schedule, sms)
     names = {0: "three-phase (summary, scan, output)", 1: "three-phase on CUDA cores",
              2: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,1>", 3: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,2>",
-             4: "gla_umma_kernel"}
+             4: "gla_umma_kernel", 5: f"gla_walk_kernel<{w.d_k},WALK_SEQ>"}
     return plan, names.get(plan, "unknown")
 
 
@@ -292,7 +292,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS))
-    ap.add_argument("--schedule", default="auto", choices=["auto", "fused", "three_phase", "three_phase_simt", "fused_tcgen05"])
+    ap.add_argument("--schedule", default="auto", choices=sorted(gtr_gla.SCHEDULES))
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)

@@ -79,26 +79,35 @@ typedef enum {
 } gtr_status_t;
 
 typedef enum {
-    GTR_SCHED_AUTO = 0,             /* library choice: GTR_SCHED_THREE_PHASE for at most 24
-                                       sequences (B*heads); else GTR_SCHED_FUSED_TCGEN05 for its
-                                       shape when there are at least 2 sequences per SM, else
-                                       GTR_SCHED_FUSED */
+    GTR_SCHED_AUTO = 0,             /* library choice (gtr_gla_plan): GTR_SCHED_THREE_PHASE for at
+                                       most 24 sequences (B*heads); else GTR_SCHED_WALK_TCGEN05
+                                       for its shapes; else the fused mma.sync kernel */
     GTR_SCHED_FUSED = 1,            /* one kernel (mma.sync tensor cores): summaries, chained
                                        boundary states, outputs */
-    GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output (tensor cores) */
+    GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output on tensor
+                                       cores (tcgen05 for chunk 64, d_k in {32, 64, 128},
+                                       d_v in {64, 128}; mma.sync otherwise) */
     GTR_SCHED_THREE_PHASE_SIMT = 3, /* the same three phases on CUDA cores only (comparison) */
-    GTR_SCHED_FUSED_TCGEN05 = 4     /* fused, whole-chunk products on tcgen05 tensor cores with
-                                       tensor-memory accumulators (d_k = d_v = 64, chunk 64;
-                                       other shapes run GTR_SCHED_FUSED) */
+    GTR_SCHED_FUSED_TCGEN05 = 4,    /* fused, one (sequence, chunk) tile per CTA with the boundary
+                                       state chained between CTAs, whole-chunk products on
+                                       tcgen05 (d_k = d_v = 64, chunk 64; other shapes run
+                                       GTR_SCHED_FUSED) */
+    GTR_SCHED_WALK_TCGEN05 = 5      /* one CTA per (sequence, 64 value columns) walks the chunks
+                                       in scan order with its slice of the state on chip,
+                                       whole-chunk products on tcgen05 (chunk 64, d_k in
+                                       {32, 64, 128}, d_v in {64, 128}; other shapes run
+                                       GTR_SCHED_FUSED) */
 } gtr_schedule_t;
 
 /* The kernels a schedule launches (gtr_gla_plan). */
 typedef enum {
-    GTR_PLAN_THREE_PHASE = 0,       /* chunk summaries, boundary scan, chunk outputs (tensor cores) */
+    GTR_PLAN_THREE_PHASE = 0,       /* chunk summaries, boundary scan, chunk outputs (tensor cores:
+                                       tcgen05 for the walk kernel's shapes, else mma.sync) */
     GTR_PLAN_THREE_PHASE_SIMT = 1,  /* the same three phases on CUDA cores */
     GTR_PLAN_FUSED_MMA = 2,         /* fused mma.sync kernel, one chunk per tile */
     GTR_PLAN_FUSED_MMA_PAIR = 3,    /* fused mma.sync kernel, two chunks per tile (d_v <= 64) */
-    GTR_PLAN_FUSED_TCGEN05 = 4      /* fused tcgen05 kernel (d_k = d_v = 64, chunk 64) */
+    GTR_PLAN_FUSED_TCGEN05 = 4,     /* fused tcgen05 kernel, chained tiles (d_k = d_v = 64, chunk 64) */
+    GTR_PLAN_WALK_TCGEN05 = 5       /* tcgen05 walk kernel, one CTA per (sequence, value slice) */
 } gtr_plan_t;
 
 /* The GLA forward over all B*heads sequences (see the operation above).
@@ -261,10 +270,10 @@ int gtr_gla_version(void);
 /* Which kernels gtr_gla_forward_ex(..., schedule, ...) launches for this
  * problem on a device with sm_count streaming multiprocessors: a gtr_plan_t,
  * or -1 for invalid arguments.  Host-only; needs no device.  AUTO takes the
- * three-phase schedule for at most 24 sequences (B*heads), the tcgen05
- * kernel for its shape when sequences are at least 2*sm_count, else the
- * mma.sync kernel with two chunks per tile below 2*sm_count sequences when
- * d_v <= 64, one chunk per tile otherwise. */
+ * three-phase schedule for at most 24 sequences (B*heads); the walk kernel
+ * for chunk 64, d_k in {32, 64, 128} and d_v in {64, 128}; else the mma.sync
+ * kernel with two chunks per tile below 2*sm_count sequences when d_v <= 64,
+ * one chunk per tile otherwise. */
 int gtr_gla_plan(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int chunk, int schedule,
                  int sm_count);
 

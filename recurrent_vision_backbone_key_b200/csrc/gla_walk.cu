@@ -1,0 +1,37 @@
+// gla_walk.cu -- instantiations and launchers of the tcgen05 walk kernel
+// (gla_walk.cuh): d_k in {32, 64, 128}, value slices of 64, chunks of 64.
+#include "gla_walk.cuh"
+
+namespace gtr {
+
+cudaError_t launch_walk(const WalkArgs &a, int mode, int grid, cudaStream_t st) {
+    const int dk = a.geo.dk;
+#define GTR_WALK_CASE(DK)                                                          \
+    if (dk == DK) {                                                                \
+        if (mode == WALK_SEQ) return launch_walk_t<DK, WALK_SEQ>(a, grid, st);     \
+        if (mode == WALK_SUMMARY) return launch_walk_t<DK, WALK_SUMMARY>(a, grid, st); \
+        return launch_walk_t<DK, WALK_OUTPUT>(a, grid, st);                        \
+    }
+    GTR_WALK_CASE(32)
+    GTR_WALK_CASE(64)
+    GTR_WALK_CASE(128)
+#undef GTR_WALK_CASE
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t walk_ctas_per_sm(int dk, int mode, int *ctas) {
+    *ctas = 0;
+#define GTR_WALK_OCC(DK)                                                           \
+    if (dk == DK) {                                                                \
+        if (mode == WALK_SEQ) return walk_occupancy<DK, WALK_SEQ>(ctas);           \
+        if (mode == WALK_SUMMARY) return walk_occupancy<DK, WALK_SUMMARY>(ctas);   \
+        return walk_occupancy<DK, WALK_OUTPUT>(ctas);                              \
+    }
+    GTR_WALK_OCC(32)
+    GTR_WALK_OCC(64)
+    GTR_WALK_OCC(128)
+#undef GTR_WALK_OCC
+    return cudaSuccess;
+}
+
+}  // namespace gtr

@@ -13,6 +13,7 @@
 
 #include "gla_common.cuh"
 #include "gla_tc.cuh"
+#include "gla_walk.cuh"
 
 namespace gtr {
 
@@ -173,7 +174,7 @@ gtr_status_t status_word(cudaStream_t st, unsigned **out) {
     return s;
 }
 
-constexpr int kSchedLast = GTR_SCHED_FUSED_TCGEN05;  // largest gtr_schedule_t value
+constexpr int kSchedLast = GTR_SCHED_WALK_TCGEN05;  // largest gtr_schedule_t value
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
 // At most this many (batch, head) sequences: GTR_SCHED_AUTO runs the
 // three-phase schedule (the fused chain is the bottleneck then).  Measured at
@@ -209,28 +210,85 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
 }
 
 bool tcgen05_shape(const Geom &g) { return g.dk == 64 && g.dv == 64 && g.chunk == 64; }
+// Shapes of the tcgen05 walk kernel (and of the tcgen05 three-phase phases).
+bool walk_shape(const Geom &g) {
+    return g.chunk == 64 && (g.dk == 32 || g.dk == 64 || g.dk == 128) && (g.dv == 64 || g.dv == 128) &&
+           (int64_t)g.B * g.heads * g.nc * (g.dv / 64) < ((int64_t)1 << 31);
+}
 
 // The kernels a schedule launches for a problem: a host-only decision, so
-// it can be asked without a device (gtr_gla_plan).  With three_phase_ok
-// false (the bounded-wait test hook) AUTO keeps to the fused kernels.
-gtr_plan_t plan_for(const Geom &geo, int schedule, int sms, bool three_phase_ok = true) {
+// it can be asked without a device (gtr_gla_plan).  With chain_only (the
+// bounded-wait test hook) AUTO keeps to the fused kernels whose tiles wait
+// on one another.
+gtr_plan_t plan_for(const Geom &geo, int schedule, int sms, bool chain_only = false) {
     const int64_t nseq = (int64_t)geo.B * geo.heads;
     if (schedule == GTR_SCHED_THREE_PHASE) return GTR_PLAN_THREE_PHASE;
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return GTR_PLAN_THREE_PHASE_SIMT;
-    // With few sequences the fused kernels wait on the chain of boundary
-    // states (one L2 hand-over per chunk step); the three-phase schedule has
-    // no such chain (its scan is a pipelined sweep) and its state traffic is
-    // small then, so AUTO takes it.
-    if (schedule == GTR_SCHED_AUTO && three_phase_ok && nseq <= kFewSequences) return GTR_PLAN_THREE_PHASE;
+    // With few sequences every per-sequence chain (the walk's chunk loop or
+    // the fused kernels' hand-over of boundary states) is long next to the
+    // work; the three-phase schedule has chunk-parallel phases and a
+    // pipelined scan, and its state traffic is small then, so AUTO takes it.
+    if (schedule == GTR_SCHED_AUTO && !chain_only && nseq <= kFewSequences) return GTR_PLAN_THREE_PHASE;
+    if (walk_shape(geo) && (schedule == GTR_SCHED_WALK_TCGEN05 || (schedule == GTR_SCHED_AUTO && !chain_only)))
+        return GTR_PLAN_WALK_TCGEN05;
     // Few sequences leave the chain of boundary states as the critical path:
     // then two chunks per tile halve its length (d_v <= 64).  Many sequences
     // keep every SM busy anyway: then one chunk per tile gives more resident
-    // CTAs.  The tcgen05 kernel does one chunk per tile: AUTO uses it when
-    // sequences are many; GTR_SCHED_FUSED_TCGEN05 forces it for its shape.
+    // CTAs.  The chained tcgen05 kernel does one chunk per tile.
     const bool pair = nseq < 2 * (int64_t)sms;
     if (tcgen05_shape(geo) && (schedule == GTR_SCHED_FUSED_TCGEN05 || (schedule == GTR_SCHED_AUTO && !pair)))
         return GTR_PLAN_FUSED_TCGEN05;
     return (pair && geo.dv <= 64) ? GTR_PLAN_FUSED_MMA_PAIR : GTR_PLAN_FUSED_MMA;
+}
+
+// Grid of a persistent walk launch over `items` work items: every resident
+// CTA slot of the device, at most one per item (cached per device and mode).
+cudaError_t walk_grid(int dk, int mode, int64_t items, int *grid) {
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> cache;  // (device, dk*8 + mode) -> slots
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = sm_count(&sms)) != cudaSuccess) return e;
+    int slots = 0;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        auto key = std::make_pair(dev, dk * 8 + mode);
+        auto it = cache.find(key);
+        if (it == cache.end()) {
+            int per_sm = 0;
+            if ((e = walk_ctas_per_sm(dk, mode, &per_sm)) != cudaSuccess) return e;
+            it = cache.emplace(key, std::max(1, per_sm) * sms).first;
+        }
+        slots = it->second;
+    }
+    *grid = (int)std::min<int64_t>(items, slots);
+    return cudaSuccess;
+}
+
+WalkArgs make_walk_args(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo,
+                        unsigned *status) {
+    WalkArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.q = q; a.k = k; a.v = v; a.g = g; a.geo = geo; a.status = status;
+    a.vs = geo.dv / 64;
+    return a;
+}
+
+// The whole forward as one walk launch: one CTA per (sequence, value slice).
+// S0 / SN: initial and final states [B*heads][d_k][d_v] fp32, or null.
+gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo,
+                      __half *out, cudaStream_t st, const float *S0 = nullptr, float *SN = nullptr) {
+    unsigned *status = nullptr;
+    gtr_status_t s = status_word(st, &status);
+    if (s != GTR_OK) return s;
+    WalkArgs a = make_walk_args(q, k, v, g, geo, status);
+    a.out = out;
+    a.S0 = S0;
+    a.SN = SN;
+    a.items = geo.B * geo.heads * a.vs;
+    cudaError_t e = launch_walk(a, WALK_SEQ, a.items, st);
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "walk kernel launch");
 }
 
 gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const float *g,
@@ -259,8 +317,20 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "fused kernel launch");
 }
 
+// Phase 1 and phase 3 on tensor cores: the tcgen05 walk kernel in its
+// single-chunk modes for its shapes, the mma.sync kernel otherwise.
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
-                       float *gamma, cudaStream_t st) {
+                       float *gamma, cudaStream_t st, unsigned *status) {
+    if (walk_shape(geo)) {
+        WalkArgs a = make_walk_args(nullptr, k, v, g, geo, status);
+        a.dS = dS;
+        a.gamma = gamma;
+        a.items = geo.B * geo.heads * geo.nc * a.vs;
+        int grid = 0;
+        cudaError_t e = walk_grid(geo.dk, WALK_SUMMARY, a.items, &grid);
+        if (e != cudaSuccess) return e;
+        return launch_walk(a, WALK_SUMMARY, grid, st);
+    }
     TcArgs a = make_args(nullptr, k, v, g, geo);
     a.dS = dS;
     a.gamma = gamma;
@@ -268,7 +338,17 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
 }
 
 cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const float *g,
-                      const float *S_enter, const Geom &geo, __half *out, cudaStream_t st) {
+                      const float *S_enter, const Geom &geo, __half *out, cudaStream_t st, unsigned *status) {
+    if (walk_shape(geo)) {
+        WalkArgs a = make_walk_args(q, k, v, g, geo, status);
+        a.S_enter = S_enter;
+        a.out = out;
+        a.items = geo.B * geo.heads * geo.nc * a.vs;
+        int grid = 0;
+        cudaError_t e = walk_grid(geo.dk, WALK_OUTPUT, a.items, &grid);
+        if (e != cudaSuccess) return e;
+        return launch_walk(a, WALK_OUTPUT, grid, st);
+    }
     TcArgs a = make_args(q, k, v, g, geo);
     a.S_enter = S_enter;
     a.out = out;
@@ -281,18 +361,20 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     void *ws = nullptr;
     gtr_status_t s = get_workspace(three_phase_ws(geo), st, &ws);
     if (s != GTR_OK) return s;
+    unsigned *status = nullptr;
+    if ((s = status_word(st, &status)) != GTR_OK) return s;
     size_t nseq = (size_t)geo.B * geo.heads;
     float *dS = static_cast<float *>(ws);
     float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                              align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
     cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
-                         : summary_tc(k, v, g, geo, dS, gamma, st);
+                         : summary_tc(k, v, g, geo, dS, gamma, st, status);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
                                            align256(nseq * geo.nc * geo.dk * sizeof(float)));
     e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
-    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st);
+    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st, status);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
     return GTR_OK;
 }
@@ -325,6 +407,7 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     const gtr_plan_t plan = plan_for(geo, schedule, sms);
     if (plan == GTR_PLAN_THREE_PHASE || plan == GTR_PLAN_THREE_PHASE_SIMT)
         return run_three_phase(hq, hk, hv, g, geo, ho, st, plan == GTR_PLAN_THREE_PHASE_SIMT);
+    if (plan == GTR_PLAN_WALK_TCGEN05) return run_walk(hq, hk, hv, g, geo, ho, st);
     return run_fused(hq, hk, hv, g, geo, ho, st, plan);
 }
 
@@ -502,8 +585,10 @@ gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g,
         if (overlap(rs, r) || overlap(rg, r)) return fail(GTR_ERR_ALIAS, "an output overlaps an input%s");
     if (overlap(rs, rg)) return fail(GTR_ERR_ALIAS, "dS overlaps gamma%s");
     if (empty) return GTR_OK;
+    unsigned *status = nullptr;
+    if ((s = status_word(static_cast<cudaStream_t>(stream), &status)) != GTR_OK) return s;
     cudaError_t e = summary_tc(static_cast<const __half *>(k), static_cast<const __half *>(v), g, geo,
-                               dS, gamma, static_cast<cudaStream_t>(stream));
+                               dS, gamma, static_cast<cudaStream_t>(stream), status);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk summary launch");
 }
 
@@ -558,9 +643,11 @@ gtr_status_t gtr_gla_chunk_output(const void *q, const void *k, const void *v, c
     for (const Range &r : in)
         if (overlap(ro, r)) return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
     if (empty) return GTR_OK;
+    unsigned *status = nullptr;
+    if ((s = status_word(static_cast<cudaStream_t>(stream), &status)) != GTR_OK) return s;
     cudaError_t e = output_tc(static_cast<const __half *>(q), static_cast<const __half *>(k),
                               static_cast<const __half *>(v), g, S_enter, geo, static_cast<__half *>(out),
-                              static_cast<cudaStream_t>(stream));
+                              static_cast<cudaStream_t>(stream), status);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "chunk output launch");
 }
 
@@ -573,7 +660,9 @@ size_t gtr_gla_workspace_bytes_ex(int B, int heads, int grid_h, int grid_w, int 
     const size_t status = 256;  // the stream's device status word
     if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT)
         return three_phase_ws(geo) + status;
-    if (schedule == GTR_SCHED_AUTO) return std::max(three_phase_ws(geo), fused_ws(geo)) + status;
+    const size_t fused = walk_shape(geo) ? 0 : fused_ws(geo);  // the walk needs no workspace
+    if (schedule == GTR_SCHED_AUTO) return std::max(three_phase_ws(geo), fused) + status;
+    if (schedule == GTR_SCHED_WALK_TCGEN05) return fused + status;
     return fused_ws(geo) + status;
 }
 
@@ -627,7 +716,7 @@ gtr_status_t gtr_gla_debug_forward_fused(const void *q, const void *k, const voi
     if (e != cudaSuccess) return cuda_fail(e, "device query");
     return run_fused(static_cast<const __half *>(q), static_cast<const __half *>(k),
                      static_cast<const __half *>(v), g, geo, static_cast<__half *>(out),
-                     static_cast<cudaStream_t>(stream), plan_for(geo, schedule, sms, false), hold_seq,
+                     static_cast<cudaStream_t>(stream), plan_for(geo, schedule, sms, true), hold_seq,
                      hold_chunk, spin_limit);
 }
 

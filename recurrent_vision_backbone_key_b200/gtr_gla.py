@@ -29,7 +29,8 @@ STATUS_NAMES = {
     7: "GTR_ERR_OOM",
 }
 DIRECTIONS = {"l2r": 0, "r2l": 1, "t2b": 2, "b2t": 3}
-SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4}
+SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4,
+             "walk_tcgen05": 5}
 
 # Every symbol include/gtr_gla.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -221,7 +222,8 @@ def gtr_gla_launch_count() -> int:
     return int(load().gtr_gla_launch_count())
 
 
-PLANS = {0: "three_phase", 1: "three_phase_simt", 2: "fused_mma", 3: "fused_mma_pair", 4: "fused_tcgen05"}
+PLANS = {0: "three_phase", 1: "three_phase_simt", 2: "fused_mma", 3: "fused_mma_pair", 4: "fused_tcgen05",
+         5: "walk_tcgen05"}
 
 
 def gtr_gla_plan(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule, sm_count) -> int:

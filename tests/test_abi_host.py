@@ -123,23 +123,26 @@ def test_workspace_bytes(lib):
 def test_dispatch_plan(lib):
     """The kernels each schedule launches (host-only decision, 148 SMs)."""
     plan = lambda B, heads, H, W, dk, dv, C, sched: lib.gtr_gla_plan(B, heads, H, W, dk, dv, C, sched, 148)
-    # batched: many sequences at d = 64, chunk 64 -> the tcgen05 kernel
-    assert plan(32, 12, 40, 40, 64, 64, 64, "auto") == 4
+    # batched: many sequences, chunk 64 -> the tcgen05 walk kernel
+    assert plan(32, 12, 40, 40, 64, 64, 64, "auto") == 5
     # latency configs and the B1 sweep: at most 24 sequences -> three phases
     assert plan(1, 6, 40, 40, 64, 64, 64, "auto") == 0
     assert plan(1, 6, 80, 80, 64, 64, 64, "auto") == 0
     assert plan(1, 8, 256, 256, 128, 128, 64, "auto") == 0
-    assert plan(2, 8, 40, 40, 64, 64, 64, "auto") == 0
     assert plan(2, 12, 40, 40, 64, 64, 64, "auto") == 0   # 24 sequences
-    assert plan(5, 5, 40, 40, 64, 64, 64, "auto") == 3    # 25: the two-chunk fused kernel
-    # B8 sweep: 64 sequences, d_v = 128 -> mma.sync, one chunk per tile
-    assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 2
-    # 64 sequences at d = 64: fewer than 2 per SM -> mma.sync with two chunks per tile
-    assert plan(8, 8, 64, 64, 64, 64, 64, "auto") == 3
+    assert plan(5, 5, 40, 40, 64, 64, 64, "auto") == 5    # 25: the walk
+    # B8 sweep (64 sequences, d = 128) and the deployment shape d_k=32, d_v=64
+    assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 5
+    assert plan(8, 8, 64, 64, 32, 64, 64, "auto") == 5
+    # shapes outside the walk kernel keep the mma.sync kernels
+    assert plan(8, 8, 64, 64, 16, 64, 64, "auto") == 3     # d_k = 16, few sequences: two chunks a tile
+    assert plan(32, 12, 40, 40, 64, 64, 32, "auto") == 2   # chunk 32, many sequences
+    assert plan(8, 8, 64, 64, 64, 32, 64, "walk_tcgen05") == 3  # d_v = 32: not a walk shape
+    # explicit schedules
     assert plan(8, 8, 64, 64, 64, 64, 64, "fused_tcgen05") == 4
     assert plan(8, 8, 64, 64, 32, 64, 64, "fused_tcgen05") == 3  # not its shape
     assert plan(32, 12, 40, 40, 64, 64, 64, "fused") == 2
-    assert plan(32, 12, 40, 40, 64, 64, 32, "auto") == 2  # chunk 32: not the tcgen05 shape
+    assert plan(1, 1, 8, 8, 64, 64, 64, "walk_tcgen05") == 5
     assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase") == 0
     assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase_simt") == 1
     # invalid arguments

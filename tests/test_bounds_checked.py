@@ -16,7 +16,8 @@ from gpu_util import compare
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4}
+SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4,
+             "walk_tcgen05": 5}
 
 
 @pytest.fixture(scope="module")
@@ -49,7 +50,8 @@ def assert_no_skips(lib):
 
 
 @pytest.mark.parametrize("schedule", list(SCHEDULES))
-@pytest.mark.parametrize("dk,dv,chunk", [(16, 16, 16), (32, 64, 32), (64, 64, 64), (128, 128, 64)])
+@pytest.mark.parametrize("dk,dv,chunk", [(16, 16, 16), (32, 64, 32), (64, 64, 64), (128, 128, 64), (32, 64, 64),
+                                         (64, 128, 64)])
 def test_checked_build_odd_shapes(clib, oracle_mod, schedule, dk, dv, chunk):
     for B, H, W, heads in ((1, 7, 9, 1), (2, 7, 9, 3)):
         q, k, v, g = make_inputs(B, H, W, heads, dk, dv, seed=dk + chunk + B)

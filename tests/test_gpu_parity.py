@@ -15,7 +15,9 @@ from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, s
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["auto", "fused", "fused_tcgen05", "three_phase", "three_phase_simt"]
+SCHEDULES = ["auto", "fused", "fused_tcgen05", "three_phase", "three_phase_simt", "walk_tcgen05"]
+# the shapes of the tcgen05 walk kernel and of the tcgen05 three-phase phases
+WALK_SHAPES = [(32, 64), (64, 64), (128, 128), (64, 128), (128, 64), (32, 128)]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -94,9 +96,11 @@ def test_gtr_s_640_all_directions(oracle_mod, direction):
         compare(out, ref)
 
 
-def test_phases_against_oracle_intermediates(oracle_mod):
-    """chunk_summary, boundary_scan and chunk_output one by one."""
-    H, W, heads, dk, dv, chunk = 10, 13, 2, 32, 64, 32
+@pytest.mark.parametrize("dk,dv,chunk", [(32, 64, 32), (64, 64, 64), (128, 128, 64), (32, 64, 64)])
+def test_phases_against_oracle_intermediates(oracle_mod, dk, dv, chunk):
+    """chunk_summary, boundary_scan and chunk_output one by one (chunk 64:
+    the tcgen05 phases; chunk 32: the mma.sync phases)."""
+    H, W, heads = 10, 13, 2
     q, k, v, g = gpu_inputs(2, H, W, heads, dk, dv, seed=77)
     direction = 3
     ref_out, ref_dS, ref_gamma, ref_Se = oracle_mod.gla_chunked(
@@ -349,3 +353,39 @@ def test_cuda_graph_twelve_call_stack(B, heads):
             assert torch.equal(o, e), rep
     assert gtr_gla.gtr_gla_get_last_device_status() == 0
     del graph
+
+
+@pytest.mark.parametrize("dk,dv", WALK_SHAPES)
+@pytest.mark.parametrize("schedule", ["walk_tcgen05", "three_phase"])
+def test_walk_shapes_all_directions(oracle_mod, dk, dv, schedule):
+    """Every shape of the tcgen05 walk kernel and of the tcgen05 phases, all
+    four directions, on a ragged grid (7 x 19 = 133 tokens: two full chunks
+    and a tail of 5) and a grid of several full chunks, B = 2, 3 heads."""
+    for (H, W) in [(7, 19), (16, 24)]:
+        q, k, v, g = gpu_inputs(2, H, W, 3, dk, dv, seed=dk * 7 + dv + H)
+        for direction in range(4):
+            out = run_forward(q, k, v, g, H, W, direction, 64, schedule)
+            compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, direction))
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (128, 128), (32, 64)])
+def test_walk_special_gates(oracle_mod, dk, dv):
+    """Open, closed, strong and mixed gates, and a few |q~| > 16 tokens,
+    through the walk kernel: the whole-chunk form and the exact score path."""
+    H, W = 10, 13
+    q, k, v, g = gpu_inputs(2, H, W, 2, dk, dv, seed=31 + dk)
+    cases = {
+        "open": torch.zeros_like(g),
+        "closed": torch.full_like(g, -1.0e4),
+        "strong": gpu_inputs(2, H, W, 2, dk, dv, seed=31 + dk, gate="strong")[3],
+        "mixed": torch.where(torch.rand_like(g) < 0.97, g, g * 60.0),
+    }
+    for name, gg in cases.items():
+        for direction in (0, 3):
+            out = run_forward(q, k, v, gg, H, W, direction, 64, "walk_tcgen05")
+            compare(out, oracle_full(oracle_mod, q, k, v, gg, H, W, direction))
+    gen = torch.Generator(device="cuda").manual_seed(6)
+    big = torch.rand(q.shape[:3], device="cuda", generator=gen) < 0.05
+    qb = torch.where(big[..., None], q.float() * 300.0, q.float()).half()
+    out = run_forward(qb, k, v, g, H, W, 1, 64, "walk_tcgen05")
+    compare(out, oracle_full(oracle_mod, qb, k, v, g, H, W, 1))
