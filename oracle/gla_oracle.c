@@ -66,6 +66,10 @@ typedef struct {
     double *dS, *gamma, *S_enter;
     /* serial form extra: state after c*chunk tokens, [B][heads][nc+1][dk][dv] */
     double *states;
+    /* serial form extras: the state before the first token (NULL: zero) and
+     * the state after the last one, each [B][heads][dk][dv] */
+    const double *S0;
+    double *SN;
     const int *slices; /* optional list of (b*heads+h) slices to compute */
     int n_slices;
     int next;          /* work counter */
@@ -82,6 +86,8 @@ static void serial_slice(const job_t *j, int b, int h) {
     const int64_t N = (int64_t)j->H * j->W;
     const double scale = 1.0 / sqrt((double)dk);
     double *S = (double *)calloc((size_t)dk * dv, sizeof(double));
+    const int64_t slice = (int64_t)b * j->heads + h;
+    if (j->S0) memcpy(S, j->S0 + slice * dk * dv, sizeof(double) * dk * dv);
     int64_t nc = j->chunk > 0 ? (N + j->chunk - 1) / j->chunk : 0;
     double *st = NULL;
     if (j->states) {
@@ -111,6 +117,7 @@ static void serial_slice(const job_t *j, int b, int h) {
             memcpy(st + ci * dk * dv, S, sizeof(double) * dk * dv);
         }
     }
+    if (j->SN) memcpy(j->SN + slice * dk * dv, S, sizeof(double) * dk * dv);
     free(S);
 }
 
@@ -279,4 +286,72 @@ int gla_oracle_chunked(const double *q, const double *k, const double *v, const 
     j.chunk = chunk; j.dS = dS; j.gamma = gamma; j.S_enter = S_enter;
     j.slices = slices; j.n_slices = n_slices;
     return run(&j, 1, nthreads);
+}
+
+/* The serial recurrence from a given initial state, returning the final
+ * state as well: the state carried across frames that the ai.info summary
+ * names as the natural extension ("Future Directions").  S0 (may be NULL for
+ * zero) and SN (may be NULL) are [B][heads][dk][dv]; everything else as
+ * gla_oracle_serial.  Returns 0 on success. */
+int gla_oracle_serial_state(const double *q, const double *k, const double *v, const double *g,
+                            int B, int heads, int H, int W, int dk, int dv, int dir,
+                            const double *S0, double *out, double *SN,
+                            const int *slices, int n_slices, int nthreads) {
+    job_t j;
+    memset(&j, 0, sizeof j);
+    j.q = q; j.k = k; j.v = v; j.g = g; j.out = out;
+    j.B = B; j.heads = heads; j.H = H; j.W = W; j.dk = dk; j.dv = dv; j.dir = dir;
+    j.S0 = S0; j.SN = SN; j.slices = slices; j.n_slices = n_slices;
+    return run(&j, 0, nthreads);
+}
+
+/* The output gate on the RMS-normalised mixer output (ai.info summary,
+ * "Methodology in Plain English": a data-dependent output gate applied to
+ * the RMS-normalised output).  For every row of d_v values (one token of
+ * one head) o, gate pre-activation r and the norm weight w:
+ *     y[e] = o[e] / sqrt(mean_e'(o[e']^2) + eps) * w[e] * r[e] * sigmoid(r[e])
+ * Root-mean-square normalisation as in Zhang and Sennrich (RMSNorm, on the
+ * mlsanity reference list of GTR); the swish gate as in gated linear
+ * attention (Yang et al., same list).  o, r, y: [rows][dv]; w: [dv]. */
+void gla_oracle_output_gate(const double *o, const double *r, const double *w, double eps,
+                            int64_t rows, int dv, double *y) {
+    for (int64_t i = 0; i < rows; ++i) {
+        const double *orow = o + i * dv, *rrow = r + i * dv;
+        double ms = 0.0;
+        for (int e = 0; e < dv; ++e) ms += orow[e] * orow[e];
+        ms /= dv;
+        const double inv = 1.0 / sqrt(ms + eps);
+        for (int e = 0; e < dv; ++e) {
+            const double sig = 1.0 / (1.0 + exp(-rrow[e]));
+            y[i * dv + e] = orow[e] * inv * w[e] * rrow[e] * sig;
+        }
+    }
+}
+
+/* Spatial SwiGLU's gating with its 3x3 depthwise convolution (ai.info
+ * summary, "Methodology in Plain English": a 3x3 depthwise convolution in the
+ * value branch of a SwiGLU block, applied on the 2-D patch grid; GTR project
+ * page, "Spatial SwiGLU").  a (gate branch) and bv (value branch) are
+ * [B][H*W][C] in row-major spatial order, wc [C][3][3], bias [C] (may be
+ * NULL); zero padding at the grid border:
+ *     y[b][p][c] = silu(a[b][p][c]) * (bias[c] + sum_{dy,dx} wc[c][dy+1][dx+1] * bv[b][p + dy*W + dx][c])
+ * with silu(x) = x * sigmoid(x).  y: [B][H*W][C]. */
+void gla_oracle_sswiglu(const double *a, const double *bv, const double *wc, const double *bias,
+                        int B, int H, int W, int C, double *y) {
+    for (int b = 0; b < B; ++b)
+        for (int r = 0; r < H; ++r)
+            for (int col = 0; col < W; ++col)
+                for (int c = 0; c < C; ++c) {
+                    double acc = bias ? bias[c] : 0.0;
+                    for (int dy = -1; dy <= 1; ++dy)
+                        for (int dx = -1; dx <= 1; ++dx) {
+                            const int rr = r + dy, cc = col + dx;
+                            if (rr < 0 || rr >= H || cc < 0 || cc >= W) continue;
+                            acc += wc[c * 9 + (dy + 1) * 3 + (dx + 1)] *
+                                   bv[(((int64_t)b * H + rr) * W + cc) * C + c];
+                        }
+                    const int64_t o = (((int64_t)b * H + r) * W + col) * C + c;
+                    const double x = a[o];
+                    y[o] = x / (1.0 + exp(-x)) * acc;
+                }
 }

@@ -73,6 +73,12 @@ def _load():
             lib.gla_oracle_serial.argtypes = [P, P, P, P, i, i, i, i, i, i, i, P, i, P, IP, i, i]
             lib.gla_oracle_chunked.restype = i
             lib.gla_oracle_chunked.argtypes = [P, P, P, P, i, i, i, i, i, i, i, i, P, P, P, P, IP, i, i]
+            lib.gla_oracle_serial_state.restype = i
+            lib.gla_oracle_serial_state.argtypes = [P, P, P, P, i, i, i, i, i, i, i, P, P, P, IP, i, i]
+            lib.gla_oracle_output_gate.restype = None
+            lib.gla_oracle_output_gate.argtypes = [P, P, P, ctypes.c_double, ctypes.c_int64, i, P]
+            lib.gla_oracle_sswiglu.restype = None
+            lib.gla_oracle_sswiglu.argtypes = [P, P, P, P, i, i, i, i, P]
             _lib = lib
     return _lib
 
@@ -169,3 +175,50 @@ def gla_chunked(q, k, v, g, grid_h, grid_w, direction, chunk, *, slices=None, nt
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out, dS, gamma, S_enter
+
+
+def gla_serial_state(q, k, v, g, grid_h, grid_w, direction, S0=None, *, slices=None, nthreads=None):
+    """Serial recurrence from the initial state ``S0`` (``[B, heads, dk, dv]``,
+    None for zero); returns ``(out, SN)`` with ``SN`` the state after the last
+    token, ``[B, heads, dk, dv]``."""
+    q, k, v, g = (_as_f64(x) for x in (q, k, v, g))
+    B, N, heads, dk, dv = _shapes(q, v, grid_h, grid_w)
+    s0 = None
+    if S0 is not None:
+        s0 = _as_f64(S0)
+        if s0.shape != (B, heads, dk, dv):
+            raise ValueError(f"S0 shape {s0.shape} != {(B, heads, dk, dv)}")
+    out = np.zeros((B, N, heads, dv), dtype=np.float64)
+    SN = np.zeros((B, heads, dk, dv), dtype=np.float64)
+    keep, sp, ns = _slices_arg(slices)
+    rc = _load().gla_oracle_serial_state(_ptr(q), _ptr(k), _ptr(v), _ptr(g), B, heads, grid_h, grid_w,
+                                         dk, dv, _dir(direction), _ptr(s0), _ptr(out), _ptr(SN), sp, ns,
+                                         nthreads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out, SN
+
+
+def output_gate(o, r, w, eps=1e-5):
+    """``o / sqrt(mean(o**2) + eps) * w * silu(r)`` over the last axis (d_v)."""
+    o, r, w = _as_f64(o), _as_f64(r), _as_f64(w)
+    if o.shape != r.shape or w.shape != (o.shape[-1],):
+        raise ValueError("shapes: o and r alike, w of length d_v")
+    dv = o.shape[-1]
+    y = np.zeros(o.shape, dtype=np.float64)
+    _load().gla_oracle_output_gate(_ptr(o), _ptr(r), _ptr(w), float(eps), int(o.size // dv), dv, _ptr(y))
+    return y
+
+
+def sswiglu(a, b, wc, bias, grid_h, grid_w):
+    """Spatial SwiGLU gating: ``silu(a) * (3x3 depthwise conv of b + bias)``
+    on the ``grid_h x grid_w`` patch grid, zero padding; ``a``, ``b``:
+    ``[B, N, C]``, ``wc``: ``[C, 3, 3]``, ``bias``: ``[C]`` or None."""
+    a, b, wc = _as_f64(a), _as_f64(b), _as_f64(wc)
+    B, N, C = a.shape
+    if N != grid_h * grid_w or b.shape != a.shape or wc.shape != (C, 3, 3):
+        raise ValueError("shapes")
+    bb = None if bias is None else _as_f64(bias)
+    y = np.zeros(a.shape, dtype=np.float64)
+    _load().gla_oracle_sswiglu(_ptr(a), _ptr(b), _ptr(wc), _ptr(bb), B, grid_h, grid_w, C, _ptr(y))
+    return y
