@@ -52,7 +52,10 @@ def measured_peaks():
 
 # Committed ncu summaries: (file, kernel sources hashed into it) per kernel.
 PROFILE_SUMMARIES = {
-    "gla_umma_kernel": ("gla_umma_fused_d64_batched.md", ("gla_umma.cuh", "gla_tc.cuh", "gla_common.cuh")),
+    "gla_walk_kernel<64,WALK_SEQ>": ("gla_walk_d64_batched.md",
+                                     ("gla_walk.cuh", "gla_tcgen05.cuh", "gla_tc.cuh", "gla_common.cuh")),
+    "gla_umma_kernel": ("gla_umma_fused_d64_batched.md",
+                        ("gla_umma.cuh", "gla_tcgen05.cuh", "gla_tc.cuh", "gla_common.cuh")),
     "gla_tc_kernel<64,64,FUSED,1>": ("gla_tc_fused_d64_batched.md", ("gla_tc.cuh", "gla_common.cuh")),
 }
 
@@ -64,7 +67,8 @@ def planned_kernel(w, schedule):
     plan = gtr_gla.gtr_gla_plan(w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, w.chunk, schedule, sms)
     names = {0: "three-phase (summary, scan, output)", 1: "three-phase on CUDA cores",
              2: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,1>", 3: f"gla_tc_kernel<{w.d_k},{w.d_v},FUSED,2>",
-             4: "gla_umma_kernel", 5: f"gla_walk_kernel<{w.d_k},WALK_SEQ>"}
+             4: "gla_umma_kernel", 5: f"gla_walk_kernel<{w.d_k},WALK_SEQ>",
+             6: "three-phase, mma.sync phases (summary, scan, output)"}
     return plan, names.get(plan, "unknown")
 
 
@@ -353,7 +357,7 @@ def main():
     per_forward_ms = ms / args.steps
     plan, dominant = planned_kernel(w, args.schedule)
     phase_ms = None
-    if plan in (0, 1):  # three phases: time them one by one as well
+    if plan in (0, 1, 6):  # three phases: time them one by one as well
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
     achieved = alg_bytes / (per_forward_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",

@@ -79,35 +79,41 @@ typedef enum {
 } gtr_status_t;
 
 typedef enum {
-    GTR_SCHED_AUTO = 0,             /* library choice (gtr_gla_plan): GTR_SCHED_THREE_PHASE for at
-                                       most 24 sequences (B*heads); else GTR_SCHED_WALK_TCGEN05
-                                       for its shapes; else the fused mma.sync kernel */
+    GTR_SCHED_AUTO = 0,             /* library choice (gtr_gla_plan), the fastest measured for the
+                                       problem's size: GTR_SCHED_THREE_PHASE_MMA for at most 24
+                                       sequences (B*heads); GTR_SCHED_WALK_TCGEN05 for its shapes
+                                       with d_k <= 64 and 2 to 3 (sequence, value slice) items per
+                                       SM; else GTR_SCHED_FUSED_TCGEN05 for its shape with at least
+                                       2 sequences per SM; else GTR_SCHED_FUSED */
     GTR_SCHED_FUSED = 1,            /* one kernel (mma.sync tensor cores): summaries, chained
                                        boundary states, outputs */
-    GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output on tensor
-                                       cores (tcgen05 for chunk 64, d_k in {32, 64, 128},
-                                       d_v in {64, 128}; mma.sync otherwise) */
+    GTR_SCHED_THREE_PHASE = 2,      /* chunk_summary -> boundary_scan -> chunk_output, the phases on
+                                       tcgen05 tensor cores for chunk 64, d_k in {32, 64, 128},
+                                       d_v in {64, 128} (mma.sync for other shapes) */
     GTR_SCHED_THREE_PHASE_SIMT = 3, /* the same three phases on CUDA cores only (comparison) */
     GTR_SCHED_FUSED_TCGEN05 = 4,    /* fused, one (sequence, chunk) tile per CTA with the boundary
                                        state chained between CTAs, whole-chunk products on
                                        tcgen05 (d_k = d_v = 64, chunk 64; other shapes run
                                        GTR_SCHED_FUSED) */
-    GTR_SCHED_WALK_TCGEN05 = 5      /* one CTA per (sequence, 64 value columns) walks the chunks
+    GTR_SCHED_WALK_TCGEN05 = 5,     /* one CTA per (sequence, 64 value columns) walks the chunks
                                        in scan order with its slice of the state on chip,
                                        whole-chunk products on tcgen05 (chunk 64, d_k in
                                        {32, 64, 128}, d_v in {64, 128}; other shapes run
                                        GTR_SCHED_FUSED) */
+    GTR_SCHED_THREE_PHASE_MMA = 6   /* the three phases with mma.sync tensor-core phases, every
+                                       shape */
 } gtr_schedule_t;
 
 /* The kernels a schedule launches (gtr_gla_plan). */
 typedef enum {
-    GTR_PLAN_THREE_PHASE = 0,       /* chunk summaries, boundary scan, chunk outputs (tensor cores:
-                                       tcgen05 for the walk kernel's shapes, else mma.sync) */
+    GTR_PLAN_THREE_PHASE = 0,       /* chunk summaries, boundary scan, chunk outputs; tcgen05 phases
+                                       for the walk kernel's shapes, else mma.sync */
     GTR_PLAN_THREE_PHASE_SIMT = 1,  /* the same three phases on CUDA cores */
     GTR_PLAN_FUSED_MMA = 2,         /* fused mma.sync kernel, one chunk per tile */
     GTR_PLAN_FUSED_MMA_PAIR = 3,    /* fused mma.sync kernel, two chunks per tile (d_v <= 64) */
     GTR_PLAN_FUSED_TCGEN05 = 4,     /* fused tcgen05 kernel, chained tiles (d_k = d_v = 64, chunk 64) */
-    GTR_PLAN_WALK_TCGEN05 = 5       /* tcgen05 walk kernel, one CTA per (sequence, value slice) */
+    GTR_PLAN_WALK_TCGEN05 = 5,      /* tcgen05 walk kernel, one CTA per (sequence, value slice) */
+    GTR_PLAN_THREE_PHASE_MMA = 6    /* the three phases with mma.sync phases */
 } gtr_plan_t;
 
 /* The GLA forward over all B*heads sequences (see the operation above).
@@ -131,6 +137,46 @@ gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const 
 gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, const float *g,
                                 int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                 int direction, int chunk, int schedule, void *out, void *stream);
+
+/* The forward from a given initial state, returning the final state: the
+ * recurrence above with S_0 = S0 instead of zero, and SN = S_N, the state
+ * after the last token of the scan.  This carries the state across calls,
+ * e.g. across video frames (ai.info summary, "Future Directions": carrying
+ * the state across frames is the natural extension; the pages' own operator
+ * fixes S_0 = 0, "Methodology in Plain English").
+ *   S0 (device, fp32) [B][heads][d_k][d_v] row-major per (b, h), or NULL for
+ *   a zero initial state; SN (device, fp32) [B][heads][d_k][d_v], or NULL
+ *   when the final state is not wanted; other arguments as gtr_gla_forward.
+ * Runs the walk kernel (GTR_SCHED_WALK_TCGEN05) and supports its shapes only:
+ * chunk 64, d_k in {32, 64, 128}, d_v in {64, 128} (else
+ * GTR_ERR_UNSUPPORTED_SHAPE).  SN may be the same buffer as S0 (updated in
+ * place); any other overlap of SN with S0, an input or out, or of out with
+ * S0, is GTR_ERR_ALIAS.  S0 and SN must be 16-byte aligned.  With no token
+ * (grid_h*grid_w == 0) SN receives S0 (or zeros).  Needs no workspace. */
+gtr_status_t gtr_gla_forward_state(const void *q, const void *k, const void *v, const float *g,
+                                   const float *S0, int B, int heads, int grid_h, int grid_w, int d_k,
+                                   int d_v, int direction, int chunk, void *out, float *SN, void *stream);
+
+/* The forward followed by the output gate on the RMS-normalised output
+ * (ai.info summary, "Methodology in Plain English": a separate data-dependent
+ * output gate applied to the RMS-normalised output), fused into the output
+ * store.  For every token t and head h, with o = o_t of that head (d_v values):
+ *     out[e] = o[e] / sqrt(mean_e'(o[e']^2) + norm_eps) * norm_weight[e]
+ *              * gate[e] * sigmoid(gate[e])
+ * (RMSNorm over the head's d_v values, Zhang and Sennrich; the swish gate of
+ * gated linear attention, Yang et al.; both on the GTR reference list).
+ *   gate (device, fp16) [B][N][heads][d_v]: the gate's pre-activation;
+ *   norm_weight (device, fp32) [d_v]; norm_eps >= 0 and finite;
+ *   out (device, fp16) [B][N][heads][d_v] receives the gated values (o
+ *   itself is not stored); other arguments as gtr_gla_forward.
+ * Runs the walk kernel with d_v = 64 (the pages' deployment shape): chunk
+ * 64, d_k in {32, 64, 128}, d_v = 64 (else GTR_ERR_UNSUPPORTED_SHAPE).  out
+ * must not overlap any input (GTR_ERR_ALIAS); gate and norm_weight must be
+ * 16-byte aligned.  Needs no workspace. */
+gtr_status_t gtr_gla_forward_gated(const void *q, const void *k, const void *v, const float *g,
+                                   const void *gate, const float *norm_weight, float norm_eps, int B,
+                                   int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                                   int chunk, void *out, void *stream);
 
 /* End-to-end call on HOST buffers: copies q, k, v, g (host) to the device,
  * runs the forward (GTR_SCHED_AUTO), copies the result into out (host) and
@@ -270,10 +316,12 @@ int gtr_gla_version(void);
 /* Which kernels gtr_gla_forward_ex(..., schedule, ...) launches for this
  * problem on a device with sm_count streaming multiprocessors: a gtr_plan_t,
  * or -1 for invalid arguments.  Host-only; needs no device.  AUTO takes the
- * three-phase schedule for at most 24 sequences (B*heads); the walk kernel
- * for chunk 64, d_k in {32, 64, 128} and d_v in {64, 128}; else the mma.sync
- * kernel with two chunks per tile below 2*sm_count sequences when d_v <= 64,
- * one chunk per tile otherwise. */
+ * three-phase schedule with mma.sync phases for at most 24 sequences
+ * (B*heads); the walk kernel for chunk 64, d_k in {32, 64}, d_v in {64, 128}
+ * when B*heads*d_v/64 lies in [2*sm_count, 3*sm_count]; the chained tcgen05
+ * kernel for d_k = d_v = 64, chunk 64 with at least 2*sm_count sequences;
+ * else the mma.sync kernel with two chunks per tile below 2*sm_count
+ * sequences when d_v <= 64, one chunk per tile otherwise. */
 int gtr_gla_plan(int B, int heads, int grid_h, int grid_w, int d_k, int d_v, int chunk, int schedule,
                  int sm_count);
 

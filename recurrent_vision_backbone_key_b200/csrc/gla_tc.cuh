@@ -75,6 +75,10 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool fu
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(smem)), "l"(gmem),
                  "r"(full ? 16 : 0));
 }
+// The same with a shared-state-space address.
+__device__ __forceinline__ void cp_async16_s(uint32_t saddr, const void *gmem, bool full) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(gmem), "r"(full ? 16 : 0));
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;\n" ::: "memory"); }
 // Wait until at most N of this thread's cp.async groups are still pending.
@@ -130,7 +134,6 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
 __device__ __forceinline__ void st_release(int *p, int v) {
     asm volatile("st.release.gpu.global.b32 [%0], %1;\n" ::"l"(p), "r"(v) : "memory");
 }
-
 // ------------------------------------------------------------ smem layout
 
 // One block of shared memory per chunk of the tile (NCH chunks per tile).

@@ -6,11 +6,14 @@ namespace gtr {
 
 cudaError_t launch_walk(const WalkArgs &a, int mode, int grid, cudaStream_t st) {
     const int dk = a.geo.dk;
-#define GTR_WALK_CASE(DK)                                                          \
-    if (dk == DK) {                                                                \
-        if (mode == WALK_SEQ) return launch_walk_t<DK, WALK_SEQ>(a, grid, st);     \
-        if (mode == WALK_SUMMARY) return launch_walk_t<DK, WALK_SUMMARY>(a, grid, st); \
-        return launch_walk_t<DK, WALK_OUTPUT>(a, grid, st);                        \
+    if (a.gate && (mode != WALK_SEQ || a.vs != 1)) return cudaErrorInvalidValue;
+#define GTR_WALK_CASE(DK)                                                                 \
+    if (dk == DK) {                                                                       \
+        if (mode == WALK_SEQ)                                                             \
+            return a.gate ? launch_walk_t<DK, WALK_SEQ, true>(a, grid, st)                \
+                          : launch_walk_t<DK, WALK_SEQ, false>(a, grid, st);              \
+        if (mode == WALK_SUMMARY) return launch_walk_t<DK, WALK_SUMMARY, false>(a, grid, st); \
+        return launch_walk_t<DK, WALK_OUTPUT, false>(a, grid, st);                        \
     }
     GTR_WALK_CASE(32)
     GTR_WALK_CASE(64)
@@ -23,9 +26,9 @@ cudaError_t walk_ctas_per_sm(int dk, int mode, int *ctas) {
     *ctas = 0;
 #define GTR_WALK_OCC(DK)                                                           \
     if (dk == DK) {                                                                \
-        if (mode == WALK_SEQ) return walk_occupancy<DK, WALK_SEQ>(ctas);           \
-        if (mode == WALK_SUMMARY) return walk_occupancy<DK, WALK_SUMMARY>(ctas);   \
-        return walk_occupancy<DK, WALK_OUTPUT>(ctas);                              \
+        if (mode == WALK_SEQ) return walk_occupancy<DK, WALK_SEQ, false>(ctas);    \
+        if (mode == WALK_SUMMARY) return walk_occupancy<DK, WALK_SUMMARY, false>(ctas); \
+        return walk_occupancy<DK, WALK_OUTPUT, false>(ctas);                       \
     }
     GTR_WALK_OCC(32)
     GTR_WALK_OCC(64)

@@ -66,6 +66,10 @@ struct WalkArgs {
     unsigned *status;      // GTR_ERR_TIMEOUT if a wait for tensor-core work gave up
     int vs;                // 64-wide value slices per sequence (d_v / 64)
     int items;             // SEQ: nseq * vs; SUMMARY, OUTPUT: nseq * nc * vs
+    // gated output (d_v = 64): out = o / sqrt(mean(o^2) + eps) * w * silu(gate)
+    const __half *gate;    // [B][N][heads][d_v] gate pre-activation
+    const float *norm_w;   // [d_v] RMS-norm weight
+    float norm_eps;
 };
 
 template <int DK>
@@ -83,7 +87,7 @@ struct WalkLayout {
     static constexpr uint32_t MISC = ROW + 2u * 64u * 8u;  // tmem base, two mbarriers
     static constexpr uint32_t BYTES = MISC + 64;
     static constexpr uint32_t ALLOC = BYTES + 1024;     // slack for aligning the base to 1024
-    static constexpr uint32_t TMEM_COLS = DK > 64 ? 128u : 64u;
+    static constexpr uint32_t TMEM_COLS = 128u;  // A | O (lanes 0-15), dS^T (lanes 16-31)
     static constexpr int MIN_CTAS = kGsmem ? 1 : 3;
 };
 
@@ -93,7 +97,10 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
     return (uint32_t)((col >> 6) * 8192) + sw128(row, col & 63);
 }
 
-template <int DK, int MODE>
+// GATED (WALK_SEQ, d_v = 64): the output store applies the output gate on
+// the RMS-normalised output (ai.info summary, "Methodology in Plain English"):
+// out = o / sqrt(mean over the head's d_v values of o^2 + eps) * w * silu(gate).
+template <int DK, int MODE, bool GATED>
 __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel(const WalkArgs args) {
     using L = WalkLayout<DK>;
     constexpr int KT = DK / 8;           // 8-wide key tiles of the state fragment
@@ -131,46 +138,61 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         }
     };
 
-    // ---- loads of one step into a stage, each warp its own 16 rows
+    // ---- loads of one step into a stage, each warp its own 16 rows: lanes
+    // 0-15 compute the rows of tokens 16w..16w+15, then lane l copies half
+    // of the 16-byte pieces of row 16w + l/2 of every tensor
     auto issue_loads = [&](int it, int c, int stage) {
         int64_t *rowt = sRow + stage * 64;
-        const uint32_t sb = (uint32_t)stage * L::STAGE;
+        const uint32_t sb = base_addr + (uint32_t)stage * L::STAGE;
         if (it < args.items) {
             const int seq = seq_of(it), sl = it % args.vs;
             const int b = seq / geo.heads, h = seq - b * geo.heads;
             const int t0 = c * 64, len = min(64, geo.N - t0);
+            int64_t r_own = -1;
             if (lane < 16) {
                 const int t = 16 * warp + lane;
-                int64_t r = t < len ? ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h
-                                    : (int64_t)-1;
-                if (r >= 0 && !GTR_INB(r, rows, BS_WALK_ROW)) r = -1;
-                rowt[t] = r;
+                if (t < len)
+                    r_own = ((int64_t)b * geo.N + scan_pos(geo.dir, t0 + t, geo.H, geo.W, geo.N)) * geo.heads + h;
+                if (r_own >= 0 && !GTR_INB(r_own, rows, BS_WALK_ROW)) r_own = -1;
+                rowt[t] = r_own;
             }
-            __syncwarp();
-            constexpr int QCH = DK / 8;  // 16-byte pieces of a q or k row
-            for (int idx = lane; idx < 16 * QCH; idx += 32) {
-                const int t = 16 * warp + idx / QCH, j = idx % QCH;
-                const int64_t r = rowt[t];
-                const bool ok = r >= 0 && GTR_INB(r * DK + j * 8 + 7, rows * DK, BS_WALK_LOAD);
-                const int64_t o = ok ? r * DK + j * 8 : 0;
-                const uint32_t so = (uint32_t)(j >> 3) * 8192u + t * 128 + ((((j & 7) ^ (t & 7)) & 7) << 4);
-                if (kOut) cp_async16(base + sb + L::SQ + so, args.q + o, ok);
-                cp_async16(base + sb + L::SK + so, args.k + o, ok);
+            // consecutive lanes copy consecutive 16-byte pieces of a row (whole
+            // 128-byte lines per 8 lanes); the row index comes from the lane
+            // that computed it
+            constexpr int QCH = DK / 8;         // pieces of a q or k row
+            constexpr int QRPI = 32 / QCH;      // rows per instruction
+            const int jq = lane % QCH, rq = lane / QCH;
+#pragma unroll
+            for (int i = 0; i < 16 / QRPI; ++i) {
+                const int tl = rq + QRPI * i, t = 16 * warp + tl;
+                const int64_t r = __shfl_sync(0xffffffffu, r_own, tl);
+                const bool ok = r >= 0 && GTR_INB(r * DK + jq * 8 + 7, rows * DK, BS_WALK_LOAD);
+                const int64_t o = ok ? r * DK + jq * 8 : 0;
+                const uint32_t so = (uint32_t)(jq >> 3) * 8192u + (uint32_t)t * 128u +
+                                    ((((uint32_t)jq & 7u) ^ (uint32_t)(t & 7)) << 4);
+                if (kOut) cp_async16_s(sb + L::SQ + so, args.q + o, ok);
+                cp_async16_s(sb + L::SK + so, args.k + o, ok);
             }
-            for (int idx = lane; idx < 16 * 8; idx += 32) {
-                const int t = 16 * warp + (idx >> 3), j = idx & 7;
-                const int64_t r = rowt[t];
-                const int64_t o = r * DV + sl * DV_CTA + j * 8;
+            const int jv = lane & 7, rv = lane >> 3;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int tl = rv + 4 * i, t = 16 * warp + tl;
+                const int64_t r = __shfl_sync(0xffffffffu, r_own, tl);
+                const int64_t o = r * DV + sl * DV_CTA + jv * 8;
                 const bool ok = r >= 0 && GTR_INB(o + 7, rows * DV, BS_WALK_LOAD);
-                cp_async16(base + sb + L::SV + t * 128 + (((j ^ (t & 7)) & 7) << 4), args.v + (ok ? o : 0), ok);
+                cp_async16_s(sb + L::SV + (uint32_t)t * 128u + ((((uint32_t)jv) ^ (uint32_t)(t & 7)) << 4),
+                             args.v + (ok ? o : 0), ok);
             }
             if constexpr (L::kGsmem) {
-                constexpr int GCH = DK / 4;
-                for (int idx = lane; idx < 16 * GCH; idx += 32) {
-                    const int t = 16 * warp + idx / GCH, j = idx % GCH;
-                    const int64_t r = rowt[t];
-                    const bool ok = r >= 0 && GTR_INB(r * DK + j * 4 + 3, rows * DK, BS_WALK_LOAD);
-                    cp_async16(base + sb + L::SG + (t * DK + j * 4) * 4, args.g + (ok ? r * DK + j * 4 : 0), ok);
+                constexpr int GCH = DK / 4;     // pieces of a g row (fp32)
+                constexpr int GRPI = 32 / GCH;  // rows per instruction (1 for d_k = 128)
+                const int jg = lane % GCH, rg = lane / GCH;
+#pragma unroll
+                for (int i = 0; i < 16 / GRPI; ++i) {
+                    const int tl = rg + GRPI * i, t = 16 * warp + tl;
+                    const int64_t r = __shfl_sync(0xffffffffu, r_own, tl);
+                    const bool ok = r >= 0 && GTR_INB(r * DK + jg * 4 + 3, rows * DK, BS_WALK_LOAD);
+                    cp_async16_s(sb + L::SG + (uint32_t)t * (DK * 4) + jg * 16, args.g + (ok ? r * DK + jg * 4 : 0), ok);
                 }
             }
         }
@@ -180,13 +202,16 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     // g of one step into registers (d_k <= 64): lane l, key pair (2l, 2l+1)
     // of each of this warp's 16 tokens; padding rows get g = 0 (a = 1)
     auto load_g = [&](int stage, float2 (&gv)[16]) {
-        const int64_t *rowt = sRow + stage * 64;
+        const int64_t *rowt = sRow + stage * 64 + 16 * warp;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int64_t r = rowt[16 * warp + t];
-            gv[t] = (lane_on && r >= 0 && GTR_INB(r * DK + 2 * lane + 1, rows * DK, BS_WALK_G))
-                        ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * DK + 2 * lane))
-                        : make_float2(0.f, 0.f);
+        for (int t = 0; t < 16; t += 2) {
+            const longlong2 rr = *reinterpret_cast<const longlong2 *>(rowt + t);
+            const int64_t r2[2] = {rr.x, rr.y};
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+                gv[t + u] = (lane_on && r2[u] >= 0 && GTR_INB(r2[u] * DK + 2 * lane + 1, rows * DK, BS_WALK_G))
+                                ? __ldcs(reinterpret_cast<const float2 *>(args.g + r2[u] * DK + 2 * lane))
+                                : make_float2(0.f, 0.f);
         }
     };
 
@@ -219,7 +244,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(mbar1, 1);
+        mbar_init(mbar1, kOut ? 2 : 1);  // pass 1 completes from threads 0 and 32
         mbar_init(mbar2, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
@@ -227,7 +252,17 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
-    constexpr uint32_t kDsLanes = 16u << 16;
+    constexpr uint32_t kDsLanes = 16u << 16;  // dS^T: lanes 16-31 of each 32-lane group
+    constexpr uint32_t kOCol = 64;            // O: columns 64-127 of lanes 0-15
+    // matrix descriptors of stage 0 (a stage's tiles sit L::STAGE bytes
+    // further; a descriptor's start-address field counts 16-byte units, so
+    // an offset inside shared memory is added as offset >> 4)
+    const uint64_t dQk = umma_desc_sw128(base_addr + L::SQ, 16, 1024);    // qh, K-major
+    const uint64_t dKk = umma_desc_sw128(base_addr + L::SK, 16, 1024);    // ke, K-major
+    const uint64_t dKm = umma_desc_sw128(base_addr + L::SK, 8192, 1024);  // ke, MN-major
+    const uint64_t dVm = umma_desc_sw128(base_addr + L::SV, 8192, 1024);  // v, MN-major
+    const uint64_t dP = umma_desc_sw128(base_addr + L::P, 16, 1024);
+    const uint64_t dSP = umma_desc_sw128(base_addr + L::SP, 16, 1024);
     uint32_t ph1 = 0, ph2 = 0;
     bool mma_ok = true;
 
@@ -261,8 +296,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             if (itn < args.items) load_g(s ^ 1, gnext);  // next step's g, consumed one step later
         }
         cp_async_wait_group<1>();  // this step's stage (the next one may still be in flight)
+        __syncwarp();              // the warp's own rows (its own copies) visible to the warp
         if constexpr (L::kGsmem) {
-            __syncwarp();  // each warp stages and reads only its own rows
             const float *sg = reinterpret_cast<const float *>(base + sb + L::SG);
 #pragma unroll
             for (int p = 0; p < PPL; ++p)
@@ -281,9 +316,39 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             }
             if (lane_on) *reinterpret_cast<float2 *>(sTot + warp * DK + 64 * p + 2 * lane) = tot;
         }
-        __syncthreads();  // (A) every warp's rows landed, sub-chunk totals visible
+        // ---- this lane's column pairs of the warp's 16 rows of q and k, read
+        // once (all loads before any store), and the |q~| test
+        uint32_t ro[PPL][16];
+        __half2 qv[PPL][16], kv[PPL][16];
+        float qm = 0.f;
+#pragma unroll
+        for (int p = 0; p < PPL; ++p) {
+            if (!lane_on) break;
+            const int dc = (2 * lane) & 63;
+            const uint32_t cb = (uint32_t)p * 8192u + (uint32_t)(dc & 7) * 2u;
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                const int row = 16 * warp + t;
+                ro[p][t] = cb + (uint32_t)row * 128u + (((uint32_t)(dc >> 3) ^ (uint32_t)(row & 7)) << 4);
+            }
+#pragma unroll
+            for (int t = 0; t < 16; ++t) kv[p][t] = *reinterpret_cast<const __half2 *>(base + sb + L::SK + ro[p][t]);
+            if (kOut) {
+                __half2 qmax = __float2half2_rn(0.f);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    qv[p][t] = *reinterpret_cast<const __half2 *>(base + sb + L::SQ + ro[p][t]);
+                    qmax = __hmax2(qmax, __habs2(qv[p][t]));
+                }
+                const float2 qf = __half22float2(qmax);
+                qm = fmaxf(qm, fmaxf(qf.x, qf.y));
+            }
+        }
+        // (A) every warp's totals visible; any |q~| > 16 in the chunk
+        const bool qbig = __syncthreads_or(kOut && qm * qscale > 16.f) != 0;
 
-        // ---- prep: ke = k Suf (always <= |k|), qh = q~ E / gamma (or qe = q~ E)
+        // ---- prep: ke = k Suf (always <= |k|), qh = q~ E / gamma (whole-chunk
+        // form) or qe = q~ E (exact form), written over the raw tiles
         float2 Eb[PPL], Sb[PPL], gam[PPL];
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
@@ -306,100 +371,101 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         for (int p = 0; p < PPL; ++p)
             in_range = in_range && gam[p].x >= lo && gam[p].y >= lo && gam[p].x <= 1.f / lo && gam[p].y <= 1.f / lo;
         const bool gam_ok = __all_sync(0xffffffffu, in_range);
-        float qm = 0.f;
+        // the whole-chunk form needs the gate range and |q~| <= 16 (qh then fits fp16)
+        const bool exact = kOut && (!gam_ok || qbig);
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
             if (!lane_on) break;
             const int d0 = 64 * p + 2 * lane;
             if (kOut) {
-                __half2 qmax = __float2half2_rn(0.f);
-                float2 E = gam_ok ? make_float2(Eb[p].x * (qscale / gam[p].x), Eb[p].y * (qscale / gam[p].y))
-                                  : make_float2(Eb[p].x * qscale, Eb[p].y * qscale);
+                float2 E = exact ? make_float2(Eb[p].x * qscale, Eb[p].y * qscale)
+                                 : make_float2(Eb[p].x * (qscale / gam[p].x), Eb[p].y * (qscale / gam[p].y));
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
-                    __half2 *ptr = reinterpret_cast<__half2 *>(base + sb + L::SQ + swz(16 * warp + t, d0));
-                    const __half2 qv = *ptr;
-                    qmax = __hmax2(qmax, __habs2(qv));
                     E.x *= av[p][t].x;
                     E.y *= av[p][t].y;
-                    *ptr = __hmul2(qv, __floats2half2_rn(E.x, E.y));
+                    *reinterpret_cast<__half2 *>(base + sb + L::SQ + ro[p][t]) = __hmul2(qv[p][t], __floats2half2_rn(E.x, E.y));
                 }
-                const float2 qf = __half22float2(qmax);
-                qm = fmaxf(qm, fmaxf(qf.x, qf.y));
             }
             float2 S = Sb[p];  // decay after token t to the chunk end
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
-                __half2 *ptr = reinterpret_cast<__half2 *>(base + sb + L::SK + swz(16 * warp + t, d0));
-                *ptr = __hmul2(*ptr, __floats2half2_rn(S.x, S.y));
+                *reinterpret_cast<__half2 *>(base + sb + L::SK + ro[p][t]) = __hmul2(kv[p][t], __floats2half2_rn(S.x, S.y));
                 S.x *= av[p][t].x;
                 S.y *= av[p][t].y;
             }
             if (warp == 0) *reinterpret_cast<float2 *>(sGam + d0) = gam[p];
         }
-        fence_async_shared();
-        tc_fence_before();
-        // the whole-chunk form needs the gate range and |q~| <= 16 (qh then fits fp16)
-        const bool exact = kOut && __syncthreads_or(!gam_ok || qm * qscale > 16.f) != 0;
-        if (!kOut) __syncthreads();  // (B) operands written, gamma visible
 
         const bool have_state = MODE == WALK_OUTPUT || (MODE == WALK_SEQ && (c > 0 || args.S0 != nullptr));
-        // ---- pass 1: A = qh ke^T (lanes 0-15), dS^T = V^T ke (lanes 16-31)
+        if (kOut && have_state) {
+            // ---- S'^T = (sc . S_enter)^T, K-major B operand of the readout
+            // (rows: this slice's value columns); sc = gamma (whole-chunk form)
+            // or 1 (exact form), gamma of key dim dk taken from the lane of this
+            // warp that computed it; pass 2 of the previous step has read it
+            const int v0 = 16 * warp + tr;
+            const uint32_t rb0 = (uint32_t)v0 * 128u + (uint32_t)kc * 2u, rb1 = rb0 + 8u * 128u;
+            const uint32_t x0 = (uint32_t)(v0 & 7), x1 = (uint32_t)((v0 + 8) & 7);
+#pragma unroll
+            for (int n = 0; n < KT; ++n) {
+                const int src = 4 * (n & 7) + (lane & 3);
+                const int p = n >> 3;
+                float gx = 1.f, gy = 1.f;
+#pragma unroll
+                for (int pp = 0; pp < PPL; ++pp) {
+                    const float ax = __shfl_sync(0xffffffffu, gam[pp].x, src);
+                    const float ay = __shfl_sync(0xffffffffu, gam[pp].y, src);
+                    if (pp == p) { gx = ax; gy = ay; }
+                }
+                if (exact) gx = gy = 1.f;
+                const uint32_t hb = (uint32_t)p * 8192u, ch = (uint32_t)(n & 7);
+                *reinterpret_cast<uint32_t *>(base + L::SP + hb + rb0 + ((ch ^ x0) << 4)) =
+                    pack_h2(gx * Se[n][0], gy * Se[n][1]);
+                *reinterpret_cast<uint32_t *>(base + L::SP + hb + rb1 + ((ch ^ x1) << 4)) =
+                    pack_h2(gx * Se[n][2], gy * Se[n][3]);
+            }
+        }
+        fence_async_shared();
+        tc_fence_before();
+        __syncthreads();  // (B) operands, S' and gamma written
+
+        // ---- pass 1: A = qh ke^T (lanes 0-15, columns 0-63) and dS^T = V^T ke
+        // (lanes 16-31) from thread 0; the readout O = qh S' (lanes 0-15,
+        // columns 64-127) from thread 32 at the same time
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t aQ = base_addr + sb + L::SQ, aK = base_addr + sb + L::SK, aV = base_addr + sb + L::SV;
+            const uint64_t so = (uint64_t)(sb >> 4);
             if (kOut && !exact) {
                 constexpr uint32_t id = umma_idesc(0, 0, 64, 64);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
-                    const uint32_t ko = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;
-                    umma_f16(tmem, umma_desc_sw128(aQ + ko, 16, 1024), umma_desc_sw128(aK + ko, 16, 1024), id, ks > 0);
+                    const uint64_t ko = so + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
+                    umma_f16(tmem, dQk + ko, dKk + ko, id, ks > 0);
                 }
             }
             constexpr uint32_t id2 = umma_idesc(1, 1, 64, DK);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tmem + kDsLanes, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
-                         umma_desc_sw128(aK + 2048 * ks, 8192, 1024), id2, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) umma_f16(tmem + kDsLanes, dVm + so + 128 * ks, dKm + so + 128 * ks, id2, ks > 0);
             umma_commit(mbar1);
         }
-
-        if (kOut) {
-            // ---- S'^T = (sc . S_enter)^T, K-major B operand of the readout
-            // (rows: this slice's value columns); sc = gamma (whole-chunk form)
-            // or 1 (exact form); pass 2 of the previous step has read it
+        if (kOut && tid == 32) {
+            if (have_state) {
+                tc_fence_after();
+                const uint64_t so = (uint64_t)(sb >> 4);
+                constexpr uint32_t id_qs = umma_idesc(0, 0, 64, 64);
 #pragma unroll
-            for (int n = 0; n < KT; ++n) {
-                const int dk = 8 * n + kc;
-                const float2 sc = exact ? make_float2(1.f, 1.f) : *reinterpret_cast<const float2 *>(sGam + dk);
-                const int v0 = 16 * warp + tr;
-                *reinterpret_cast<uint32_t *>(base + L::SP + swz(v0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
-                *reinterpret_cast<uint32_t *>(base + L::SP + swz(v0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint64_t ko = (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
+                    umma_f16(tmem + kOCol, dQk + so + ko, dSP + ko, id_qs, ks > 0);
+                }
+                umma_commit(mbar1);
+            } else {
+                mbar_arrive(mbar1);
             }
         }
 
         // ---- exact form: the score matrix on CUDA cores from the raw operands
         if (kOut && exact) {
-            if (gam_ok) {
-                // qh was written with 1 / gamma: rewrite qe = q~ E_t from the raw rows
-#pragma unroll
-                for (int p = 0; p < PPL; ++p) {
-                    if (!lane_on) break;
-                    const int d0 = 64 * p + 2 * lane;
-                    float2 E = Eb[p];
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const int64_t r = rowt[16 * warp + t];
-                        const bool ok = r >= 0 && GTR_INB(r * DK + d0 + 1, rows * DK, BS_WALK_EXACT);
-                        const __half2 qv = ok ? *reinterpret_cast<const __half2 *>(args.q + r * DK + d0)
-                                              : __float2half2_rn(0.f);
-                        E.x *= av[p][t].x;
-                        E.y *= av[p][t].y;
-                        *reinterpret_cast<__half2 *>(base + sb + L::SQ + swz(16 * warp + t, d0)) =
-                            __hmul2(qv, __floats2half2_rn(E.x * qscale, E.y * qscale));
-                    }
-                }
-            }
             // thread -> query row t = tid / 2, keys s in [32*(tid&1), +32); the
             // log2-domain in-chunk prefix of g, 16 key dims at a time, staged
             // in the score region
@@ -520,24 +586,29 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             tc_fence_before();
             __syncthreads();  // (C) P and S' written; A and dS^T read by every warp
 
-            // ---- pass 2: O = P V + qh S'
+            // ---- pass 2: O += P V (O holds qh S' from pass 1 when there is state)
             if (tid == 0) {
                 tc_fence_after();
-                const uint32_t aP = base_addr + L::P, aSP = base_addr + L::SP;
-                const uint32_t aQ = base_addr + sb + L::SQ, aV = base_addr + sb + L::SV;
-                constexpr uint32_t id_pv = umma_idesc(0, 1, 64, 64), id_qs = umma_idesc(0, 0, 64, 64);
+                const uint64_t so = (uint64_t)(sb >> 4);
+                constexpr uint32_t id_pv = umma_idesc(0, 1, 64, 64);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem, umma_desc_sw128(aP + 32 * ks, 16, 1024), umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
-                             id_pv, ks > 0);
-                if (have_state) {
-#pragma unroll
-                    for (int ks = 0; ks < DK / 16; ++ks) {
-                        const uint32_t ko = (uint32_t)(ks >> 2) * 8192u + (uint32_t)(ks & 3) * 32u;
-                        umma_f16(tmem, umma_desc_sw128(aQ + ko, 16, 1024), umma_desc_sw128(aSP + ko, 16, 1024), id_qs, 1);
-                    }
-                }
+                    umma_f16(tmem + kOCol, dP + 2 * ks, dVm + so + 128 * ks, id_pv, (ks > 0 || have_state) ? 1u : 0u);
                 umma_commit(mbar2);
+            }
+            // gate rows of this warp's tokens (16-byte pieces, the store
+            // pattern below), in flight while pass 2 runs
+            int4 gr[4];
+            if constexpr (GATED) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
+                    const int64_t r = rowt[t];
+                    const int64_t o_off = r * DV + j * 8;
+                    gr[i] = (t < len && r >= 0 && GTR_INB(o_off + 7, rows * DV, BS_WALK_GATE))
+                                ? __ldcs(reinterpret_cast<const int4 *>(args.gate + o_off))
+                                : make_int4(0, 0, 0, 0);
+                }
             }
             if (!mbar_wait(mbar2, ph2)) mma_ok = false;
             ph2 ^= 1u;
@@ -547,9 +618,43 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             // score region) and writes them as 16-byte row pieces
             {
                 float o[32];
-                tmem_ld_16x64(tmem + ((uint32_t)(32 * warp) << 16), o);
+                tmem_ld_16x64(tmem + kOCol + ((uint32_t)(32 * warp) << 16), o);
                 tc_wait_ld();
                 unsigned char *st = base + L::P;
+                if constexpr (GATED) {
+                    // the gate rows into the S' tile (pass 2 has read it), swizzled
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
+                        *reinterpret_cast<int4 *>(base + L::SP + t * 128 + (((j ^ (t & 7)) & 7) << 4)) = gr[i];
+                    }
+                    __syncwarp();
+                    // 1 / rms of rows tr and tr + 8 (fp32, over the 64 values
+                    // that lanes 4tr..4tr+3 hold)
+                    float ss0 = 0.f, ss1 = 0.f;
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        ss0 = fmaf(o[4 * n], o[4 * n], fmaf(o[4 * n + 1], o[4 * n + 1], ss0));
+                        ss1 = fmaf(o[4 * n + 2], o[4 * n + 2], fmaf(o[4 * n + 3], o[4 * n + 3], ss1));
+                    }
+                    ss0 += __shfl_xor_sync(0xffffffffu, ss0, 1);
+                    ss1 += __shfl_xor_sync(0xffffffffu, ss1, 1);
+                    ss0 += __shfl_xor_sync(0xffffffffu, ss0, 2);
+                    ss1 += __shfl_xor_sync(0xffffffffu, ss1, 2);
+                    const float inv0 = rsqrtf(ss0 * (1.f / 64.f) + args.norm_eps);
+                    const float inv1 = rsqrtf(ss1 * (1.f / 64.f) + args.norm_eps);
+#pragma unroll
+                    for (int n = 0; n < 8; ++n) {
+                        const int t = 16 * warp + tr, col = 8 * n + kc;
+                        const float2 w = __ldg(reinterpret_cast<const float2 *>(args.norm_w + col));
+                        const float2 r0 = __half22float2(*reinterpret_cast<const __half2 *>(base + L::SP + sw128(t, col)));
+                        const float2 r1 = __half22float2(*reinterpret_cast<const __half2 *>(base + L::SP + sw128(t + 8, col)));
+                        o[4 * n + 0] *= inv0 * w.x * (r0.x / (1.f + __expf(-r0.x)));
+                        o[4 * n + 1] *= inv0 * w.y * (r0.y / (1.f + __expf(-r0.y)));
+                        o[4 * n + 2] *= inv1 * w.x * (r1.x / (1.f + __expf(-r1.x)));
+                        o[4 * n + 3] *= inv1 * w.y * (r1.y / (1.f + __expf(-r1.y)));
+                    }
+                }
 #pragma unroll
                 for (int n = 0; n < 8; ++n) {
                     const int t = 16 * warp + tr, col = 8 * n + kc;
@@ -599,31 +704,32 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 }
 
 // Resident CTAs per SM of one instantiation (cached per device by the caller).
-template <int DK, int MODE>
+template <int DK, int MODE, bool GATED>
 cudaError_t walk_occupancy(int *ctas) {
     using L = WalkLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::ALLOC);
+    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, gla_walk_kernel<DK, MODE>, 128, L::ALLOC);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, gla_walk_kernel<DK, MODE, GATED>, 128, L::ALLOC);
 }
 
-template <int DK, int MODE>
+template <int DK, int MODE, bool GATED>
 cudaError_t launch_walk_t(const WalkArgs &a, int grid, cudaStream_t st) {
     using L = WalkLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)L::ALLOC);
+    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    gla_walk_kernel<DK, MODE><<<grid, 128, L::ALLOC, st>>>(a);
+    gla_walk_kernel<DK, MODE, GATED><<<grid, 128, L::ALLOC, st>>>(a);
     count_launch();
     return cudaGetLastError();
 }
 
-// Launchers (gla_walk.cu): grid CTAs; `grid` <= a.items.
+// Launchers (gla_walk.cu): grid CTAs; `grid` <= a.items.  a.gate != null
+// selects the gated output (WALK_SEQ with d_v = 64 only).
 cudaError_t launch_walk(const WalkArgs &a, int mode, int grid, cudaStream_t st);
 // Resident CTAs per SM for (d_k, mode), or 0 for an unsupported d_k.
 cudaError_t walk_ctas_per_sm(int dk, int mode, int *ctas);

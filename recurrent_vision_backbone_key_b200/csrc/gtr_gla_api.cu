@@ -45,6 +45,8 @@ gtr_status_t fail(gtr_status_t s, const char *fmt, const char *detail = "") {
     return s;
 }
 
+void t_err_clear() { t_err[0] = '\0'; }
+
 gtr_status_t cuda_fail(cudaError_t e, const char *what) {
     std::snprintf(t_err, sizeof t_err, "%s: %s", what, cudaGetErrorString(e));
     return GTR_ERR_CUDA;
@@ -93,7 +95,9 @@ size_t tok_bytes(const Geom &g, int d, size_t elem) {
 // Internal workspaces: one grow-only, zero-initialised device buffer per
 // (device, stream, kind).  Kinds keep the schedules apart: the fused
 // kernel's control words must never be overwritten by another schedule.
-enum WsKind { WS_THREE_PHASE = 0, WS_FUSED = 1, WS_STAGING = 2, WS_STATUS = 3, WS_SCAN = 4 };
+enum WsKind {
+    WS_THREE_PHASE = 0, WS_FUSED = 1, WS_STAGING = 2, WS_STATUS = 3, WS_SCAN = 4
+};
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
@@ -164,7 +168,6 @@ size_t fused_ctrl_bytes(const Geom &g) { return align256(((size_t)g.B * g.heads 
 size_t fused_ws(const Geom &g) {
     return fused_ctrl_bytes(g) + (size_t)g.B * g.heads * 2 * g.dk * g.dv * sizeof(float);
 }
-
 // Device status word of (current device, stream), zeroed at creation: the
 // kernels a call enqueues on `st` record a bounded wait that gave up here.
 gtr_status_t status_word(cudaStream_t st, unsigned **out) {
@@ -174,7 +177,7 @@ gtr_status_t status_word(cudaStream_t st, unsigned **out) {
     return s;
 }
 
-constexpr int kSchedLast = GTR_SCHED_WALK_TCGEN05;  // largest gtr_schedule_t value
+constexpr int kSchedLast = GTR_SCHED_THREE_PHASE_MMA;  // largest gtr_schedule_t value
 constexpr long long kSpinLimit = 1LL << 22;  // bounded wait: about a second of polling
 // At most this many (batch, head) sequences: GTR_SCHED_AUTO runs the
 // three-phase schedule (the fused chain is the bottleneck then).  Measured at
@@ -223,13 +226,24 @@ bool walk_shape(const Geom &g) {
 gtr_plan_t plan_for(const Geom &geo, int schedule, int sms, bool chain_only = false) {
     const int64_t nseq = (int64_t)geo.B * geo.heads;
     if (schedule == GTR_SCHED_THREE_PHASE) return GTR_PLAN_THREE_PHASE;
+    if (schedule == GTR_SCHED_THREE_PHASE_MMA) return GTR_PLAN_THREE_PHASE_MMA;
     if (schedule == GTR_SCHED_THREE_PHASE_SIMT) return GTR_PLAN_THREE_PHASE_SIMT;
-    // With few sequences every per-sequence chain (the walk's chunk loop or
-    // the fused kernels' hand-over of boundary states) is long next to the
+    if (schedule == GTR_SCHED_WALK_TCGEN05 && walk_shape(geo)) return GTR_PLAN_WALK_TCGEN05;
+    // With few sequences every per-sequence chain (the fused kernels' hand-
+    // over of boundary states, or the walk's chunk loop) is long next to the
     // work; the three-phase schedule has chunk-parallel phases and a
-    // pipelined scan, and its state traffic is small then, so AUTO takes it.
-    if (schedule == GTR_SCHED_AUTO && !chain_only && nseq <= kFewSequences) return GTR_PLAN_THREE_PHASE;
-    if (walk_shape(geo) && (schedule == GTR_SCHED_WALK_TCGEN05 || (schedule == GTR_SCHED_AUTO && !chain_only)))
+    // pipelined scan, and its state traffic is small then, so AUTO takes it
+    // (with the mma.sync phases: measured faster there than the tcgen05 ones,
+    // whose one-chunk CTAs wait on their own tensor-core passes).
+    if (schedule == GTR_SCHED_AUTO && !chain_only && nseq <= kFewSequences) return GTR_PLAN_THREE_PHASE_MMA;
+    // The walk keeps each (sequence, value slice) on one CTA with no chain
+    // between CTAs; it is the fastest measured when those items fill between
+    // two and three CTAs per SM (one wave at its occupancy of 3 per SM for
+    // d_k <= 64): the batched workload.  Fewer items leave SMs idle, more
+    // need a second wave.
+    const int64_t items = nseq * (geo.dv / 64);
+    if (schedule == GTR_SCHED_AUTO && !chain_only && walk_shape(geo) && geo.dk <= 64 && items >= 2 * (int64_t)sms &&
+        items <= 3 * (int64_t)sms)
         return GTR_PLAN_WALK_TCGEN05;
     // Few sequences leave the chain of boundary states as the critical path:
     // then two chunks per tile halve its length (d_v <= 64).  Many sequences
@@ -278,7 +292,8 @@ WalkArgs make_walk_args(const __half *q, const __half *k, const __half *v, const
 // The whole forward as one walk launch: one CTA per (sequence, value slice).
 // S0 / SN: initial and final states [B*heads][d_k][d_v] fp32, or null.
 gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo,
-                      __half *out, cudaStream_t st, const float *S0 = nullptr, float *SN = nullptr) {
+                      __half *out, cudaStream_t st, const float *S0 = nullptr, float *SN = nullptr,
+                      const __half *gate = nullptr, const float *norm_w = nullptr, float norm_eps = 0.f) {
     unsigned *status = nullptr;
     gtr_status_t s = status_word(st, &status);
     if (s != GTR_OK) return s;
@@ -286,6 +301,9 @@ gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const f
     a.out = out;
     a.S0 = S0;
     a.SN = SN;
+    a.gate = gate;
+    a.norm_w = norm_w;
+    a.norm_eps = norm_eps;
     a.items = geo.B * geo.heads * a.vs;
     cudaError_t e = launch_walk(a, WALK_SEQ, a.items, st);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "walk kernel launch");
@@ -307,7 +325,9 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
     a.spin_limit = spin_limit;
     a.hold_seq = hold_seq;
     a.hold_chunk = hold_chunk;
-    // Ticket and flags start from zero for every launch.
+    // Ticket and flags start from zero for every launch (a memset of the
+    // current problem's control words, recorded into a graph with the
+    // launch when captured).
     cudaError_t e = cudaMemsetAsync(a.ctrl, 0, fused_ctrl_bytes(geo), st);
     if (e != cudaSuccess) return cuda_fail(e, "control-word reset");
     if (plan == GTR_PLAN_FUSED_TCGEN05)
@@ -320,8 +340,8 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
 // Phase 1 and phase 3 on tensor cores: the tcgen05 walk kernel in its
 // single-chunk modes for its shapes, the mma.sync kernel otherwise.
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
-                       float *gamma, cudaStream_t st, unsigned *status) {
-    if (walk_shape(geo)) {
+                       float *gamma, cudaStream_t st, unsigned *status, bool tcgen05 = true) {
+    if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(nullptr, k, v, g, geo, status);
         a.dS = dS;
         a.gamma = gamma;
@@ -338,8 +358,9 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
 }
 
 cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const float *g,
-                      const float *S_enter, const Geom &geo, __half *out, cudaStream_t st, unsigned *status) {
-    if (walk_shape(geo)) {
+                      const float *S_enter, const Geom &geo, __half *out, cudaStream_t st, unsigned *status,
+                      bool tcgen05 = true) {
+    if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(q, k, v, g, geo, status);
         a.S_enter = S_enter;
         a.out = out;
@@ -357,7 +378,8 @@ cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const f
 
 // Three-phase schedule; `simt` selects the CUDA-core summary/output kernels.
 gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, const float *g,
-                             const Geom &geo, __half *out, cudaStream_t st, bool simt) {
+                             const Geom &geo, __half *out, cudaStream_t st, gtr_plan_t plan) {
+    const bool simt = plan == GTR_PLAN_THREE_PHASE_SIMT, mma = plan == GTR_PLAN_THREE_PHASE_MMA;
     void *ws = nullptr;
     gtr_status_t s = get_workspace(three_phase_ws(geo), st, &ws);
     if (s != GTR_OK) return s;
@@ -368,13 +390,13 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                              align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
     cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
-                         : summary_tc(k, v, g, geo, dS, gamma, st, status);
+                         : summary_tc(k, v, g, geo, dS, gamma, st, status, !mma);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
                                            align256(nseq * geo.nc * geo.dk * sizeof(float)));
     e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
-    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st, status);
+    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st, status, !mma);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
     return GTR_OK;
 }
@@ -405,10 +427,29 @@ gtr_status_t forward_impl(const void *q, const void *k, const void *v, const flo
     cudaError_t e = sm_count(&sms);
     if (e != cudaSuccess) return cuda_fail(e, "device query");
     const gtr_plan_t plan = plan_for(geo, schedule, sms);
-    if (plan == GTR_PLAN_THREE_PHASE || plan == GTR_PLAN_THREE_PHASE_SIMT)
-        return run_three_phase(hq, hk, hv, g, geo, ho, st, plan == GTR_PLAN_THREE_PHASE_SIMT);
+    if (plan == GTR_PLAN_THREE_PHASE || plan == GTR_PLAN_THREE_PHASE_SIMT || plan == GTR_PLAN_THREE_PHASE_MMA)
+        return run_three_phase(hq, hk, hv, g, geo, ho, st, plan);
     if (plan == GTR_PLAN_WALK_TCGEN05) return run_walk(hq, hk, hv, g, geo, ho, st);
     return run_fused(hq, hk, hv, g, geo, ho, st, plan);
+}
+
+// Checks shared by the walk-only entry points (state in/out, gated output):
+// the forward's checks plus the walk kernel's shapes.
+gtr_status_t check_walk_call(const void *q, const void *k, const void *v, const float *g, int B, int heads,
+                             int grid_h, int grid_w, int d_k, int d_v, int direction, int chunk, const void *out,
+                             Geom &geo, bool &empty) {
+    gtr_status_t s = check_shape(B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, geo, empty);
+    if (s != GTR_OK) return s;
+    if (!walk_shape(geo))
+        return fail(GTR_ERR_UNSUPPORTED_SHAPE, "this call needs chunk 64, d_k in {32, 64, 128}, d_v in {64, 128}%s");
+    if (!q || !k || !v || !g || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(out))
+        return fail(GTR_ERR_MISALIGNED, "device pointers must be 16-byte aligned%s");
+    Range ro = span(out, tok_bytes(geo, d_v, 2));
+    if (overlap(ro, span(q, tok_bytes(geo, d_k, 2))) || overlap(ro, span(k, tok_bytes(geo, d_k, 2))) ||
+        overlap(ro, span(v, tok_bytes(geo, d_v, 2))) || overlap(ro, span(g, tok_bytes(geo, d_k, 4))))
+        return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
+    return GTR_OK;
 }
 
 }  // namespace
@@ -439,6 +480,64 @@ gtr_status_t gtr_gla_forward_ex(const void *q, const void *k, const void *v, con
                                 int direction, int chunk, int schedule, void *out, void *stream) {
     return forward_impl(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk,
                         schedule, out, stream);
+}
+
+gtr_status_t gtr_gla_forward_state(const void *q, const void *k, const void *v, const float *g,
+                                              const float *S0, int B, int heads, int grid_h, int grid_w,
+                                              int d_k, int d_v, int direction, int chunk, void *out, float *SN,
+                                              void *stream) {
+    t_err_clear();
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_walk_call(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                                     geo, empty);
+    if (s != GTR_OK) return s;
+    if ((S0 && !aligned16(S0)) || (SN && !aligned16(SN)))
+        return fail(GTR_ERR_MISALIGNED, "S0 and SN must be 16-byte aligned%s");
+    const size_t sb = (size_t)B * heads * d_k * d_v * 4;
+    if (SN) {
+        const Range rn = span(SN, sb);
+        if (overlap(rn, span(q, tok_bytes(geo, d_k, 2))) || overlap(rn, span(k, tok_bytes(geo, d_k, 2))) ||
+            overlap(rn, span(v, tok_bytes(geo, d_v, 2))) || overlap(rn, span(g, tok_bytes(geo, d_k, 4))) ||
+            overlap(rn, span(out, tok_bytes(geo, d_v, 2))))
+            return fail(GTR_ERR_ALIAS, "SN overlaps an input or out%s");
+        if (S0 && S0 != SN && overlap(rn, span(S0, sb))) return fail(GTR_ERR_ALIAS, "SN partially overlaps S0%s");
+    }
+    if (S0 && overlap(span(out, tok_bytes(geo, d_v, 2)), span(S0, sb))) return fail(GTR_ERR_ALIAS, "out overlaps S0%s");
+    if (empty) {
+        // no token: the final state is the initial one (or zero)
+        if (!SN || B == 0 || heads == 0) return GTR_OK;
+        cudaError_t e = S0 ? (S0 == SN ? cudaSuccess
+                                       : cudaMemcpyAsync(SN, S0, sb, cudaMemcpyDeviceToDevice, (cudaStream_t)stream))
+                           : cudaMemsetAsync(SN, 0, sb, (cudaStream_t)stream);
+        return e == cudaSuccess ? GTR_OK : cuda_fail(e, "empty-problem state copy");
+    }
+    return run_walk(static_cast<const __half *>(q), static_cast<const __half *>(k), static_cast<const __half *>(v),
+                    g, geo, static_cast<__half *>(out), static_cast<cudaStream_t>(stream), S0, SN);
+}
+
+gtr_status_t gtr_gla_forward_gated(const void *q, const void *k, const void *v, const float *g,
+                                              const void *gate, const float *norm_weight, float norm_eps, int B,
+                                              int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                                              int chunk, void *out, void *stream) {
+    t_err_clear();
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_walk_call(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                                     geo, empty);
+    if (s != GTR_OK) return s;
+    if (d_v != 64) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "the gated output needs d_v = 64%s");
+    if (!gate || !norm_weight) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(gate) || !aligned16(norm_weight))
+        return fail(GTR_ERR_MISALIGNED, "gate and norm_weight must be 16-byte aligned%s");
+    if (!(norm_eps >= 0.f) || norm_eps > 1e30f) return fail(GTR_ERR_INVALID_ARG, "norm_eps must be finite and >= 0%s");
+    const Range ro = span(out, tok_bytes(geo, d_v, 2));
+    if (overlap(ro, span(gate, tok_bytes(geo, d_v, 2))) || overlap(ro, span(norm_weight, (size_t)d_v * 4)))
+        return fail(GTR_ERR_ALIAS, "out overlaps the gate or the norm weight%s");
+    if (empty) return GTR_OK;
+    return run_walk(static_cast<const __half *>(q), static_cast<const __half *>(k), static_cast<const __half *>(v),
+                    g, geo, static_cast<__half *>(out), static_cast<cudaStream_t>(stream), nullptr, nullptr,
+                    static_cast<const __half *>(gate), norm_weight, norm_eps);
 }
 
 // Copy/compute pipeline of the host-buffer entry point.  Every batch item is
@@ -658,11 +757,11 @@ size_t gtr_gla_workspace_bytes_ex(int B, int heads, int grid_h, int grid_w, int 
     if (check_shape(B, heads, grid_h, grid_w, d_k, d_v, 0, chunk, geo, empty) != GTR_OK) return 0;
     if (schedule < GTR_SCHED_AUTO || schedule > kSchedLast || empty) return 0;
     const size_t status = 256;  // the stream's device status word
-    if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT)
+    if (schedule == GTR_SCHED_THREE_PHASE || schedule == GTR_SCHED_THREE_PHASE_SIMT ||
+        schedule == GTR_SCHED_THREE_PHASE_MMA)
         return three_phase_ws(geo) + status;
-    const size_t fused = walk_shape(geo) ? 0 : fused_ws(geo);  // the walk needs no workspace
-    if (schedule == GTR_SCHED_AUTO) return std::max(three_phase_ws(geo), fused) + status;
-    if (schedule == GTR_SCHED_WALK_TCGEN05) return fused + status;
+    if (schedule == GTR_SCHED_AUTO) return std::max(three_phase_ws(geo), fused_ws(geo)) + status;
+    if (schedule == GTR_SCHED_WALK_TCGEN05) return (walk_shape(geo) ? 0 : fused_ws(geo)) + status;
     return fused_ws(geo) + status;
 }
 

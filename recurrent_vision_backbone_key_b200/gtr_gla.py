@@ -30,7 +30,7 @@ STATUS_NAMES = {
 }
 DIRECTIONS = {"l2r": 0, "r2l": 1, "t2b": 2, "b2t": 3}
 SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4,
-             "walk_tcgen05": 5}
+             "walk_tcgen05": 5, "three_phase_mma": 6}
 
 # Every symbol include/gtr_gla.h declares, with (restype, argtypes).
 _P = ctypes.c_void_p
@@ -40,6 +40,9 @@ SIGNATURES = {
     "gtr_gla_forward_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_forward_state": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "gtr_gla_forward_gated": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _I, _I, _I, _I, _I, _I, _I, _I,
+                                   _P, _P]),
     "gtr_gla_chunk_summary": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gtr_gla_boundary_scan": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -169,6 +172,20 @@ def gtr_gla_forward_noalloc(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, dire
                                           _stream(stream))
 
 
+def gtr_gla_forward_state(q, k, v, g, S0, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                          SN, stream=None) -> int:
+    return load().gtr_gla_forward_state(_addr(q), _addr(k), _addr(v), _addr(g), _addr(S0), B, heads,
+                                        grid_h, grid_w, d_k, d_v, _dir(direction), chunk, _addr(out),
+                                        _addr(SN), _stream(stream))
+
+
+def gtr_gla_forward_gated(q, k, v, g, gate, norm_weight, norm_eps, B, heads, grid_h, grid_w, d_k, d_v,
+                          direction, chunk, out, stream=None) -> int:
+    return load().gtr_gla_forward_gated(_addr(q), _addr(k), _addr(v), _addr(g), _addr(gate),
+                                        _addr(norm_weight), float(norm_eps), B, heads, grid_h, grid_w,
+                                        d_k, d_v, _dir(direction), chunk, _addr(out), _stream(stream))
+
+
 def gtr_gla_chunk_summary(k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, dS, gamma,
                           stream=None) -> int:
     return load().gtr_gla_chunk_summary(_addr(k), _addr(v), _addr(g), B, heads, grid_h, grid_w,
@@ -223,7 +240,7 @@ def gtr_gla_launch_count() -> int:
 
 
 PLANS = {0: "three_phase", 1: "three_phase_simt", 2: "fused_mma", 3: "fused_mma_pair", 4: "fused_tcgen05",
-         5: "walk_tcgen05"}
+         5: "walk_tcgen05", 6: "three_phase_mma"}
 
 
 def gtr_gla_plan(B, heads, grid_h, grid_w, d_k, d_v, chunk, schedule, sm_count) -> int:

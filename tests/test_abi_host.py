@@ -123,27 +123,32 @@ def test_workspace_bytes(lib):
 def test_dispatch_plan(lib):
     """The kernels each schedule launches (host-only decision, 148 SMs)."""
     plan = lambda B, heads, H, W, dk, dv, C, sched: lib.gtr_gla_plan(B, heads, H, W, dk, dv, C, sched, 148)
-    # batched: many sequences, chunk 64 -> the tcgen05 walk kernel
+    # batched: 384 sequences at d = 64 (2.6 per SM) -> the tcgen05 walk kernel
     assert plan(32, 12, 40, 40, 64, 64, 64, "auto") == 5
-    # latency configs and the B1 sweep: at most 24 sequences -> three phases
-    assert plan(1, 6, 40, 40, 64, 64, 64, "auto") == 0
-    assert plan(1, 6, 80, 80, 64, 64, 64, "auto") == 0
-    assert plan(1, 8, 256, 256, 128, 128, 64, "auto") == 0
-    assert plan(2, 12, 40, 40, 64, 64, 64, "auto") == 0   # 24 sequences
-    assert plan(5, 5, 40, 40, 64, 64, 64, "auto") == 5    # 25: the walk
-    # B8 sweep (64 sequences, d = 128) and the deployment shape d_k=32, d_v=64
-    assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 5
-    assert plan(8, 8, 64, 64, 32, 64, 64, "auto") == 5
-    # shapes outside the walk kernel keep the mma.sync kernels
-    assert plan(8, 8, 64, 64, 16, 64, 64, "auto") == 3     # d_k = 16, few sequences: two chunks a tile
-    assert plan(32, 12, 40, 40, 64, 64, 32, "auto") == 2   # chunk 32, many sequences
-    assert plan(8, 8, 64, 64, 64, 32, 64, "walk_tcgen05") == 3  # d_v = 32: not a walk shape
+    assert plan(25, 12, 8, 8, 64, 64, 64, "auto") == 5     # 300 items
+    assert plan(64, 12, 40, 40, 64, 64, 64, "auto") == 4   # 768: more than one wave -> chained
+    assert plan(32, 12, 40, 40, 32, 64, 64, "auto") == 5   # the deployment shape, batched
+    assert plan(16, 12, 40, 40, 64, 128, 64, "auto") == 5  # 192 sequences x 2 value slices
+    # latency configs and the B1 sweep: at most 24 sequences -> three phases (mma.sync phases)
+    assert plan(1, 6, 40, 40, 64, 64, 64, "auto") == 6
+    assert plan(1, 6, 80, 80, 64, 64, 64, "auto") == 6
+    assert plan(1, 8, 256, 256, 128, 128, 64, "auto") == 6
+    assert plan(2, 12, 40, 40, 64, 64, 64, "auto") == 6   # 24 sequences
+    assert plan(5, 5, 40, 40, 64, 64, 64, "auto") == 3    # 25: the two-chunk mma.sync kernel
+    # B8 sweep: 64 sequences, d_v = 128 -> mma.sync, one chunk per tile
+    assert plan(8, 8, 256, 256, 128, 128, 64, "auto") == 2
+    # 64 sequences at d = 64: fewer than 2 per SM -> mma.sync with two chunks per tile
+    assert plan(8, 8, 64, 64, 64, 64, 64, "auto") == 3
+    assert plan(32, 12, 40, 40, 64, 64, 32, "auto") == 2   # chunk 32: not the tcgen05 shape
     # explicit schedules
     assert plan(8, 8, 64, 64, 64, 64, 64, "fused_tcgen05") == 4
     assert plan(8, 8, 64, 64, 32, 64, 64, "fused_tcgen05") == 3  # not its shape
     assert plan(32, 12, 40, 40, 64, 64, 64, "fused") == 2
-    assert plan(1, 1, 8, 8, 64, 64, 64, "walk_tcgen05") == 5
+    assert plan(8, 8, 256, 256, 128, 128, 64, "walk_tcgen05") == 5
+    assert plan(8, 8, 64, 64, 32, 64, 64, "walk_tcgen05") == 5
+    assert plan(8, 8, 64, 64, 64, 32, 64, "walk_tcgen05") == 3  # d_v = 32: not a walk shape
     assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase") == 0
+    assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase_mma") == 6
     assert plan(1, 1, 8, 8, 16, 16, 16, "three_phase_simt") == 1
     # invalid arguments
     assert lib.gtr_gla_plan(1, 1, 8, 8, 16, 16, 16, 9, 148) == -1
@@ -191,3 +196,38 @@ def test_host_entry_alias_check(lib):
     g = torch.zeros((1, 16, 2, 16), dtype=torch.float32)
     st = lib.gtr_gla_forward_host(q, q, q, g, 1, 2, 4, 4, 16, 16, 0, 16, q, 0)
     assert st == 4 and "overlaps" in lib.last_error()
+
+
+def test_state_and_gated_entry_points_validate(lib):
+    """Argument checks of the state-carrying and the gated forward, before
+    any device work (fake, aligned addresses)."""
+    base = dict(q=A, k=2 * A, v=3 * A, g=4 * A, B=1, heads=2, grid_h=4, grid_w=4, d_k=64, d_v=64,
+                direction=0, chunk=64, out=5 * A, stream=0)
+
+    def state(**kw):
+        a = dict(base, S0=6 * A, SN=7 * A)
+        a.update(kw)
+        return lib.gtr_gla_forward_state(**a)
+
+    assert state(d_k=16) == 2 and "chunk 64" in lib.last_error()
+    assert state(chunk=32) == 2
+    assert state(d_v=32) == 2
+    assert state(q=None) == 1
+    assert state(S0=6 * A + 4) == 3
+    assert state(SN=7 * A + 8) == 3
+    assert state(SN=A) == 4            # SN over q
+    assert state(SN=6 * A + 256) == 4  # SN partly over S0
+    assert state(S0=5 * A) == 4        # out over S0
+
+    def gated(**kw):
+        a = dict(base, gate=6 * A, norm_weight=7 * A, norm_eps=1e-5)
+        a.update(kw)
+        return lib.gtr_gla_forward_gated(**a)
+
+    assert gated(d_v=128) == 2 and "d_v = 64" in lib.last_error()
+    assert gated(gate=None) == 1
+    assert gated(norm_weight=None) == 1
+    assert gated(norm_eps=-1.0) == 1
+    assert gated(norm_eps=float("nan")) == 1
+    assert gated(gate=6 * A + 2) == 3
+    assert gated(out=6 * A) == 4

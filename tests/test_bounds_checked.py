@@ -17,7 +17,7 @@ from gpu_util import compare
 pytestmark = pytest.mark.gpu
 
 SCHEDULES = {"auto": 0, "fused": 1, "three_phase": 2, "three_phase_simt": 3, "fused_tcgen05": 4,
-             "walk_tcgen05": 5}
+             "walk_tcgen05": 5, "three_phase_mma": 6}
 
 
 @pytest.fixture(scope="module")

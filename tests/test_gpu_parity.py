@@ -15,7 +15,7 @@ from gpu_util import REL_TOL, compare, gpu_inputs, run_forward, sample_slices, s
 
 pytestmark = pytest.mark.gpu
 
-SCHEDULES = ["auto", "fused", "fused_tcgen05", "three_phase", "three_phase_simt", "walk_tcgen05"]
+SCHEDULES = ["auto", "fused", "fused_tcgen05", "three_phase", "three_phase_simt", "walk_tcgen05", "three_phase_mma"]
 # the shapes of the tcgen05 walk kernel and of the tcgen05 three-phase phases
 WALK_SHAPES = [(32, 64), (64, 64), (128, 128), (64, 128), (128, 64), (32, 128)]
 
@@ -356,7 +356,7 @@ def test_cuda_graph_twelve_call_stack(B, heads):
 
 
 @pytest.mark.parametrize("dk,dv", WALK_SHAPES)
-@pytest.mark.parametrize("schedule", ["walk_tcgen05", "three_phase"])
+@pytest.mark.parametrize("schedule", ["walk_tcgen05", "three_phase", "three_phase_mma"])
 def test_walk_shapes_all_directions(oracle_mod, dk, dv, schedule):
     """Every shape of the tcgen05 walk kernel and of the tcgen05 phases, all
     four directions, on a ragged grid (7 x 19 = 133 tokens: two full chunks
@@ -389,3 +389,21 @@ def test_walk_special_gates(oracle_mod, dk, dv):
     qb = torch.where(big[..., None], q.float() * 300.0, q.float()).half()
     out = run_forward(qb, k, v, g, H, W, 1, 64, "walk_tcgen05")
     compare(out, oracle_full(oracle_mod, qb, k, v, g, H, W, 1))
+
+
+def test_chained_tcgen05_control_block_resets_itself(oracle_mod):
+    """The chained tcgen05 kernel's ticket and flags are never cleared by the
+    host: each launch leaves them ready for the next.  Launches of different
+    grid sizes (different sequences and chunk counts) on one stream, each
+    checked against the oracle, then the first shape again; a large problem
+    (400 sequences), a small one and the large one again, so that the small
+    problem's ring would overwrite the large problem's flags if the two
+    shared a buffer."""
+    shapes = [(2, 24, 24, 4), (3, 16, 40, 5), (1, 7, 9, 3), (2, 24, 24, 4), (40, 16, 16, 10), (1, 16, 16, 2),
+              (40, 16, 16, 10)]
+    for i, (B, H, W, heads) in enumerate(shapes):
+        q, k, v, g = gpu_inputs(B, H, W, heads, 64, 64, seed=600 + i)
+        for direction in (i % 4, (i + 1) % 4):
+            out = run_forward(q, k, v, g, H, W, direction, 64, "fused_tcgen05")
+            compare(out, oracle_full(oracle_mod, q, k, v, g, H, W, direction))
+    assert gtr_gla.gtr_gla_get_last_device_status() == 0
