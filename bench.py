@@ -33,7 +33,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from recurrent_vision_backbone_key_b200 import gtr_gla  # noqa: E402
-from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs  # noqa: E402
+from recurrent_vision_backbone_key_b200.synthetic import (  # noqa: E402
+    SSWIGLU_WORKLOADS, WORKLOADS, make_sswiglu_inputs, make_workload_inputs)
 from recurrent_vision_backbone_key_b200 import dist as rdist  # noqa: E402
 
 METRIC = "GLA forward tokens/s and % of roofline (HBM GB/s or TC util) at 1 B200"
@@ -295,14 +296,21 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="batched", choices=sorted(WORKLOADS) + sorted(SSWIGLU_WORKLOADS))
     ap.add_argument("--schedule", default="auto", choices=sorted(gtr_gla.SCHEDULES))
+    ap.add_argument("--dtype", default="f16", choices=["f16", "bf16"],
+                    help="element type of q, k, v and out (bf16: gtr_gla_forward_bf16)")
+    ap.add_argument("--variant", default="plain", choices=["plain", "gated", "state"],
+                    help="gated: output gate on the RMS-normalised output (gtr_gla_forward_gated); "
+                         "state: initial state in, final state out (gtr_gla_forward_state)")
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.workload in SSWIGLU_WORKLOADS:
+        return run_sswiglu(args, SSWIGLU_WORKLOADS[args.workload])
     w = WORKLOADS[args.workload]
 
     if args.impl == "reference":
@@ -315,14 +323,37 @@ def main():
     stream = torch.cuda.current_stream()
     sched = gtr_gla.SCHEDULES[args.schedule]
 
-    q, k, v, g = make_workload_inputs(w, seed=rank, device=f"cuda:{dev}")
-    out = torch.empty((w.B, w.N, w.heads, w.d_v), dtype=torch.float16, device=f"cuda:{dev}")
+    tdtype = torch.bfloat16 if args.dtype == "bf16" else torch.float16
+    if args.dtype == "bf16" and args.variant != "plain":
+        raise SystemExit("--dtype bf16 runs the plain forward only")
+    q, k, v, g = make_workload_inputs(w, seed=rank, device=f"cuda:{dev}", dtype=tdtype)
+    out = torch.empty((w.B, w.N, w.heads, w.d_v), dtype=tdtype, device=f"cuda:{dev}")
     dirs = list(w.directions)
+    extra_bytes = 0  # algorithmic bytes of the variant beyond the forward's
+    if args.variant == "gated":
+        gate = torch.randn((w.B, w.N, w.heads, w.d_v), device=f"cuda:{dev}").to(torch.float16)
+        norm_w = torch.ones(w.d_v, device=f"cuda:{dev}")
+        extra_bytes = w.token_heads * 2 * w.d_v  # the gate read
+    if args.variant == "state":
+        S0 = torch.randn((w.B, w.heads, w.d_k, w.d_v), device=f"cuda:{dev}") * 0.1
+        SN = torch.empty_like(S0)
+        extra_bytes = 2 * S0.numel() * 4  # S_0 read, S_N written
 
     def step(i):
-        gtr_gla.check(gtr_gla.gtr_gla_forward_ex(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w,
-                                                 w.d_k, w.d_v, dirs[i % len(dirs)], w.chunk, sched,
-                                                 out, stream))
+        d = dirs[i % len(dirs)]
+        if args.dtype == "bf16":
+            st = gtr_gla.gtr_gla_forward_bf16(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d,
+                                              w.chunk, out, stream)
+        elif args.variant == "gated":
+            st = gtr_gla.gtr_gla_forward_gated(q, k, v, g, gate, norm_w, 1e-5, w.B, w.heads, w.grid_h, w.grid_w,
+                                               w.d_k, w.d_v, d, w.chunk, out, stream)
+        elif args.variant == "state":
+            st = gtr_gla.gtr_gla_forward_state(q, k, v, g, S0, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d,
+                                               w.chunk, out, SN, stream)
+        else:
+            st = gtr_gla.gtr_gla_forward_ex(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d,
+                                            w.chunk, sched, out, stream)
+        gtr_gla.check(st)
 
     # Inputs smaller than twice L2 would be read from L2 by the next step:
     # then L2 is flushed (a write larger than L2) before every timed step.
@@ -353,9 +384,13 @@ def main():
     # three-phase schedule's per-phase times are reported beside it, their
     # chunk-state traffic counts as overhead, not as work.
     hbm_peak, tc_peak, peak_kind = measured_peaks()
-    alg_bytes = w.algorithmic_bytes()
+    alg_bytes = w.algorithmic_bytes() + extra_bytes
     per_forward_ms = ms / args.steps
     plan, dominant = planned_kernel(w, args.schedule)
+    if args.dtype == "bf16" or args.variant != "plain":  # these entry points always run the walk kernel
+        plan = 5
+        dominant = (f"gla_walk_kernel<{w.d_k},WALK_SEQ>" + (",gated" if args.variant == "gated" else "")
+                    + (",bf16" if args.dtype == "bf16" else ""))
     phase_ms = None
     if plan in (0, 1, 6):  # three phases: time them one by one as well
         phase_ms = time_phases(w, q, k, v, g, out, stream, max(3, min(args.steps, 50)))
@@ -375,14 +410,14 @@ def main():
     # The pages' latency protocol: median CUDA-event time of one forward
     # replayed from a CUDA graph (outside the timed region above).
     graph = None
-    if not args.no_graph:
+    if not args.no_graph and args.dtype == "f16" and args.variant == "plain":
         graph = graph_replay_ms(lambda d, st: gtr_gla.check(gtr_gla.gtr_gla_forward_ex(
             q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, d, w.chunk, sched, out, st)), dirs)
 
     # End to end through the host-buffer entry point: pinned host inputs in,
     # host output back, every step.
     e2e = None
-    if args.e2e_steps > 0:
+    if args.e2e_steps > 0 and args.dtype == "f16" and args.variant == "plain":
         qh, kh, vh, gh = (x.cpu().pin_memory() for x in (q, k, v, g))
         oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
         def e2e_step(i):
@@ -414,11 +449,12 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max / args.steps,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": args.dtype,
             "data": "synthetic",
             "config": {"workload": describe(w), "B": w.B, "grid": [w.grid_h, w.grid_w],
                        "heads": w.heads, "d_k": w.d_k, "d_v": w.d_v, "chunk": w.chunk,
-                       "schedule": args.schedule, "parallelism": f"dp{world} (independent batches)",
+                       "schedule": args.schedule, "variant": args.variant,
+                       "parallelism": f"dp{world} (independent batches)",
                        "l2": (f"inputs larger than L2 ({alg_bytes_total(w) / 1e6:.0f} MB per step), no flush"
                               if flush is None else
                               f"L2 flushed before every timed step ({2 * l2 / 1e6:.0f} MB write, outside the "
@@ -426,6 +462,91 @@ def main():
             "token_heads_per_s": value * w.heads,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "graph": graph,
             "gpu_launches": int(launches), "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    rdist.finalize()
+    return 0
+
+
+def run_sswiglu(args, wl):
+    """Spatial SwiGLU gating with the fused 3x3 depthwise convolution: one
+    gtr_sswiglu_forward call per step over the workload's [B, H*W, C] branches."""
+    rank, world = rdist.init_from_env(backend="nccl")
+    dev = rdist.local_device()
+    torch.cuda.set_device(dev)
+    gtr_gla.load()
+    stream = torch.cuda.current_stream()
+    a, v, wc, bias = make_sswiglu_inputs(wl.B, wl.grid_h, wl.grid_w, wl.C, seed=rank, device=f"cuda:{dev}")
+    out = torch.empty_like(a)
+
+    def step(i):
+        gtr_gla.check(gtr_gla.gtr_sswiglu_forward(a, v, wc, bias, wl.B, wl.grid_h, wl.grid_w, wl.C, out, stream))
+
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = None
+    if wl.algorithmic_bytes() < 2 * l2:
+        scrub = torch.empty(2 * l2, dtype=torch.uint8, device=f"cuda:{dev}")
+        flush = lambda: scrub.fill_(1)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    rdist.barrier()
+    l0 = gtr_gla.gtr_gla_launch_count()
+    with ClockSampler(dev) as clocks:
+        torch.cuda.synchronize()
+        ms = time_steps(step, args.steps, stream, flush)
+        torch.cuda.synchronize()
+    launches = gtr_gla.gtr_gla_launch_count() - l0
+    rdist.barrier()
+    ms_max = rdist.max_over_ranks(ms)
+    value = float(wl.B * wl.N * args.steps * world) / (ms_max * 1e-3)
+    hbm_peak, _, peak_kind = measured_peaks()
+    achieved = wl.algorithmic_bytes() / (ms / args.steps * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s", "frac": achieved / hbm_peak,
+                "traffic": None, "kernel": "sswiglu_kernel", "peak_kind": f"{peak_kind} hbm_gbs (copy, burst)",
+                "algorithmic_bytes_per_launch": wl.algorithmic_bytes()}
+    e2e = None
+    if args.e2e_steps > 0:
+        ah, vh = a.cpu().pin_memory(), v.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        def e2e_step():
+            a.copy_(ah, non_blocking=True)
+            v.copy_(vh, non_blocking=True)
+            step(0)
+            oh.copy_(out, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+        e2e_step()
+        rdist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e2e_s = rdist.max_over_ranks(time.perf_counter() - t0)
+        e2e = {"value": float(wl.B * wl.N * args.e2e_steps * world / e2e_s), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(2 * a.numel() * 2), "d2h_bytes_per_step": int(out.numel() * 2),
+               "steps": args.e2e_steps, "timer": "host wall clock around copies in, the call, the copy out"}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle
+        oracle.build()
+        ac, vc, wcc, bc = a.cpu(), v.cpu(), wc.cpu(), bias.cpu()
+        t0, n = time.perf_counter(), 0
+        while time.perf_counter() - t0 < min(args.cpu_budget, 10.0) and n < wl.B:
+            oracle.sswiglu(ac[n:n + 1], vc[n:n + 1], wcc, bc, wl.grid_h, wl.grid_w)
+            n += 1
+        dt = time.perf_counter() - t0
+        cpu = {"value": n * wl.N / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+               "sample": f"{n} batch items of {wl.N} tokens x {wl.C} channels, fp64, one thread, {dt:.1f} s"}
+    if rank == 0:
+        line = {
+            "metric": "S-SwiGLU gating (3x3 depthwise conv fused) tokens/s and % of HBM roofline at 1 B200",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16", "data": "synthetic",
+            "config": {"workload": f"{wl.name}: B{wl.B} {wl.grid_h}x{wl.grid_w} grid, C={wl.C}",
+                       "parallelism": f"dp{world} (independent batches)",
+                       "l2": ("inputs larger than L2, no flush" if flush is None else "L2 flushed before every step")},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
     rdist.finalize()

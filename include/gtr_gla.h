@@ -157,6 +157,19 @@ gtr_status_t gtr_gla_forward_state(const void *q, const void *k, const void *v, 
                                    const float *S0, int B, int heads, int grid_h, int grid_w, int d_k,
                                    int d_v, int direction, int chunk, void *out, float *SN, void *stream);
 
+/* gtr_gla_forward with bf16 instead of fp16 for q, k, v and out (g stays
+ * fp32): the same recurrence, layouts, checks and error statuses.  The GTR
+ * pages specialise their operator to fp16 and leave other precisions open
+ * (ai.info summary, "Future Directions": broadening kernel coverage to other
+ * precisions); this is that variant.  The tensor-core operands (the
+ * decay-scaled q and k, the masked scores and the scaled state) are bf16,
+ * accumulation and the state fp32.  Runs the walk kernel: chunk 64, d_k in
+ * {32, 64, 128}, d_v in {64, 128} (else GTR_ERR_UNSUPPORTED_SHAPE).  Needs
+ * no workspace. */
+gtr_status_t gtr_gla_forward_bf16(const void *q, const void *k, const void *v, const float *g, int B,
+                                  int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
+                                  int chunk, void *out, void *stream);
+
 /* The forward followed by the output gate on the RMS-normalised output
  * (ai.info summary, "Methodology in Plain English": a separate data-dependent
  * output gate applied to the RMS-normalised output), fused into the output
@@ -222,6 +235,26 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
 gtr_status_t gtr_gla_forward_noalloc(const void *q, const void *k, const void *v, const float *g,
                                      int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                                      int direction, int chunk, void *out, void *stream);
+
+/* Spatial SwiGLU's gating with its 3x3 depthwise convolution, the other
+ * half of each GTR block (ai.info summary, "Methodology in Plain English":
+ * a 3x3 depthwise convolution inserted in the value branch of a SwiGLU
+ * block, on the 2-D patch grid; GTR project page, "Spatial SwiGLU").  For
+ * every batch b, token p = row*grid_w + col and channel c:
+ *     out[b][p][c] = silu(a[b][p][c])
+ *                    * (bias[c] + sum_{dy,dx in -1..1} w[c][dy+1][dx+1] * v[b][p + dy*grid_w + dx][c])
+ * with silu(x) = x * sigmoid(x) and zero padding outside the grid.
+ *   a (device, fp16) [B][grid_h*grid_w][C]: the gate branch;
+ *   v (device, fp16) [B][grid_h*grid_w][C]: the value branch;
+ *   w (device, fp32) [C][3][3]: the depthwise filter; bias (device, fp32) [C],
+ *   or NULL for none; out (device, fp16) [B][grid_h*grid_w][C].
+ * The projections around it (into a and v, and out of the block) are plain
+ * GEMMs outside this library.  C must be a multiple of 8
+ * (GTR_ERR_UNSUPPORTED_SHAPE); a, v and out 16-byte aligned, w and bias 4-byte
+ * aligned (GTR_ERR_MISALIGNED); out must not overlap an input (GTR_ERR_ALIAS).
+ * B == 0, an empty grid or C == 0 is an empty problem.  Needs no workspace. */
+gtr_status_t gtr_sswiglu_forward(const void *a, const void *v, const float *w, const float *bias, int B,
+                                 int grid_h, int grid_w, int C, void *out, void *stream);
 
 /* Phase 1, chunk summaries (GTR project page, "A Kernel That Makes
  * Recurrence Fast": per-chunk summaries in parallel over the chunk x head

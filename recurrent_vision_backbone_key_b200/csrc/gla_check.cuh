@@ -27,6 +27,7 @@ enum BoundsSite : int {
     BS_TC_ROW = 20, BS_TC_LOAD, BS_TC_EXACT, BS_TC_SUMMARY, BS_TC_SENTER, BS_TC_RING, BS_TC_FLAG, BS_TC_OUT,
     BS_SIMT_LOAD = 40, BS_SIMT_SUMMARY, BS_SIMT_SCAN, BS_SIMT_SENTER, BS_SIMT_OUT,
     BS_WALK_ROW = 60, BS_WALK_LOAD, BS_WALK_G, BS_WALK_EXACT, BS_WALK_OUT, BS_WALK_STATE, BS_WALK_SUMMARY, BS_WALK_GATE,
+    BS_SSWIGLU_LOAD = 80, BS_SSWIGLU_W, BS_SSWIGLU_OUT,
 };
 
 // Host: each checked translation unit registers a reader of its report

@@ -43,10 +43,41 @@
 // layout and owns value rows 16w..16w+15 of the state slice.
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "gla_tc.cuh"
 #include "gla_tcgen05.cuh"
 
 namespace gtr {
+
+// Element type of q, k, v, the gate and the output (fp16 or bf16): the
+// tensor-core operands (q, k, v, the masked scores P and the scaled state S')
+// are in this type, accumulation and the state stay fp32.
+template <typename T>
+struct IoType;
+template <>
+struct IoType<__half> {
+    using T2 = __half2;
+    static constexpr int kBf16 = 0;
+    static __device__ __forceinline__ T2 from_f2(float x, float y) { return __floats2half2_rn(x, y); }
+    static __device__ __forceinline__ float2 to_f2(T2 x) { return __half22float2(x); }
+    static __device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
+    static __device__ __forceinline__ __half zero() { return __float2half(0.f); }
+};
+template <>
+struct IoType<__nv_bfloat16> {
+    using T2 = __nv_bfloat162;
+    static constexpr int kBf16 = 1;
+    static __device__ __forceinline__ T2 from_f2(float x, float y) { return __floats2bfloat162_rn(x, y); }
+    static __device__ __forceinline__ float2 to_f2(T2 x) { return __bfloat1622float2(x); }
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+    static __device__ __forceinline__ __nv_bfloat16 zero() { return __float2bfloat16(0.f); }
+};
+template <typename T>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    typename IoType<T>::T2 h = IoType<T>::from_f2(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
 
 enum WalkMode : int { WALK_SEQ = 0, WALK_SUMMARY = 1, WALK_OUTPUT = 2 };
 
@@ -54,10 +85,10 @@ enum WalkMode : int { WALK_SEQ = 0, WALK_SUMMARY = 1, WALK_OUTPUT = 2 };
 constexpr float kWalkChunkRange = 8.0f;
 
 struct WalkArgs {
-    const __half *q, *k, *v;
+    const void *q, *k, *v; // fp16 or bf16 (the kernel's element type)
     const float *g;
     Geom geo;
-    __half *out;           // SEQ, OUTPUT
+    void *out;             // SEQ, OUTPUT
     const float *S0;       // SEQ: initial state [nseq][dk][dv] fp32, or null for zero
     float *SN;             // SEQ: final state [nseq][dk][dv] fp32, or null
     float *dS;             // SUMMARY: [nseq][nc][dk][dv]
@@ -67,7 +98,7 @@ struct WalkArgs {
     int vs;                // 64-wide value slices per sequence (d_v / 64)
     int items;             // SEQ: nseq * vs; SUMMARY, OUTPUT: nseq * nc * vs
     // gated output (d_v = 64): out = o / sqrt(mean(o^2) + eps) * w * silu(gate)
-    const __half *gate;    // [B][N][heads][d_v] gate pre-activation
+    const void *gate;      // [B][N][heads][d_v] gate pre-activation (element type)
     const float *norm_w;   // [d_v] RMS-norm weight
     float norm_eps;
 };
@@ -100,8 +131,13 @@ __device__ __forceinline__ uint32_t swz(int row, int col) {
 // GATED (WALK_SEQ, d_v = 64): the output store applies the output gate on
 // the RMS-normalised output (ai.info summary, "Methodology in Plain English"):
 // out = o / sqrt(mean over the head's d_v values of o^2 + eps) * w * silu(gate).
-template <int DK, int MODE, bool GATED>
+template <int DK, int MODE, bool GATED, typename T>
 __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel(const WalkArgs args) {
+    using IO = IoType<T>;
+    using T2 = typename IO::T2;
+    const T *gq_ = static_cast<const T *>(args.q), *gk_ = static_cast<const T *>(args.k);
+    const T *gv_ = static_cast<const T *>(args.v);
+    T *gout_ = static_cast<T *>(args.out);
     using L = WalkLayout<DK>;
     constexpr int KT = DK / 8;           // 8-wide key tiles of the state fragment
     constexpr int PPL = DK > 64 ? 2 : 1; // key-dimension pairs per lane in the prep
@@ -170,8 +206,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 const int64_t o = ok ? r * DK + jq * 8 : 0;
                 const uint32_t so = (uint32_t)(jq >> 3) * 8192u + (uint32_t)t * 128u +
                                     ((((uint32_t)jq & 7u) ^ (uint32_t)(t & 7)) << 4);
-                if (kOut) cp_async16_s(sb + L::SQ + so, args.q + o, ok);
-                cp_async16_s(sb + L::SK + so, args.k + o, ok);
+                if (kOut) cp_async16_s(sb + L::SQ + so, gq_ + o, ok);
+                cp_async16_s(sb + L::SK + so, gk_ + o, ok);
             }
             const int jv = lane & 7, rv = lane >> 3;
 #pragma unroll
@@ -181,7 +217,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 const int64_t o = r * DV + sl * DV_CTA + jv * 8;
                 const bool ok = r >= 0 && GTR_INB(o + 7, rows * DV, BS_WALK_LOAD);
                 cp_async16_s(sb + L::SV + (uint32_t)t * 128u + ((((uint32_t)jv) ^ (uint32_t)(t & 7)) << 4),
-                             args.v + (ok ? o : 0), ok);
+                             gv_ + (ok ? o : 0), ok);
             }
             if constexpr (L::kGsmem) {
                 constexpr int GCH = DK / 4;     // pieces of a g row (fp32)
@@ -319,7 +355,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         // ---- this lane's column pairs of the warp's 16 rows of q and k, read
         // once (all loads before any store), and the |q~| test
         uint32_t ro[PPL][16];
-        __half2 qv[PPL][16], kv[PPL][16];
+        T2 qv[PPL][16], kv[PPL][16];
         float qm = 0.f;
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
@@ -332,16 +368,14 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 ro[p][t] = cb + (uint32_t)row * 128u + (((uint32_t)(dc >> 3) ^ (uint32_t)(row & 7)) << 4);
             }
 #pragma unroll
-            for (int t = 0; t < 16; ++t) kv[p][t] = *reinterpret_cast<const __half2 *>(base + sb + L::SK + ro[p][t]);
+            for (int t = 0; t < 16; ++t) kv[p][t] = *reinterpret_cast<const T2 *>(base + sb + L::SK + ro[p][t]);
             if (kOut) {
-                __half2 qmax = __float2half2_rn(0.f);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
-                    qv[p][t] = *reinterpret_cast<const __half2 *>(base + sb + L::SQ + ro[p][t]);
-                    qmax = __hmax2(qmax, __habs2(qv[p][t]));
+                    qv[p][t] = *reinterpret_cast<const T2 *>(base + sb + L::SQ + ro[p][t]);
+                    const float2 qf = IO::to_f2(qv[p][t]);
+                    qm = fmaxf(qm, fmaxf(fabsf(qf.x), fabsf(qf.y)));
                 }
-                const float2 qf = __half22float2(qmax);
-                qm = fmaxf(qm, fmaxf(qf.x, qf.y));
             }
         }
         // (A) every warp's totals visible; any |q~| > 16 in the chunk
@@ -384,13 +418,13 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 for (int t = 0; t < 16; ++t) {
                     E.x *= av[p][t].x;
                     E.y *= av[p][t].y;
-                    *reinterpret_cast<__half2 *>(base + sb + L::SQ + ro[p][t]) = __hmul2(qv[p][t], __floats2half2_rn(E.x, E.y));
+                    *reinterpret_cast<T2 *>(base + sb + L::SQ + ro[p][t]) = __hmul2(qv[p][t], IO::from_f2(E.x, E.y));
                 }
             }
             float2 S = Sb[p];  // decay after token t to the chunk end
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
-                *reinterpret_cast<__half2 *>(base + sb + L::SK + ro[p][t]) = __hmul2(kv[p][t], __floats2half2_rn(S.x, S.y));
+                *reinterpret_cast<T2 *>(base + sb + L::SK + ro[p][t]) = __hmul2(kv[p][t], IO::from_f2(S.x, S.y));
                 S.x *= av[p][t].x;
                 S.y *= av[p][t].y;
             }
@@ -420,9 +454,9 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 if (exact) gx = gy = 1.f;
                 const uint32_t hb = (uint32_t)p * 8192u, ch = (uint32_t)(n & 7);
                 *reinterpret_cast<uint32_t *>(base + L::SP + hb + rb0 + ((ch ^ x0) << 4)) =
-                    pack_h2(gx * Se[n][0], gy * Se[n][1]);
+                    pack2<T>(gx * Se[n][0], gy * Se[n][1]);
                 *reinterpret_cast<uint32_t *>(base + L::SP + hb + rb1 + ((ch ^ x1) << 4)) =
-                    pack_h2(gx * Se[n][2], gy * Se[n][3]);
+                    pack2<T>(gx * Se[n][2], gy * Se[n][3]);
             }
         }
         fence_async_shared();
@@ -436,14 +470,14 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             tc_fence_after();
             const uint64_t so = (uint64_t)(sb >> 4);
             if (kOut && !exact) {
-                constexpr uint32_t id = umma_idesc(0, 0, 64, 64);
+                constexpr uint32_t id = umma_idesc(0, 0, 64, 64, IO::kBf16);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint64_t ko = so + (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
                     umma_f16(tmem, dQk + ko, dKk + ko, id, ks > 0);
                 }
             }
-            constexpr uint32_t id2 = umma_idesc(1, 1, 64, DK);
+            constexpr uint32_t id2 = umma_idesc(1, 1, 64, DK, IO::kBf16);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) umma_f16(tmem + kDsLanes, dVm + so + 128 * ks, dKm + so + 128 * ks, id2, ks > 0);
             umma_commit(mbar1);
@@ -452,7 +486,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             if (have_state) {
                 tc_fence_after();
                 const uint64_t so = (uint64_t)(sb >> 4);
-                constexpr uint32_t id_qs = umma_idesc(0, 0, 64, 64);
+                constexpr uint32_t id_qs = umma_idesc(0, 0, 64, 64, IO::kBf16);
 #pragma unroll
                 for (int ks = 0; ks < DK / 16; ++ks) {
                     const uint64_t ko = (uint64_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4);
@@ -473,8 +507,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             float pe[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) pe[j] = 0.f;
-            __half *xq = reinterpret_cast<__half *>(base + L::P);         // [64][16]
-            __half *xk = reinterpret_cast<__half *>(base + L::P + 2048);  // [64][16]
+            T *xq = reinterpret_cast<T *>(base + L::P);         // [64][16]
+            T *xk = reinterpret_cast<T *>(base + L::P + 2048);  // [64][16]
             float *xb = reinterpret_cast<float *>(base + L::P + 4096);    // [64][16]
             for (int hd = 0; hd < DK / 16; ++hd) {
                 __syncthreads();
@@ -483,8 +517,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                     const int64_t r = rowt[tt];
                     const int64_t o = (r < 0 ? 0 : r) * DK + 16 * hd + d;
                     const bool ok = r >= 0 && GTR_INB(o, rows * DK, BS_WALK_EXACT);
-                    xq[idx] = ok ? args.q[o] : __float2half(0.f);
-                    xk[idx] = ok ? args.k[o] : __float2half(0.f);
+                    xq[idx] = ok ? gq_[o] : IO::zero();
+                    xk[idx] = ok ? gk_[o] : IO::zero();
                     xb[idx] = ok ? args.g[o] * kLog2e : 0.f;
                 }
                 __syncthreads();
@@ -497,24 +531,39 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 }
                 __syncthreads();
                 for (int d = 0; d < 16; ++d) {
-                    const float qq = __half2float(xq[t * 16 + d]) * qscale;
+                    const float qq = IO::to_f(xq[t * 16 + d]) * qscale;
                     const float bt = xb[t * 16 + d];
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int sk = sbk + j;
-                        if (sk <= t) pe[j] = fmaf(qq * __half2float(xk[sk * 16 + d]), ex2(bt - xb[sk * 16 + d]), pe[j]);
+                        if (sk <= t) pe[j] = fmaf(qq * IO::to_f(xk[sk * 16 + d]), ex2(bt - xb[sk * 16 + d]), pe[j]);
                     }
                 }
             }
             __syncthreads();  // the staging in the score region is consumed
 #pragma unroll
             for (int j = 0; j < 32; j += 2)
-                *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sbk + j)) = pack_h2(pe[j], pe[j + 1]);
+                *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sbk + j)) = pack2<T>(pe[j], pe[j + 1]);
         }
 
         if (!mbar_wait(mbar1, ph1)) mma_ok = false;
         ph1 ^= 1u;
         tc_fence_after();
+        if constexpr (GATED) {
+            // the gate rows of this warp's tokens into the S' tile (pass 1 has
+            // read it; the readout is in TMEM), swizzled like the output rows,
+            // in flight while the scores and pass 2 are done
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
+                const int64_t r = rowt[t];
+                const int64_t o_off = r * DV + j * 8;
+                const bool ok = t < len && r >= 0 && GTR_INB(o_off + 7, rows * DV, BS_WALK_GATE);
+                cp_async16_s(base_addr + L::SP + t * 128 + (((j ^ (t & 7)) & 7) << 4),
+                             static_cast<const T *>(args.gate) + (ok ? o_off : 0), ok);
+            }
+            cp_async_commit();
+        }
 
         // ---- the chunk summary of this value slice: the state update, or
         // (phase 1) dS_c and gamma_c written out
@@ -578,7 +627,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                         const int t = 16 * warp + tr + 8 * hf, sk = 8 * n + kc;
                         const float x0 = sk <= t ? a[4 * n + 2 * hf] : 0.f;
                         const float x1 = sk + 1 <= t ? a[4 * n + 2 * hf + 1] : 0.f;
-                        *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sk)) = pack_h2(x0, x1);
+                        *reinterpret_cast<uint32_t *>(base + L::P + sw128(t, sk)) = pack2<T>(x0, x1);
                     }
                 }
             }
@@ -590,25 +639,11 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             if (tid == 0) {
                 tc_fence_after();
                 const uint64_t so = (uint64_t)(sb >> 4);
-                constexpr uint32_t id_pv = umma_idesc(0, 1, 64, 64);
+                constexpr uint32_t id_pv = umma_idesc(0, 1, 64, 64, IO::kBf16);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     umma_f16(tmem + kOCol, dP + 2 * ks, dVm + so + 128 * ks, id_pv, (ks > 0 || have_state) ? 1u : 0u);
                 umma_commit(mbar2);
-            }
-            // gate rows of this warp's tokens (16-byte pieces, the store
-            // pattern below), in flight while pass 2 runs
-            int4 gr[4];
-            if constexpr (GATED) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
-                    const int64_t r = rowt[t];
-                    const int64_t o_off = r * DV + j * 8;
-                    gr[i] = (t < len && r >= 0 && GTR_INB(o_off + 7, rows * DV, BS_WALK_GATE))
-                                ? __ldcs(reinterpret_cast<const int4 *>(args.gate + o_off))
-                                : make_int4(0, 0, 0, 0);
-                }
             }
             if (!mbar_wait(mbar2, ph2)) mma_ok = false;
             ph2 ^= 1u;
@@ -622,12 +657,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 tc_wait_ld();
                 unsigned char *st = base + L::P;
                 if constexpr (GATED) {
-                    // the gate rows into the S' tile (pass 2 has read it), swizzled
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
-                        *reinterpret_cast<int4 *>(base + L::SP + t * 128 + (((j ^ (t & 7)) & 7) << 4)) = gr[i];
-                    }
+                    // the gate rows (copied into the S' tile after pass 1) have landed
+                    cp_async_wait_group<0>();
                     __syncwarp();
                     // 1 / rms of rows tr and tr + 8 (fp32, over the 64 values
                     // that lanes 4tr..4tr+3 hold)
@@ -647,19 +678,19 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                     for (int n = 0; n < 8; ++n) {
                         const int t = 16 * warp + tr, col = 8 * n + kc;
                         const float2 w = __ldg(reinterpret_cast<const float2 *>(args.norm_w + col));
-                        const float2 r0 = __half22float2(*reinterpret_cast<const __half2 *>(base + L::SP + sw128(t, col)));
-                        const float2 r1 = __half22float2(*reinterpret_cast<const __half2 *>(base + L::SP + sw128(t + 8, col)));
-                        o[4 * n + 0] *= inv0 * w.x * (r0.x / (1.f + __expf(-r0.x)));
-                        o[4 * n + 1] *= inv0 * w.y * (r0.y / (1.f + __expf(-r0.y)));
-                        o[4 * n + 2] *= inv1 * w.x * (r1.x / (1.f + __expf(-r1.x)));
-                        o[4 * n + 3] *= inv1 * w.y * (r1.y / (1.f + __expf(-r1.y)));
+                        const float2 r0 = IO::to_f2(*reinterpret_cast<const T2 *>(base + L::SP + sw128(t, col)));
+                        const float2 r1 = IO::to_f2(*reinterpret_cast<const T2 *>(base + L::SP + sw128(t + 8, col)));
+                        o[4 * n + 0] *= inv0 * w.x * __fdividef(r0.x, 1.f + __expf(-r0.x));
+                        o[4 * n + 1] *= inv0 * w.y * __fdividef(r0.y, 1.f + __expf(-r0.y));
+                        o[4 * n + 2] *= inv1 * w.x * __fdividef(r1.x, 1.f + __expf(-r1.x));
+                        o[4 * n + 3] *= inv1 * w.y * __fdividef(r1.y, 1.f + __expf(-r1.y));
                     }
                 }
 #pragma unroll
                 for (int n = 0; n < 8; ++n) {
                     const int t = 16 * warp + tr, col = 8 * n + kc;
-                    *reinterpret_cast<uint32_t *>(st + sw128(t, col)) = pack_h2(o[4 * n], o[4 * n + 1]);
-                    *reinterpret_cast<uint32_t *>(st + sw128(t + 8, col)) = pack_h2(o[4 * n + 2], o[4 * n + 3]);
+                    *reinterpret_cast<uint32_t *>(st + sw128(t, col)) = pack2<T>(o[4 * n], o[4 * n + 1]);
+                    *reinterpret_cast<uint32_t *>(st + sw128(t + 8, col)) = pack2<T>(o[4 * n + 2], o[4 * n + 3]);
                 }
                 __syncwarp();
 #pragma unroll
@@ -668,7 +699,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                     const int64_t r = rowt[t];
                     const int64_t o_off = r * DV + sl * DV_CTA + j * 8;
                     if (t < len && r >= 0 && GTR_INB(o_off + 7, rows * DV, BS_WALK_OUT))
-                        *reinterpret_cast<int4 *>(args.out + o_off) =
+                        *reinterpret_cast<int4 *>(gout_ + o_off) =
                             *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
                 }
             }
@@ -704,33 +735,34 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 }
 
 // Resident CTAs per SM of one instantiation (cached per device by the caller).
-template <int DK, int MODE, bool GATED>
+template <int DK, int MODE, bool GATED, typename T>
 cudaError_t walk_occupancy(int *ctas) {
     using L = WalkLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>,
+    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, gla_walk_kernel<DK, MODE, GATED>, 128, L::ALLOC);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, gla_walk_kernel<DK, MODE, GATED, T>, 128, L::ALLOC);
 }
 
-template <int DK, int MODE, bool GATED>
+template <int DK, int MODE, bool GATED, typename T>
 cudaError_t launch_walk_t(const WalkArgs &a, int grid, cudaStream_t st) {
     using L = WalkLayout<DK>;
-    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>,
+    cudaError_t e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::ALLOC);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    gla_walk_kernel<DK, MODE, GATED><<<grid, 128, L::ALLOC, st>>>(a);
+    gla_walk_kernel<DK, MODE, GATED, T><<<grid, 128, L::ALLOC, st>>>(a);
     count_launch();
     return cudaGetLastError();
 }
 
 // Launchers (gla_walk.cu): grid CTAs; `grid` <= a.items.  a.gate != null
-// selects the gated output (WALK_SEQ with d_v = 64 only).
-cudaError_t launch_walk(const WalkArgs &a, int mode, int grid, cudaStream_t st);
+// selects the gated output (WALK_SEQ with d_v = 64 only); bf16 selects bf16
+// q, k, v, gate and output (WALK_SEQ only).
+cudaError_t launch_walk(const WalkArgs &a, int mode, int grid, cudaStream_t st, bool bf16 = false);
 // Resident CTAs per SM for (d_k, mode), or 0 for an unsupported d_k.
 cudaError_t walk_ctas_per_sm(int dk, int mode, int *ctas);
 

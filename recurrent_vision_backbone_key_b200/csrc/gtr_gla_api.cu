@@ -293,7 +293,8 @@ WalkArgs make_walk_args(const __half *q, const __half *k, const __half *v, const
 // S0 / SN: initial and final states [B*heads][d_k][d_v] fp32, or null.
 gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const float *g, const Geom &geo,
                       __half *out, cudaStream_t st, const float *S0 = nullptr, float *SN = nullptr,
-                      const __half *gate = nullptr, const float *norm_w = nullptr, float norm_eps = 0.f) {
+                      const __half *gate = nullptr, const float *norm_w = nullptr, float norm_eps = 0.f,
+                      bool bf16 = false) {
     unsigned *status = nullptr;
     gtr_status_t s = status_word(st, &status);
     if (s != GTR_OK) return s;
@@ -305,7 +306,7 @@ gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const f
     a.norm_w = norm_w;
     a.norm_eps = norm_eps;
     a.items = geo.B * geo.heads * a.vs;
-    cudaError_t e = launch_walk(a, WALK_SEQ, a.items, st);
+    cudaError_t e = launch_walk(a, WALK_SEQ, a.items, st, bf16);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "walk kernel launch");
 }
 
@@ -516,6 +517,23 @@ gtr_status_t gtr_gla_forward_state(const void *q, const void *k, const void *v, 
                     g, geo, static_cast<__half *>(out), static_cast<cudaStream_t>(stream), S0, SN);
 }
 
+gtr_status_t gtr_gla_forward_bf16(const void *q, const void *k, const void *v, const float *g, int B, int heads,
+                                  int grid_h, int grid_w, int d_k, int d_v, int direction, int chunk, void *out,
+                                  void *stream) {
+    t_err_clear();
+    Geom geo;
+    bool empty = false;
+    gtr_status_t s = check_walk_call(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                                     geo, empty);
+    if (s != GTR_OK) return s;
+    if (empty) return GTR_OK;
+    // the buffers hold bf16 values; the walk kernel reads them through its
+    // bf16 instantiation (the pointer types below only carry the addresses)
+    return run_walk(static_cast<const __half *>(q), static_cast<const __half *>(k), static_cast<const __half *>(v),
+                    g, geo, static_cast<__half *>(out), static_cast<cudaStream_t>(stream), nullptr, nullptr,
+                    nullptr, nullptr, 0.f, true);
+}
+
 gtr_status_t gtr_gla_forward_gated(const void *q, const void *k, const void *v, const float *g,
                                               const void *gate, const float *norm_weight, float norm_eps, int B,
                                               int heads, int grid_h, int grid_w, int d_k, int d_v, int direction,
@@ -663,6 +681,29 @@ gtr_status_t gtr_gla_forward_host(const void *q, const void *k, const void *v, c
     if ((e = cudaStreamSynchronize(hp->down)) != cudaSuccess) return drain(cuda_fail(e, "cudaStreamSynchronize"));
     // the forward ran on the internal compute stream: report its bounded waits here
     return gtr_gla_get_last_device_status(hp->run);
+}
+
+gtr_status_t gtr_sswiglu_forward(const void *a, const void *v, const float *w, const float *bias, int B, int grid_h,
+                                 int grid_w, int C, void *out, void *stream) {
+    t_err_clear();
+    if (B < 0 || grid_h < 0 || grid_w < 0 || C < 0) return fail(GTR_ERR_INVALID_ARG, "negative size%s");
+    if (C % 8 != 0) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "C must be a multiple of 8%s");
+    const int64_t N = (int64_t)grid_h * grid_w;
+    if (N > ((int64_t)1 << 30)) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "more than 2^30 tokens%s");
+    if (B > 65535 || C / 64 + 1 > 65535) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "B or C too large%s");
+    if (!a || !v || !w || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
+    if (!aligned16(a) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u) ||
+        (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
+        return fail(GTR_ERR_MISALIGNED, "a, v, out must be 16-byte aligned, w and bias 4-byte aligned%s");
+    const size_t nb = (size_t)B * N * C * 2;
+    const Range ro = span(out, nb);
+    if (overlap(ro, span(a, nb)) || overlap(ro, span(v, nb)) || overlap(ro, span(w, (size_t)C * 36)) ||
+        (bias && overlap(ro, span(bias, (size_t)C * 4))))
+        return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
+    if (B == 0 || N == 0 || C == 0) return GTR_OK;
+    cudaError_t e = launch_sswiglu(static_cast<const __half *>(a), static_cast<const __half *>(v), w, bias, B, grid_h,
+                                   grid_w, C, static_cast<__half *>(out), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? GTR_OK : cuda_fail(e, "S-SwiGLU kernel launch");
 }
 
 gtr_status_t gtr_gla_chunk_summary(const void *k, const void *v, const float *g, int B, int heads,

@@ -40,9 +40,11 @@ SIGNATURES = {
     "gtr_gla_forward_ex": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_host": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_noalloc": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
+    "gtr_gla_forward_bf16": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_forward_state": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gtr_gla_forward_gated": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_float, _I, _I, _I, _I, _I, _I, _I, _I,
                                    _P, _P]),
+    "gtr_sswiglu_forward": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_summary": (_I, [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
     "gtr_gla_boundary_scan": (_I, [_P, _P, _I, _I, _I, _I, _I, _P, _P]),
     "gtr_gla_chunk_output": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _P, _P]),
@@ -172,6 +174,12 @@ def gtr_gla_forward_noalloc(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, dire
                                           _stream(stream))
 
 
+def gtr_gla_forward_bf16(q, k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
+                         stream=None) -> int:
+    return load().gtr_gla_forward_bf16(_addr(q), _addr(k), _addr(v), _addr(g), B, heads, grid_h, grid_w,
+                                       d_k, d_v, _dir(direction), chunk, _addr(out), _stream(stream))
+
+
 def gtr_gla_forward_state(q, k, v, g, S0, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, out,
                           SN, stream=None) -> int:
     return load().gtr_gla_forward_state(_addr(q), _addr(k), _addr(v), _addr(g), _addr(S0), B, heads,
@@ -184,6 +192,11 @@ def gtr_gla_forward_gated(q, k, v, g, gate, norm_weight, norm_eps, B, heads, gri
     return load().gtr_gla_forward_gated(_addr(q), _addr(k), _addr(v), _addr(g), _addr(gate),
                                         _addr(norm_weight), float(norm_eps), B, heads, grid_h, grid_w,
                                         d_k, d_v, _dir(direction), chunk, _addr(out), _stream(stream))
+
+
+def gtr_sswiglu_forward(a, v, w, bias, B, grid_h, grid_w, C, out, stream=None) -> int:
+    return load().gtr_sswiglu_forward(_addr(a), _addr(v), _addr(w), _addr(bias), B, grid_h, grid_w, C,
+                                      _addr(out), _stream(stream))
 
 
 def gtr_gla_chunk_summary(k, v, g, B, heads, grid_h, grid_w, d_k, d_v, direction, chunk, dS, gamma,

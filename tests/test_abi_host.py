@@ -231,3 +231,24 @@ def test_state_and_gated_entry_points_validate(lib):
     assert gated(norm_eps=float("nan")) == 1
     assert gated(gate=6 * A + 2) == 3
     assert gated(out=6 * A) == 4
+
+
+def test_sswiglu_entry_point_validates(lib):
+    args = dict(a=A, v=2 * A, w=3 * A, bias=4 * A, B=1, grid_h=4, grid_w=4, C=64, out=5 * A, stream=0)
+
+    def call(**kw):
+        a = dict(args)
+        a.update(kw)
+        return lib.gtr_sswiglu_forward(**a)
+
+    assert call(C=12) == 2 and "multiple of 8" in lib.last_error()
+    assert call(B=-1) == 1
+    assert call(a=None) == 1
+    assert call(w=None) == 1
+    assert call(a=A + 8) == 3
+    assert call(w=3 * A + 2) == 3
+    assert call(out=A + 64) == 4
+    assert call(out=3 * A) == 4
+    before = lib.gtr_gla_launch_count()
+    assert call(B=0) == 0 and call(grid_h=0) == 0 and call(C=0) == 0
+    assert lib.gtr_gla_launch_count() == before

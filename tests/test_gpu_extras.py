@@ -172,3 +172,60 @@ def test_state_and_gate_reject_unsupported():
     w = torch.ones(128, device="cuda")
     assert gtr_gla.gtr_gla_forward_gated(q, k, v, g, r, w, 1e-5, 1, 1, 4, 4, 64, 128, 0, 64, out) == 2
     assert "d_v = 64" in gtr_gla.last_error()
+
+
+# bf16 I/O: the forward's bar scaled from fp16 to bf16 unit roundoff.  The
+# fp16 bar, 2e-3 of max |o_ref|, is about 4 units of fp16 roundoff (2^-11);
+# bf16 rounds 8 times coarser (2^-8 against 2^-11), so the same number of
+# units is 8 * 2e-3 = 1.6e-2 of max |o_ref|.
+BF16_TOL = 1.6e-2
+
+
+@pytest.mark.parametrize("dk,dv", WALK_SHAPES)
+def test_bf16_against_oracle(oracle_mod, dk, dv):
+    for (B, H, W, heads) in [(2, 7, 19, 3), (1, 16, 24, 2)]:
+        q, k, v, g = make_inputs(B, H, W, heads, dk, dv, seed=dk + dv + W, dtype=torch.bfloat16)
+        qd, kd, vd, gd = (x.cuda() for x in (q, k, v, g))
+        for direction in range(4):
+            out = torch.full_like(vd, float("nan"))
+            gtr_gla.check(gtr_gla.gtr_gla_forward_bf16(qd, kd, vd, gd, B, heads, H, W, dk, dv, direction, 64, out))
+            torch.cuda.synchronize()
+            compare(out, oracle_mod.gla_serial(q, k, v, g, H, W, direction), tol=BF16_TOL)
+
+
+def test_bf16_special_gates(oracle_mod):
+    B, H, W, heads, dk, dv = 2, 10, 13, 2, 64, 64
+    q, k, v, g = make_inputs(B, H, W, heads, dk, dv, seed=3, dtype=torch.bfloat16)
+    cases = {"open": torch.zeros_like(g), "closed": torch.full_like(g, -1.0e4),
+             "strong": make_inputs(B, H, W, heads, dk, dv, seed=3, gate="strong")[3]}
+    for name, gg in cases.items():
+        out = torch.empty_like(v).cuda()
+        gtr_gla.check(gtr_gla.gtr_gla_forward_bf16(q.cuda(), k.cuda(), v.cuda(), gg.cuda(), B, heads, H, W, dk, dv,
+                                                   2, 64, out))
+        torch.cuda.synchronize()
+        compare(out, oracle_mod.gla_serial(q, k, v, gg, H, W, 2), tol=BF16_TOL)
+
+
+def test_deployment_shape_full_size_sampled(oracle_mod):
+    """The pages' deployment shape (d_k = 32, d_v = 64, chunk 64) at the
+    batched size, fp16 through AUTO and bf16, 24 sampled sequences each."""
+    from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs
+    w = WORKLOADS["deploy_batched"]
+    for dtype, tol in ((torch.float16, 2e-3), (torch.bfloat16, BF16_TOL)):
+        q, k, v, g = make_workload_inputs(w, seed=5, device="cuda", dtype=dtype)
+        out = torch.empty_like(v)
+        if dtype == torch.float16:
+            gtr_gla.check(gtr_gla.gtr_gla_forward(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v, 2,
+                                                  64, out))
+        else:
+            gtr_gla.check(gtr_gla.gtr_gla_forward_bf16(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v,
+                                                       2, 64, out))
+        torch.cuda.synchronize()
+        rng = np.random.default_rng(1)
+        picks = {(0, 0), (w.B - 1, w.heads - 1)}
+        while len(picks) < 24:
+            picks.add((int(rng.integers(w.B)), int(rng.integers(w.heads))))
+        for b, h in sorted(picks):
+            sl = lambda x: x[b:b + 1, :, h:h + 1, :].cpu()
+            compare(out[b:b + 1, :, h:h + 1, :], oracle_mod.gla_serial(sl(q), sl(k), sl(v), sl(g), w.grid_h,
+                                                                       w.grid_w, 2), tol=tol)
