@@ -14,6 +14,10 @@
     what carries over: at most the forward's 2e-3 for the numerator, as much
     again through the rms itself, plus one fp16 rounding of the result
     (2^-11 ~ 4.9e-4); 2 * 2e-3 + 4.9e-4 < 5e-3.
+  * gtr_gla_forward_bf16: bf16 q, k, v and out (ai.info summary, "Future
+    Directions": other precisions), at the bar scaled by the ratio of unit
+    roundoffs (BF16_TOL below), and the pages' deployment shape d_k = 32,
+    d_v = 64 at the batched size.
 """
 import numpy as np
 import pytest
