@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(mbar1, kOut ? 2 : 1);  // pass 1 completes from threads 0 and 32
+        mbar_init(mbar1, kOut ? 3 : 1);  // pass 1 completes from threads 0, 32 and 64
         mbar_init(mbar2, 1);
         asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
     }
@@ -463,9 +463,13 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         tc_fence_before();
         __syncthreads();  // (B) operands, S' and gamma written
 
-        // ---- pass 1: A = qh ke^T (lanes 0-15, columns 0-63) and dS^T = V^T ke
-        // (lanes 16-31) from thread 0; the readout O = qh S' (lanes 0-15,
-        // columns 64-127) from thread 32 at the same time
+        // ---- pass 1, issued from three threads at once (each issuing thread
+        // pays its own per-instruction cost, so three queues of four MMAs
+        // finish issuing sooner than one of twelve): A = qh ke^T (lanes 0-15,
+        // columns 0-63) from thread 0, dS^T = V^T ke (lanes 16-31) from
+        // thread 64 (thread 0 in phase 1, which has no A), the readout
+        // O = qh S' (lanes 0-15, columns 64-127) from thread 32; the three
+        // write disjoint accumulators
         if (tid == 0) {
             tc_fence_after();
             const uint64_t so = (uint64_t)(sb >> 4);
@@ -477,6 +481,20 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                     umma_f16(tmem, dQk + ko, dKk + ko, id, ks > 0);
                 }
             }
+            if (!kOut) {
+                constexpr uint32_t id2 = umma_idesc(1, 1, 64, DK, IO::kBf16);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem + kDsLanes, dVm + so + 128 * ks, dKm + so + 128 * ks, id2, ks > 0);
+            }
+            if (kOut && exact)
+                mbar_arrive(mbar1);
+            else
+                umma_commit(mbar1);
+        }
+        if (kOut && tid == 64) {
+            tc_fence_after();
+            const uint64_t so = (uint64_t)(sb >> 4);
             constexpr uint32_t id2 = umma_idesc(1, 1, 64, DK, IO::kBf16);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) umma_f16(tmem + kDsLanes, dVm + so + 128 * ks, dKm + so + 128 * ks, id2, ks > 0);
