@@ -29,7 +29,10 @@
 //   16 x 16 diagonal blocks need exp(b_t - b_s) directly: when the decay
 //   over the sub-chunk is at most kDiagRange nats they use the reference
 //   token 7 (qd = qs / P_7, kd = ke / Suf_7, factors within e^{+-kDiagRange},
-//   fp16 tensor-core product); otherwise exact per-pair exponentials in fp32.
+//   fp16 tensor-core product); when it is at most kMidRange nats, the same
+//   reference with fp32 factors taken from the raw operands and a tf32
+//   tensor-core product (factors within e^{+-kMidRange}, inside fp32 and
+//   tf32 range); otherwise exact per-pair exponentials in fp32.
 //   Then, with E_u the decay from the chunk start to sub-chunk u,
 //     o_t = qs_t L_u + sum_{s<=t in u} A_ts v_s + (qs_t E_u) S_enter,
 //     S_leave = diag(gamma_c) S_enter + L_last.
@@ -49,6 +52,13 @@ enum TcMode : int { TC_SUMMARY = 0, TC_OUTPUT = 1, TC_FUSED = 2, TC_FUSED_PAIR =
 constexpr float kDiagRange = 5.0f;
 // Largest |q~| or |k| for that path (keeps e^{kDiagRange} * value in fp16).
 constexpr float kDiagMaxAbs = 64.0f;
+// Largest ratio (nats) between two in-sub-chunk decay prefixes for the tf32
+// form of the diagonal block, and the largest |q~| or |k| it takes (keeps
+// e^{kMidRange} * value inside fp32).
+constexpr float kMidRange = 80.0f;
+constexpr float kMidMaxAbs = 1024.0f;
+// Diagonal-block forms of a sub-chunk (its flag word).
+enum DiagForm : int { DIAG_FP16 = 0, DIAG_TF32 = 1, DIAG_EXACT = 2 };
 
 struct TcArgs {
     const __half *q, *k, *v;
@@ -105,6 +115,21 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// D += A(16x8, row) * B(8x8, col), tf32 in, fp32 accumulate.
+__device__ __forceinline__ void mma1688_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// fp32 -> tf32 (round to nearest, ties away), as a 32-bit operand.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t y;
+    asm("cvt.rna.tf32.f32 %0, %1;\n" : "=r"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
     __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&h);
@@ -137,7 +162,7 @@ __device__ __forceinline__ void st_release(int *p, int v) {
 // ------------------------------------------------------------ smem layout
 
 // One block of shared memory per chunk of the tile (NCH chunks per tile).
-template <int DK, int DV, int NCH>
+template <int DK, int DV, int NCH, bool MID>
 struct TcLayout {
     static constexpr int LDK = DK + 8;  // fp16 row stride (halves): 16-byte rows, conflict-free ldmatrix
     static constexpr int LDV = DV + 8;
@@ -163,11 +188,24 @@ struct TcLayout {
     __host__ __device__ static size_t scratch_bytes(int C) {
         size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8, gs = (size_t)C * DK * 4;
         size_t hs = NCH > 1 ? (size_t)DK * DV * 4 : 0;
+        size_t md = (size_t)(C >= 32 ? 2 : 1) * 32 * DK * 4;  // tf32 diagonal factors
         size_t m = o > e ? o : e;
         m = m > gs ? m : gs;
+        m = m > md ? m : md;
         return m > hs ? m : hs;
     }
-    __host__ __device__ static size_t block(int C) { return (scratch(C) + scratch_bytes(C) + 127) & ~(size_t)127; }
+    // MID (the fused schedule) with d_k = d_v = 128 (one CTA per SM, shared
+    // memory to spare): the prepared qs, ke go to a second pair of buffers
+    // (fp16 [2][C][LDK]) so that the raw q, k stay in the first, and the
+    // tf32 diagonal factors of every sub-chunk fit at once (fp32
+    // [nsub][2][16][DK]).  The output phase of the three-phase schedule keeps
+    // the smaller layout, which fits two CTAs per SM.
+    static constexpr bool kMidSmem = MID && DK >= 128 && DV >= 128;
+    __host__ __device__ static size_t prep(int C) { return scratch(C) + scratch_bytes(C); }
+    __host__ __device__ static size_t fac(int C) { return prep(C) + (kMidSmem ? (size_t)2 * C * LDK * 2 : 0); }
+    __host__ __device__ static size_t block(int C) {
+        return (fac(C) + (kMidSmem ? (size_t)C * DK * 8 : 0) + 127) & ~(size_t)127;
+    }
     __host__ __device__ static size_t misc(int C) { return NCH * block(C); }  // tile index
     __host__ __device__ static size_t bytes(int C) { return misc(C) + 64; }
 };
@@ -180,9 +218,9 @@ struct TcLayout {
 // through shared memory, so only every NCH-th chunk boundary goes through L2.
 
 template <int DK, int DV, int MODE, int NCH>
-__global__ void __launch_bounds__(TcLayout<DK, DV, NCH>::NT)
+__global__ void __launch_bounds__(TcLayout<DK, DV, NCH, MODE == TC_FUSED>::NT)
 gla_tc_kernel(const TcArgs args) {
-    using Lay = TcLayout<DK, DV, NCH>;
+    using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
     constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
     static_assert(NCH == 1 || MODE == TC_FUSED, "multi-chunk tiles are for the fused schedule");
@@ -209,6 +247,14 @@ gla_tc_kernel(const TcArgs args) {
     auto Row_ = [&](int i) { return reinterpret_cast<int64_t *>(blk(i) + Lay::row(C)); };  // (b*N + p)*heads + h, or -1
     auto Fl_ = [&](int i) { return reinterpret_cast<int *>(blk(i) + Lay::flags(C)); };
     auto Scr_ = [&](int i) { return blk(i) + Lay::scratch(C); };
+    auto Fac_ = [&](int i) { return reinterpret_cast<float *>(blk(i) + Lay::fac(C)); };  // kMidSmem: tf32 factors
+    // the prepared operands qs, ke: over the raw q, k, or (kMidSmem) beside them
+    auto QP_ = [&](int i) {
+        return Lay::kMidSmem ? reinterpret_cast<__half *>(blk(i) + Lay::prep(C)) : Q_(i);
+    };
+    auto KP_ = [&](int i) {
+        return Lay::kMidSmem ? reinterpret_cast<__half *>(blk(i) + Lay::prep(C)) + C * LDK : K_(i);
+    };
 
     // ------------------------------------------------ which tile
     const int nseq = geo.B * geo.heads;
@@ -264,7 +310,9 @@ gla_tc_kernel(const TcArgs args) {
     // Every row of the tile is requested at once (cp.async, 16 bytes per
     // request, rows past the sequence end zero-filled), so the whole tile is
     // in flight together; q and k land in the operand buffers and are turned
-    // into qs / ke in place, g lands in the scratch region.
+    // into qs / ke in place (d_k = d_v = 128: into the second pair of
+    // buffers, the raw tiles kept for the tf32 diagonal form), g lands in the
+    // scratch region.
     {
         constexpr int QCH = DK / 8, VCH = DV / 8, GCH = DK / 4;
         for (int idx = tid; idx < NCH * C * VCH; idx += NT) {
@@ -298,7 +346,8 @@ gla_tc_kernel(const TcArgs args) {
         const int i = part_of(task, (DK / 2) * nsub), rem = task - i * ((DK / 2) * nsub);
         const int dp = rem % (DK / 2), u = rem / (DK / 2);
         const int d0 = 2 * dp;
-        __half *sQ = Q_(i), *sK = K_(i);
+        const __half *sQ = Q_(i), *sK = K_(i);  // raw
+        __half *dQ = QP_(i), *dK = KP_(i);       // prepared
         const float *sG = reinterpret_cast<const float *>(Scr_(i));
         __half2 qv[16], kv[16];
         float2 av[16];
@@ -311,6 +360,7 @@ gla_tc_kernel(const TcArgs args) {
         }
         // forward: a_t = exp(g_t), P_t = prod a_0..a_t, qs_t = q~_t P_t
         float2 P = make_float2(1.f, 1.f), P7 = P;
+        float2 Pmn = P, Pmx = P;  // extremes of the prefixes (P_{-1} = 1 included)
         __half2 qmax = __float2half2_rn(0.f), kmax = qmax;
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -319,9 +369,11 @@ gla_tc_kernel(const TcArgs args) {
             P.x *= av[t].x;
             P.y *= av[t].y;
             if (t == 7) P7 = P;
+            Pmn = make_float2(fminf(Pmn.x, P.x), fminf(Pmn.y, P.y));
+            Pmx = make_float2(fmaxf(Pmx.x, P.x), fmaxf(Pmx.y, P.y));
             if (MODE != TC_SUMMARY) {
                 qmax = __hmax2(qmax, __habs2(qv[t]));
-                *reinterpret_cast<__half2 *>(sQ + (16 * u + t) * LDK + d0) =
+                *reinterpret_cast<__half2 *>(dQ + (16 * u + t) * LDK + d0) =
                     __hmul2(qv[t], __floats2half2_rn(P.x * qscale, P.y * qscale));
             }
         }
@@ -331,7 +383,7 @@ gla_tc_kernel(const TcArgs args) {
         for (int t = 15; t >= 0; --t) {
             if (t == 7) S7 = S;
             kmax = __hmax2(kmax, __habs2(kv[t]));
-            *reinterpret_cast<__half2 *>(sK + (16 * u + t) * LDK + d0) = __hmul2(kv[t], __floats2half2_rn(S.x, S.y));
+            *reinterpret_cast<__half2 *>(dK + (16 * u + t) * LDK + d0) = __hmul2(kv[t], __floats2half2_rn(S.x, S.y));
             S.x *= av[t].x;
             S.y *= av[t].y;
         }
@@ -341,7 +393,13 @@ gla_tc_kernel(const TcArgs args) {
             const float2 qm = __half22float2(qmax), km = __half22float2(kmax);
             const bool fast = P.x >= lo && P.y >= lo && P.x <= hi && P.y <= hi &&
                               fmaxf(qm.x, qm.y) * qscale <= kDiagMaxAbs && fmaxf(km.x, km.y) <= kDiagMaxAbs;
-            if (!fast) Fl_(i)[u] = 1;
+            // the tf32 form: every ratio of two prefixes (so every factor
+            // around token 7) within e^{+-kMidRange}
+            const float mlo = 1.8048513e-35f;  // e^-kMidRange
+            const bool mid = Pmn.x >= Pmx.x * mlo && Pmn.y >= Pmx.y * mlo && Pmx.x <= 3.0e35f &&
+                             Pmx.y <= 3.0e35f && fmaxf(qm.x, qm.y) * qscale <= kMidMaxAbs &&
+                             fmaxf(km.x, km.y) <= kMidMaxAbs;
+            if (!fast) atomicMax(&Fl_(i)[u], mid ? DIAG_TF32 : DIAG_EXACT);
             *reinterpret_cast<__half2 *>(Rp_(i) + u * DK + d0) =
                 __floats2half2_rn(P7.x > 0.f ? 1.f / P7.x : 0.f, P7.y > 0.f ? 1.f / P7.y : 0.f);
             *reinterpret_cast<__half2 *>(Rs_(i) + u * DK + d0) =
@@ -369,7 +427,7 @@ gla_tc_kernel(const TcArgs args) {
         for (int pr = warp; pr < NCH * nsub; pr += NCH * NW) {
             const int i = part_of(pr, nsub), u = pr - i * nsub;
             if (Fl_(i)[u]) continue;
-            const __half *sQ = Q_(i), *sK = K_(i), *sRp = Rp_(i), *sRs = Rs_(i);
+            const __half *sQ = QP_(i), *sK = KP_(i), *sRp = Rp_(i), *sRs = Rs_(i);
             float acc[2][4] = {};
 #pragma unroll
             for (int kk = 0; kk < DK / 16; ++kk) {
@@ -401,19 +459,124 @@ gla_tc_kernel(const TcArgs args) {
                 }
             }
         }
-        // Exact path, one flagged sub-chunk at a time by the whole CTA:
+        // tf32 form (DIAG_TF32), by the whole CTA, with beta the in-sub-chunk
+        // prefix sum of g*log2(e):
+        //   qf_t = q~_t 2^(beta_t - beta_7),  kf_s = k_s 2^(beta_7 - beta_s),
+        //   A = qf kf^T  (m16n8k8 tf32, fp32 accumulate).
+        // The factors (fp32 [sub-chunk][qf, kf][16][DK], columns XOR-swizzled
+        // by the row so that the fragment loads are free of bank conflicts)
+        // meet only inside fp32 range; pairs s > t, whose product may
+        // overflow, are dropped by the mask.
+        for (int i = 0; i < NCH; ++i) {
+            const int *fl = Fl_(i);
+            uint32_t mids = 0;  // the tf32 sub-chunks, 4 bits each, in order
+            int nm = 0;
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (u < nsub && fl[u] == DIAG_TF32) mids |= (uint32_t)u << (4 * nm++);
+            // with kMidSmem every tf32 sub-chunk at once, from the raw q, k
+            // and the staged g still in shared memory; else two at a time in
+            // the scratch region, from the raw operands in global memory
+            constexpr int kGroup = Lay::kMidSmem ? 4 : 2;
+            float *xf = Lay::kMidSmem ? Fac_(i) : reinterpret_cast<float *>(Scr_(i));
+            const int64_t *sRow = Row_(i);
+            __half *sA = A_(i);
+            auto xsw = [](int row) { return (4 * row) & 28 & (DK - 1); };
+            for (int m0 = 0; m0 < nm; m0 += kGroup) {
+                const int gcnt = min(kGroup, nm - m0);
+                if constexpr (Lay::kMidSmem) {
+                    const __half *rq = Q_(i), *rk = K_(i);  // raw q, k (kept beside qs, ke)
+                    const float *sG = reinterpret_cast<const float *>(Scr_(i));
+                    for (int task = tid; task < gcnt * DK; task += NT) {
+                        const int sl = task / DK, d = task - sl * DK;
+                        const int u = (mids >> (4 * (m0 + sl))) & 15;
+                        float bv[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) bv[t] = sG[(16 * u + t) * DK + d] * kLog2e;
+#pragma unroll
+                        for (int t = 1; t < 16; ++t) bv[t] += bv[t - 1];
+                        float *xq = xf + sl * (32 * DK), *xk = xq + 16 * DK;
+#pragma unroll 4
+                        for (int t = 0; t < 16; ++t) {
+                            const int row = 16 * u + t, cs = d ^ xsw(t);
+                            xq[t * DK + cs] = __half2float(rq[row * LDK + d]) * qscale * ex2(bv[t] - bv[7]);
+                            xk[t * DK + cs] = __half2float(rk[row * LDK + d]) * ex2(bv[7] - bv[t]);
+                        }
+                    }
+                } else {
+                    for (int task = tid; task < gcnt * DK; task += NT) {
+                        const int sl = task / DK, d = task - sl * DK;
+                        const int u = (mids >> (4 * (m0 + sl))) & 15;
+                        const int64_t *rw = sRow + 16 * u;
+                        auto off = [&](int t) {
+                            const int64_t r = rw[t];
+                            const int64_t o = (r < 0 ? 0 : r) * DK + d;
+                            return (r >= 0 && GTR_INB(o, rows * DK, BS_TC_EXACT)) ? o : (int64_t)-1;
+                        };
+                        // beta: the 16 g loads in flight together, then the prefix
+                        float bv[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            const int64_t o = off(t);
+                            bv[t] = o >= 0 ? args.g[o] * kLog2e : 0.f;
+                        }
+#pragma unroll
+                        for (int t = 1; t < 16; ++t) bv[t] += bv[t - 1];
+                        float *xq = xf + sl * (32 * DK), *xk = xq + 16 * DK;
+#pragma unroll 4
+                        for (int t = 0; t < 16; ++t) {
+                            const int64_t o = off(t);
+                            const float qv = o >= 0 ? __half2float(args.q[o]) : 0.f;
+                            const float kv = o >= 0 ? __half2float(args.k[o]) : 0.f;
+                            const int cs = d ^ xsw(t);
+                            xq[t * DK + cs] = qv * qscale * ex2(bv[t] - bv[7]);
+                            xk[t * DK + cs] = kv * ex2(bv[7] - bv[t]);
+                        }
+                    }
+                }
+                __syncthreads();
+                // job j (one warp each): sub-chunk m0 + (j >> 1), key columns 8 (j & 1) .. + 7
+                for (int job = warp; job < 2 * gcnt; job += NCH * NW) {
+                    const int sl = job >> 1, n0 = 8 * (job & 1);
+                    const float *xq = xf + sl * (32 * DK), *xk = xq + 16 * DK;
+                    const int g8 = lane >> 2, t4 = lane & 3;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                    for (int k0 = 0; k0 < DK; k0 += 8) {
+                        uint32_t af[4];
+                        af[0] = to_tf32(xq[g8 * DK + ((k0 + t4) ^ xsw(g8))]);
+                        af[1] = to_tf32(xq[(g8 + 8) * DK + ((k0 + t4) ^ xsw(g8 + 8))]);
+                        af[2] = to_tf32(xq[g8 * DK + ((k0 + t4 + 4) ^ xsw(g8))]);
+                        af[3] = to_tf32(xq[(g8 + 8) * DK + ((k0 + t4 + 4) ^ xsw(g8 + 8))]);
+                        const uint32_t b0 = to_tf32(xk[(n0 + g8) * DK + ((k0 + t4) ^ xsw(n0 + g8))]);
+                        const uint32_t b1 = to_tf32(xk[(n0 + g8) * DK + ((k0 + t4 + 4) ^ xsw(n0 + g8))]);
+                        mma1688_tf32(acc, af, b0, b1);
+                    }
+                    __half *Au = sA + ((mids >> (4 * (m0 + sl))) & 15) * 16 * LDA;
+#pragma unroll
+                    for (int hlf = 0; hlf < 2; ++hlf) {
+                        const int t = g8 + 8 * hlf, s0i = n0 + 2 * t4;
+                        const float x0 = (s0i <= t) ? acc[2 * hlf] : 0.f;
+                        const float x1 = (s0i + 1 <= t) ? acc[2 * hlf + 1] : 0.f;
+                        *reinterpret_cast<uint32_t *>(Au + t * LDA + s0i) = pack_h2(x0, x1);
+                    }
+                }
+                __syncthreads();
+            }
+        }
+        // Exact path (DIAG_EXACT), one sub-chunk at a time by the whole CTA:
         // A_ts = sum_d q~_td k_sd 2^(beta_td - beta_sd) with beta the in-sub-chunk
         // prefix sum of g*log2(e), from the raw operands.
         for (int i = 0; i < NCH; ++i) {
             int *fl = Fl_(i);
-            if (!(fl[0] | fl[1] | fl[2] | fl[3])) continue;
+            if (!((fl[0] | fl[1] | fl[2] | fl[3]) & DIAG_EXACT)) continue;
             __half *xq = reinterpret_cast<__half *>(Scr_(i));
             __half *xk = xq + 16 * DK;
             float *xb = reinterpret_cast<float *>(xk + 16 * DK);
             const int64_t *sRow = Row_(i);
             __half *sA = A_(i);
             for (int u = 0; u < nsub; ++u) {
-                if (!fl[u]) continue;
+                if (fl[u] != DIAG_EXACT) continue;
                 for (int idx = tid; idx < 16 * DK; idx += NT) {
                     const int t = idx / DK, d = idx - t * DK;
                     const int64_t r = sRow[16 * u + t];
@@ -453,7 +616,7 @@ gla_tc_kernel(const TcArgs args) {
     // Warp (ch, wl) owns value columns [16wl, 16wl+16) of chunk ch.  L^T
     // (16 x DK) lives in the accumulator layout: Lt[n][0..3] covers key
     // columns 8n..8n+7.
-    const __half *sQ = Q_(ch), *sK = K_(ch), *sV = V_(ch), *sA = A_(ch), *sEb = Eb_(ch);
+    const __half *sQ = QP_(ch), *sK = KP_(ch), *sV = V_(ch), *sA = A_(ch), *sEb = Eb_(ch);
     const float *sGu = Gu_(ch), *sGc = Gc_(ch);
     const int v0 = 16 * wl;
     const int c = c0 + ch;
@@ -682,7 +845,7 @@ gla_tc_kernel(const TcArgs args) {
 // Launch helper used by the per-d_k translation units.
 template <int DK, int DV, int MODE, int NCH>
 cudaError_t launch_tc_mode(const TcArgs &a, cudaStream_t st) {
-    using Lay = TcLayout<DK, DV, NCH>;
+    using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
     const size_t smem = Lay::bytes(a.geo.chunk);
     cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel<DK, DV, MODE, NCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -63,15 +63,35 @@ def test_checked_build_odd_shapes(clib, oracle_mod, schedule, dk, dv, chunk):
 
 
 @pytest.mark.parametrize("schedule", ["auto", "fused", "fused_tcgen05"])
-def test_checked_build_exact_paths(clib, oracle_mod, schedule):
-    """Strong gates and large queries send the fused kernels down their exact
-    score paths, which read the raw operands again."""
+@pytest.mark.parametrize("gates", ["strong", "deep"])
+def test_checked_build_exact_paths(clib, oracle_mod, schedule, gates):
+    """Strong gates and large queries send the kernels down the paths that
+    read the raw operands again: the mma.sync kernel's tf32 diagonal form
+    (strong) and its per-pair exponentials (deep: a few gates of -150 nats,
+    beyond fp32 factors), the tcgen05 kernels' exact score path (both)."""
     H, W, heads = 9, 15, 2
     q, k, v, g = make_inputs(1, H, W, heads, 64, 64, seed=31, gate="strong")
     q = torch.where(torch.rand(q.shape[:3])[..., None] < 0.05, q.float() * 300.0, q.float()).half()
+    if gates == "deep":
+        g = torch.where(torch.rand(g.shape) < 0.1, torch.full_like(g, -150.0), g)
     dq, dk_, dvv, dg = (x.cuda() for x in (q, k, v, g))
     for direction in range(4):
         out = run_checked(clib, dq, dk_, dvv, dg, H, W, direction, 64, schedule)
+        assert_no_skips(clib)
+        compare(out.cpu(), oracle_mod.gla_serial(q, k, v, g, H, W, direction))
+
+
+@pytest.mark.parametrize("gates", ["strong", "deep"])
+def test_checked_build_tf32_diagonal_d128(clib, oracle_mod, gates):
+    """d_k = d_v = 128 on the fused mma.sync kernel: its tf32 diagonal form
+    reads the raw q, k kept in shared memory beside the prepared operands."""
+    H, W, heads = 9, 15, 2
+    q, k, v, g = make_inputs(1, H, W, heads, 128, 128, seed=53, gate="strong")
+    if gates == "deep":
+        g = torch.where(torch.rand(g.shape) < 0.1, torch.full_like(g, -150.0), g)
+    dq, dk_, dvv, dg = (x.cuda() for x in (q, k, v, g))
+    for direction in range(4):
+        out = run_checked(clib, dq, dk_, dvv, dg, H, W, direction, 64, "fused")
         assert_no_skips(clib)
         compare(out.cpu(), oracle_mod.gla_serial(q, k, v, g, H, W, direction))
 
