@@ -5,9 +5,42 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "gla_check.cuh"
 
 namespace gtr {
+
+// Programmatic dependent launch.  A grid launched with programmatic stream
+// serialization may start before the grid ahead of it in the stream has
+// finished: grid_dep_wait() blocks until that grid has completed and its
+// memory is visible (immediately for a normal launch), and must come before
+// any read of what it wrote; grid_dep_launch() lets the next such grid start.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
+// kern<<<grid, block, smem, st>>>(args...), with programmatic stream
+// serialization when `pdl` is set (only for kernels that call grid_dep_wait
+// before they read the previous grid's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                          Args &&...args) {
+    if (!pdl) {
+        kern<<<grid, block, smem, st>>>(std::forward<Args>(args)...);
+        return cudaGetLastError();
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Problem geometry shared by every kernel.  Token layout [B][N][heads][d],
 // N = H*W tokens in row-major spatial order.
@@ -55,8 +88,10 @@ cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, 
 // work for long chains and few state elements); agg holds scan_agg_bytes.
 int scan_segments(int64_t nseq, int nc, int dk, int dv);
 size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv);
+// pdl: launched with programmatic stream serialization (the scan waits for
+// the grid ahead of it before it reads dS).
 cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
-                                  float *S_enter, float *agg, cudaStream_t st);
+                                  float *S_enter, float *agg, cudaStream_t st, bool pdl = false);
 void count_launch(int n = 1);
 // Spatial SwiGLU gating with the fused 3x3 depthwise convolution (sswiglu.cu).
 cudaError_t launch_sswiglu(const __half *a, const __half *v, const float *wc, const float *bias, int B, int H, int W,

@@ -154,6 +154,10 @@ template <bool APPLY>
 __global__ void __launch_bounds__(kThreads) scan_seg_kernel(const float *dS, const float *__restrict__ gamma,
                                                             int nseq, int nc, int dk, int dv, int L, int nseg,
                                                             float *agg, float *S_enter) {
+    // launched programmatically after the summary (or pass 1): let the next
+    // grid start, then wait for the one ahead before reading its results
+    grid_dep_launch();
+    grid_dep_wait();
     const int n4 = dk * dv / 4;
     const int per = (n4 + blockDim.x - 1) / blockDim.x;
     const int segs = APPLY ? nseg : nseg - 1;
@@ -315,21 +319,20 @@ size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv) {
 }
 
 cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
-                                  float *S_enter, float *agg, cudaStream_t st) {
+                                  float *S_enter, float *agg, cudaStream_t st, bool pdl) {
     const int nseg = scan_segments(nseq, nc, dk, dv);
     const int L = (nc + nseg - 1) / nseg;
     const int64_t per = ((int64_t)dk * dv / 4 + kThreads - 1) / kThreads;
     if (nseg > 1) {
-        scan_seg_kernel<false><<<(unsigned)(nseq * (int64_t)(nseg - 1) * per), kThreads, 0, st>>>(
-            dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
+        cudaError_t e = launch_kernel(scan_seg_kernel<false>, dim3((unsigned)(nseq * (int64_t)(nseg - 1) * per)),
+                                      dim3(kThreads), 0, st, pdl, dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
         count_launch();
-        cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    scan_seg_kernel<true><<<(unsigned)(nseq * (int64_t)nseg * per), kThreads, 0, st>>>(dS, gamma, nseq, nc, dk, dv, L,
-                                                                                      nseg, agg, S_enter);
+    cudaError_t e = launch_kernel(scan_seg_kernel<true>, dim3((unsigned)(nseq * (int64_t)nseg * per)), dim3(kThreads),
+                                  0, st, pdl, dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, const float *g,

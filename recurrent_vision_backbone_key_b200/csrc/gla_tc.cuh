@@ -73,6 +73,7 @@ struct TcArgs {
     unsigned *status;      // FUSED: device status word (GTR_ERR_TIMEOUT on a give-up)
     long long spin_limit;  // FUSED: polls before a wait gives up
     int hold_seq, hold_chunk;  // FUSED test hook: this tile never publishes (-1: off)
+    bool pdl;              // host side: OUTPUT launched with programmatic stream serialization
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -221,6 +222,8 @@ template <int DK, int DV, int MODE, int NCH>
 __global__ void __launch_bounds__(TcLayout<DK, DV, NCH, MODE == TC_FUSED>::NT)
 gla_tc_kernel(const TcArgs args) {
     using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
+    // the summary lets a scan launched after it start (the scan waits for it)
+    if (MODE == TC_SUMMARY) grid_dep_launch();
     constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
     static_assert(NCH == 1 || MODE == TC_FUSED, "multi-chunk tiles are for the fused schedule");
@@ -697,6 +700,9 @@ gla_tc_kernel(const TcArgs args) {
     float Se[KT][4];
     bool have_state = c > 0;
     if (MODE == TC_OUTPUT) {
+        // everything above reads only q, k, v, g: with a programmatic launch
+        // it runs while the scan that writes S_enter finishes
+        grid_dep_wait();
         const float *src = args.S_enter + (GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SENTER) ? sdx : 0) * DK * DV;
         const int vr = v0 + (lane >> 2);
 #pragma unroll
@@ -852,9 +858,10 @@ cudaError_t launch_tc_mode(const TcArgs &a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int64_t groups = (a.geo.nc + NCH - 1) / NCH;
     const unsigned grid = (unsigned)(groups * a.geo.B * a.geo.heads);
-    gla_tc_kernel<DK, DV, MODE, NCH><<<grid, Lay::NT, smem, st>>>(a);
+    e = launch_kernel(gla_tc_kernel<DK, DV, MODE, NCH>, dim3(grid), dim3(Lay::NT), smem, st,
+                      MODE == TC_OUTPUT && a.pdl, a);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 // mode TC_FUSED_PAIR: the fused schedule with two chunks per tile (d_v <= 64).

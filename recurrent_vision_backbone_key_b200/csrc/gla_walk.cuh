@@ -101,6 +101,7 @@ struct WalkArgs {
     const void *gate;      // [B][N][heads][d_v] gate pre-activation (element type)
     const float *norm_w;   // [d_v] RMS-norm weight
     float norm_eps;
+    bool pdl;              // host side: OUTPUT launched with programmatic stream serialization
 };
 
 template <int DK>
@@ -312,6 +313,11 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         if (it < args.items) load_g(0, gnext);
     }
     (void)gnext;
+    // phase 3 reads S_enter, written by the scan: with a programmatic launch
+    // the loads above are in flight while the scan finishes; phase 1 lets the
+    // scan launched after it start (the scan waits for it)
+    if (MODE == WALK_OUTPUT) grid_dep_wait();
+    if (MODE == WALK_SUMMARY) grid_dep_launch();
     if (it < args.items) load_item_state(it, c);
 
     for (int step = 0; it < args.items; ++step) {
@@ -772,9 +778,10 @@ cudaError_t launch_walk_t(const WalkArgs &a, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    gla_walk_kernel<DK, MODE, GATED, T><<<grid, 128, L::ALLOC, st>>>(a);
+    e = launch_kernel(gla_walk_kernel<DK, MODE, GATED, T>, dim3(grid), dim3(128), L::ALLOC, st,
+                      MODE == WALK_OUTPUT && a.pdl, a);
     count_launch();
-    return cudaGetLastError();
+    return e;
 }
 
 // Launchers (gla_walk.cu): grid CTAs; `grid` <= a.items.  a.gate != null

@@ -209,6 +209,7 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
     a.dS = nullptr; a.gamma = nullptr; a.S_enter = nullptr; a.out = nullptr;
     a.ctrl = nullptr; a.ring = nullptr; a.status = nullptr;
     a.spin_limit = kSpinLimit; a.hold_seq = -1; a.hold_chunk = -1;
+    a.pdl = false;
     return a;
 }
 
@@ -358,11 +359,13 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
     return launch_tc(a, TC_SUMMARY, st);
 }
 
+// pdl: launched with programmatic stream serialization after the scan.
 cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const float *g,
                       const float *S_enter, const Geom &geo, __half *out, cudaStream_t st, unsigned *status,
-                      bool tcgen05 = true) {
+                      bool tcgen05 = true, bool pdl = false) {
     if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(q, k, v, g, geo, status);
+        a.pdl = pdl;
         a.S_enter = S_enter;
         a.out = out;
         a.items = geo.B * geo.heads * geo.nc * a.vs;
@@ -372,6 +375,7 @@ cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const f
         return launch_walk(a, WALK_OUTPUT, grid, st);
     }
     TcArgs a = make_args(q, k, v, g, geo);
+    a.pdl = pdl;
     a.S_enter = S_enter;
     a.out = out;
     return launch_tc(a, TC_OUTPUT, st);
@@ -395,9 +399,14 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
                                            align256(nseq * geo.nc * geo.dk * sizeof(float)));
-    e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st);
+    // the scan and the tensor-core output phase are launched programmatically:
+    // each starts while the grid ahead of it finishes and waits for it only
+    // where it reads that grid's results (the output phase after its loads
+    // and its within-chunk work)
+    e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st, true);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
-    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st) : output_tc(q, k, v, g, dS, geo, out, st, status, !mma);
+    e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st)
+             : output_tc(q, k, v, g, dS, geo, out, st, status, !mma, true);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
     return GTR_OK;
 }
