@@ -101,7 +101,7 @@ struct WalkArgs {
     const void *gate;      // [B][N][heads][d_v] gate pre-activation (element type)
     const float *norm_w;   // [d_v] RMS-norm weight
     float norm_eps;
-    bool pdl;              // host side: OUTPUT launched with programmatic stream serialization
+    bool pdl;              // host side: SEQ / OUTPUT launched with programmatic stream serialization
 };
 
 template <int DK>
@@ -303,6 +303,13 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     uint32_t ph1 = 0, ph2 = 0;
     bool mma_ok = true;
 
+    // the whole-sequence walk, launched programmatically: the set-up above
+    // overlaps the grid ahead of it, which it waits for before any access
+    // to global memory
+    if (MODE == WALK_SEQ) {
+        grid_dep_launch();
+        grid_dep_wait();
+    }
     int it = blockIdx.x, c = it < args.items ? first_chunk(it) : 0;
     int it1 = it, c1 = c;
     next_step(it1, c1);
@@ -779,7 +786,7 @@ cudaError_t launch_walk_t(const WalkArgs &a, int grid, cudaStream_t st) {
     e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     e = launch_kernel(gla_walk_kernel<DK, MODE, GATED, T>, dim3(grid), dim3(128), L::ALLOC, st,
-                      MODE == WALK_OUTPUT && a.pdl, a);
+                      (MODE == WALK_OUTPUT || MODE == WALK_SEQ) && a.pdl, a);
     count_launch();
     return e;
 }

@@ -307,6 +307,9 @@ gtr_status_t run_walk(const __half *q, const __half *k, const __half *v, const f
     a.norm_w = norm_w;
     a.norm_eps = norm_eps;
     a.items = geo.B * geo.heads * a.vs;
+    // launched programmatically: the kernel waits for the grid ahead of it
+    // before it touches global memory, so only its set-up overlaps that grid
+    a.pdl = true;
     cudaError_t e = launch_walk(a, WALK_SEQ, a.items, st, bf16);
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "walk kernel launch");
 }
