@@ -252,7 +252,10 @@ gtr_status_t gtr_gla_forward_noalloc(const void *q, const void *k, const void *v
  * GEMMs outside this library.  C must be a multiple of 8
  * (GTR_ERR_UNSUPPORTED_SHAPE); a, v and out 16-byte aligned, w and bias 4-byte
  * aligned (GTR_ERR_MISALIGNED); out must not overlap an input (GTR_ERR_ALIAS).
- * B == 0, an empty grid or C == 0 is an empty problem.  Needs no workspace. */
+ * B == 0, an empty grid or C == 0 is an empty problem.  Needs no workspace
+ * beyond the stream's device status word: a tile whose loads did not arrive
+ * within about a second is skipped and GTR_ERR_TIMEOUT is recorded there
+ * (gtr_gla_get_last_device_status). */
 gtr_status_t gtr_sswiglu_forward(const void *a, const void *v, const float *w, const float *bias, int B,
                                  int grid_h, int grid_w, int C, void *out, void *stream);
 

@@ -95,7 +95,7 @@ cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq,
 void count_launch(int n = 1);
 // Spatial SwiGLU gating with the fused 3x3 depthwise convolution (sswiglu.cu).
 cudaError_t launch_sswiglu(const __half *a, const __half *v, const float *wc, const float *bias, int B, int H, int W,
-                           int C, __half *y, cudaStream_t st);
+                           int C, __half *y, unsigned *status, cudaStream_t st);
 // Records the calling thread's failure text (returned by gtr_gla_last_error)
 // and returns s; clear_last_error empties it at the start of a call.
 int set_last_error(int s, const char *msg);

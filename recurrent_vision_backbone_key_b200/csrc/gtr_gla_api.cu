@@ -702,7 +702,7 @@ gtr_status_t gtr_sswiglu_forward(const void *a, const void *v, const float *w, c
     if (C % 8 != 0) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "C must be a multiple of 8%s");
     const int64_t N = (int64_t)grid_h * grid_w;
     if (N > ((int64_t)1 << 30)) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "more than 2^30 tokens%s");
-    if (B > 65535 || C / 64 + 1 > 65535) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "B or C too large%s");
+    if (B > 65535 || (C + 31) / 32 > 65535) return fail(GTR_ERR_UNSUPPORTED_SHAPE, "B or C too large%s");
     if (!a || !v || !w || !out) return fail(GTR_ERR_INVALID_ARG, "null pointer%s");
     if (!aligned16(a) || !aligned16(v) || !aligned16(out) || (reinterpret_cast<uintptr_t>(w) & 3u) ||
         (bias && (reinterpret_cast<uintptr_t>(bias) & 3u)))
@@ -713,8 +713,11 @@ gtr_status_t gtr_sswiglu_forward(const void *a, const void *v, const float *w, c
         (bias && overlap(ro, span(bias, (size_t)C * 4))))
         return fail(GTR_ERR_ALIAS, "out overlaps an input%s");
     if (B == 0 || N == 0 || C == 0) return GTR_OK;
+    unsigned *status = nullptr;
+    gtr_status_t s = status_word(static_cast<cudaStream_t>(stream), &status);
+    if (s != GTR_OK) return s;
     cudaError_t e = launch_sswiglu(static_cast<const __half *>(a), static_cast<const __half *>(v), w, bias, B, grid_h,
-                                   grid_w, C, static_cast<__half *>(out), static_cast<cudaStream_t>(stream));
+                                   grid_w, C, static_cast<__half *>(out), status, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? GTR_OK : cuda_fail(e, "S-SwiGLU kernel launch");
 }
 

@@ -7,49 +7,83 @@
 // SwiGLU").  a is the gate branch, v the value branch, both [B][H*W][C] fp16
 // in row-major spatial order; y likewise.
 //
-// HBM-bound (6 bytes per element): one CTA of 128 threads takes a tile of 8
-// grid rows x 16 grid columns x 64 channels.  The value tile with its one-token
-// halo (10 x 18 tokens x 128 bytes) and the gate tile (8 x 16 tokens) are
-// staged in shared memory by cp.async, all in flight at once, zero-filled
-// outside the grid, so the stencil needs no border tests.  Thread (column c,
-// channel octet j) keeps its 9 x 8 filter taps in registers and walks the
-// tile's 8 rows down its column with a 3 x 3 window of 16-byte vectors,
-// loading one new row of three per step; the output writes are 16-byte
-// vectors, 8 threads per 128-byte line.
+// HBM-bound (6 bytes per element), so the kernel is built to issue few
+// instructions per element and to keep many tiles' loads in flight.  A tile
+// is 8 grid rows x 16 grid columns x 32 channels.  Its value block with the
+// one-token halo (10 x 18 tokens x 64 bytes) and its gate block (8 x 16
+// tokens) are two TMA tile loads of 4-D tensor maps [B][H][W][C], issued by
+// one thread; the halo's cells outside the grid and channels past C read as
+// zero, so the stencil needs no border tests (the channel coordinate, the
+// innermost, is a multiple of 32: 64-byte aligned).  One CTA of 128 threads
+// per tile, five resident per SM (90 registers, 20 KB of shared memory).
+// Thread (column c, channel quad j) keeps its 9 x 4 filter taps in registers
+// and walks the tile's 8 rows down its column with a 3 x 3 window held in
+// fp32: each step loads one new row of three 8-byte vectors, converts it
+// once, and applies the nine taps with packed fp32x2 FMAs (two channels per
+// instruction, fp32 accumulation).
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "gla_common.cuh"
+#include "gla_tcgen05.cuh"
 
 namespace gtr {
 namespace {
 
-constexpr int kRows = 8, kCols = 16, kCh = 64;  // tile: grid rows, grid columns, channels
+constexpr int kRows = 8, kCols = 16, kCh = 32;  // tile: grid rows, grid columns, channels
 constexpr int kHr = kRows + 2, kHc = kCols + 2; // with the halo
-constexpr int kThreads = kCols * (kCh / 8);     // one thread per (column, channel octet)
+constexpr int kQuads = kCh / 4;                 // 8-byte channel quads per token
+constexpr int kThreads = kCols * kQuads;        // one thread per (column, channel quad)
 
-__device__ __forceinline__ void cp16(uint32_t saddr, const void *g, bool full) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(saddr), "l"(g), "r"(full ? 16 : 0));
+constexpr uint32_t kTileBytes = kHr * kHc * kCh * 2, kGateBytes = kRows * kCols * kCh * 2;
+
+// One 4-D TMA tile load (coordinates innermost first) completing on mbar.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int x, int y, int z, int w,
+                                            uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], "
+        "[%6];\n" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(mbar)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(mbar), "r"(bytes) : "memory");
 }
 
-__device__ __forceinline__ void acc_tap(float (&acc)[8], const float (&w)[8], uint4 x) {
-    const __half2 *h = reinterpret_cast<const __half2 *>(&x);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const float2 f = __half22float2(h[e]);
-        acc[2 * e] = fmaf(w[2 * e], f.x, acc[2 * e]);
-        acc[2 * e + 1] = fmaf(w[2 * e + 1], f.y, acc[2 * e + 1]);
-    }
+// d = a * b + c on two fp32 lanes at once.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;\n"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&d);
+}
+
+// Four fp16 channels (one 8-byte vector) as two fp32 pairs.
+struct Quad {
+    float2 lo, hi;
+};
+__device__ __forceinline__ Quad to_quad(uint2 x) {
+    Quad q;
+    q.lo = __half22float2(*reinterpret_cast<const __half2 *>(&x.x));
+    q.hi = __half22float2(*reinterpret_cast<const __half2 *>(&x.y));
+    return q;
 }
 
 __device__ __forceinline__ float silu(float x) { return __fdividef(x, 1.f + __expf(-x)); }
 
-__global__ void __launch_bounds__(kThreads) sswiglu_kernel(const __half *__restrict__ a, const __half *__restrict__ v,
-                                                           const float *__restrict__ wc, const float *__restrict__ bias,
-                                                           int B, int H, int W, int C, __half *__restrict__ y) {
-    __shared__ __align__(16) uint4 tile[kHr * kHc * (kCh / 8)];     // value branch with halo
-    __shared__ __align__(16) uint4 gtile[kRows * kCols * (kCh / 8)];  // gate branch
+__global__ void __launch_bounds__(kThreads)
+    sswiglu_kernel(const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_a,
+                   const float *__restrict__ wc, const float *__restrict__ bias, int B, int H, int W, int C,
+                   __half *__restrict__ y, unsigned *status) {
+    __shared__ __align__(128) uint2 tile[kHr * kHc * kQuads];     // value branch with halo
+    __shared__ __align__(128) uint2 gtile[kRows * kCols * kQuads];  // gate branch
+    __shared__ __align__(8) uint64_t bar;
     const int tid = threadIdx.x;
     const int c0 = blockIdx.y * kCh;
     const int tiles_w = (W + kCols - 1) / kCols;
@@ -57,48 +91,51 @@ __global__ void __launch_bounds__(kThreads) sswiglu_kernel(const __half *__restr
     const int b = blockIdx.z;
     const int64_t elems = (int64_t)B * H * W * C;
 
-    // ---- the value tile with its halo and the gate tile, zero outside the
-    // grid and past C, all copies in flight at once
-    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(tile);
-    for (int idx = tid; idx < kHr * kHc * (kCh / 8); idx += kThreads) {
-        const int j = idx & 7, cell = idx >> 3;
-        const int hr = cell / kHc, hc = cell - hr * kHc;
-        const int gr = r0 - 1 + hr, gc = col0 - 1 + hc, ch = c0 + 8 * j;
-        const int64_t o = (((int64_t)b * H + gr) * W + gc) * C + ch;
-        const bool ok = gr >= 0 && gr < H && gc >= 0 && gc < W && ch < C && GTR_INB(o + 7, elems, BS_SSWIGLU_LOAD);
-        cp16(sbase + idx * 16, v + (ok ? o : 0), ok);
+    // ---- the value block with its halo and the gate block, one TMA load each
+    const uint32_t mbar = (uint32_t)__cvta_generic_to_shared(&bar);
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+        mbar_expect_tx(mbar, kTileBytes + kGateBytes);
+        tma_load_4d((uint32_t)__cvta_generic_to_shared(tile), &map_v, c0, col0 - 1, r0 - 1, b, mbar);
+        tma_load_4d((uint32_t)__cvta_generic_to_shared(gtile), &map_a, c0, col0, r0, b, mbar);
     }
-    const uint32_t gbase = (uint32_t)__cvta_generic_to_shared(gtile);
-    for (int idx = tid; idx < kRows * kCols * (kCh / 8); idx += kThreads) {
-        const int j = idx & 7, cell = idx >> 3;
-        const int tr = cell / kCols, tcol = cell - tr * kCols;
-        const int gr = r0 + tr, gc = col0 + tcol, ch = c0 + 8 * j;
-        const int64_t o = (((int64_t)b * H + gr) * W + gc) * C + ch;
-        const bool ok = gr < H && gc < W && ch < C && GTR_INB(o + 7, elems, BS_SSWIGLU_LOAD);
-        cp16(gbase + idx * 16, a + (ok ? o : 0), ok);
-    }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    __syncthreads();  // the barrier is initialised before anyone waits on it
 
-    // ---- this thread's channel octet: 9 x 8 taps and the bias (while the tiles land)
-    const int j = tid & 7, tc = tid >> 3;
-    const int ch = c0 + 8 * j;
-    const bool ch_ok = ch < C;
-    float w[9][8], bs[8];
+    // ---- this thread's channel quad: 9 x 4 taps and the bias (while the tiles land)
+    const int j = tid % kQuads, tc = tid / kQuads;
+    const int ch = c0 + 4 * j;
+    const bool ch_ok = ch < C;  // C is a multiple of 8, so the whole quad
+    float2 w[9][2], bs[2];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const bool ok = ch_ok && GTR_INB((int64_t)(ch + e) * 9 + 8, (int64_t)C * 9, BS_SSWIGLU_W);
+    for (int h = 0; h < 2; ++h) {
+        float t0[9], t1[9];
+        const int e = ch + 2 * h;
+        const bool ok = ch_ok && GTR_INB((int64_t)(e + 1) * 9 + 8, (int64_t)C * 9, BS_SSWIGLU_W);
 #pragma unroll
-        for (int tap = 0; tap < 9; ++tap) w[tap][e] = ok ? __ldg(wc + (int64_t)(ch + e) * 9 + tap) : 0.f;
-        bs[e] = (ok && bias) ? __ldg(bias + ch + e) : 0.f;
+        for (int tap = 0; tap < 9; ++tap) {
+            t0[tap] = ok ? __ldg(wc + (int64_t)e * 9 + tap) : 0.f;
+            t1[tap] = ok ? __ldg(wc + (int64_t)(e + 1) * 9 + tap) : 0.f;
+        }
+#pragma unroll
+        for (int tap = 0; tap < 9; ++tap) w[tap][h] = make_float2(t0[tap], t1[tap]);
+        bs[h] = (ok && bias) ? make_float2(__ldg(bias + e), __ldg(bias + e + 1)) : make_float2(0.f, 0.f);
     }
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
-    __syncthreads();
+    // ---- the tiles have landed (a wait that gives up records a timeout,
+    // waits once more so that no copy is left writing into this CTA's shared
+    // memory, and skips the tile)
+    if (!mbar_wait(mbar, 0)) {
+        if (tid == 0) atomicOr(status, 6u);  // GTR_ERR_TIMEOUT
+        mbar_wait(mbar, 0);
+        return;
+    }
 
-    // ---- walk down column col0 + tc: window rows (i-1, i, i+1) x columns (tc-1, tc, tc+1) of the halo tile
+    // ---- walk down column col0 + tc: window rows (i-1, i, i+1) x columns
+    // (tc-1, tc, tc+1) of the halo block, in fp32
     const int gc = col0 + tc;
     if (gc >= W || !ch_ok) return;
-    auto at = [&](int hr, int hc) { return tile[(hr * kHc + hc) * 8 + j]; };
-    uint4 win[3][3];
+    auto at = [&](int hr, int hc) { return to_quad(tile[(hr * kHc + hc) * kQuads + j]); };
+    Quad win[3][3];
 #pragma unroll
     for (int dy = 0; dy < 2; ++dy)
 #pragma unroll
@@ -109,25 +146,21 @@ __global__ void __launch_bounds__(kThreads) sswiglu_kernel(const __half *__restr
         if (gr >= H) break;
 #pragma unroll
         for (int dx = 0; dx < 3; ++dx) win[2][dx] = at(i + 2, tc + dx);
-        float acc[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = bs[e];
+        float2 lo = bs[0], hi = bs[1];
 #pragma unroll
         for (int dy = 0; dy < 3; ++dy)
 #pragma unroll
-            for (int dx = 0; dx < 3; ++dx) acc_tap(acc, w[3 * dy + dx], win[dy][dx]);
-        const int64_t o = (((int64_t)b * H + gr) * W + gc) * C + ch;
-        if (GTR_INB(o + 7, elems, BS_SSWIGLU_OUT)) {
-            const uint4 av = gtile[(i * kCols + tc) * 8 + j];
-            const __half2 *ah = reinterpret_cast<const __half2 *>(&av);
-            uint4 out;
-            __half2 *oh = reinterpret_cast<__half2 *>(&out);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __half22float2(ah[e]);
-                oh[e] = __floats2half2_rn(silu(f.x) * acc[2 * e], silu(f.y) * acc[2 * e + 1]);
+            for (int dx = 0; dx < 3; ++dx) {
+                lo = ffma2(w[3 * dy + dx][0], win[dy][dx].lo, lo);
+                hi = ffma2(w[3 * dy + dx][1], win[dy][dx].hi, hi);
             }
-            __stcs(reinterpret_cast<uint4 *>(y + o), out);
+        const int64_t o = (((int64_t)b * H + gr) * W + gc) * C + ch;
+        if (GTR_INB(o + 3, elems, BS_SSWIGLU_OUT)) {
+            const Quad g = to_quad(gtile[(i * kCols + tc) * kQuads + j]);
+            uint2 out;
+            *reinterpret_cast<__half2 *>(&out.x) = __floats2half2_rn(silu(g.lo.x) * lo.x, silu(g.lo.y) * lo.y);
+            *reinterpret_cast<__half2 *>(&out.y) = __floats2half2_rn(silu(g.hi.x) * hi.x, silu(g.hi.y) * hi.y);
+            __stcs(reinterpret_cast<uint2 *>(y + o), out);
         }
 #pragma unroll
         for (int dx = 0; dx < 3; ++dx) {
@@ -137,14 +170,54 @@ __global__ void __launch_bounds__(kThreads) sswiglu_kernel(const __half *__restr
     }
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the driver entry point the runtime hands out
+// (no link-time dependency on the driver library); nullptr if unavailable.
+EncodeTiledFn encode_tiled() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Tensor map of a [B][H][W][C] fp16 tensor with a (box_c, box_w, box_h, 1)
+// box; cells outside the tensor read as zero.
+cudaError_t make_map(CUtensorMap *m, const __half *p, int B, int H, int W, int C, int box_c, int box_w, int box_h) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return cudaErrorNotSupported;
+    const cuuint64_t dims[4] = {(cuuint64_t)C, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
+    const cuuint32_t box[4] = {(cuuint32_t)box_c, (cuuint32_t)box_w, (cuuint32_t)box_h, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, const_cast<__half *>(p), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 cudaError_t launch_sswiglu(const __half *a, const __half *v, const float *wc, const float *bias, int B, int H, int W,
-                           int C, __half *y, cudaStream_t st) {
+                           int C, __half *y, unsigned *status, cudaStream_t st) {
     const int64_t tiles = (int64_t)((H + kRows - 1) / kRows) * ((W + kCols - 1) / kCols);
     if (tiles >= ((int64_t)1 << 31) || (C + kCh - 1) / kCh > 65535 || B > 65535) return cudaErrorInvalidConfiguration;
+    CUtensorMap mv, ma;
+    cudaError_t e = make_map(&mv, v, B, H, W, C, kCh, kHc, kHr);
+    if (e == cudaSuccess) e = make_map(&ma, a, B, H, W, C, kCh, kCols, kRows);
+    if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)tiles, (unsigned)((C + kCh - 1) / kCh), (unsigned)B);
-    sswiglu_kernel<<<grid, kThreads, 0, st>>>(a, v, wc, bias, B, H, W, C, y);
+    sswiglu_kernel<<<grid, kThreads, 0, st>>>(mv, ma, wc, bias, B, H, W, C, y, status);
     count_launch();
     return cudaGetLastError();
 }
