@@ -160,7 +160,15 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     const int64_t rows = (int64_t)geo.B * geo.N * geo.heads;  // token-head rows of every tensor
     const int DV = geo.dv;
     const float qscale = rsqrtf((float)DK);
-    const bool lane_on = DK >= 64 || lane < 16;  // lanes with key dimensions in the prep
+    // the prep's lane map: lane -> key-dimension pair (2 dpair, 2 dpair + 1)
+    // of each 64-column half, over TPL of the warp's 16 tokens from tb; at
+    // d_k = 32 (16 pairs) the two half-warps take 8 tokens each, so that
+    // every lane works
+    constexpr bool kSplit = DK == 32;
+    constexpr int TPL = kSplit ? 8 : 16;
+    const int dpair = kSplit ? (lane & 15) : lane;
+    const int tb = kSplit ? 8 * (lane >> 4) : 0;
+    const bool lane_on = DK >= 64 || kSplit || lane < 16;  // lanes with key dimensions in the prep
 
     // ---- the CTA's stream of chunk steps: (item, chunk)
     auto first_chunk = [&](int it) { return MODE == WALK_SEQ ? 0 : (it / args.vs) % geo.nc; };
@@ -236,18 +244,18 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         cp_async_commit();  // one group per step, empty past the end
     };
 
-    // g of one step into registers (d_k <= 64): lane l, key pair (2l, 2l+1)
-    // of each of this warp's 16 tokens; padding rows get g = 0 (a = 1)
-    auto load_g = [&](int stage, float2 (&gv)[16]) {
-        const int64_t *rowt = sRow + stage * 64 + 16 * warp;
+    // g of one step into registers (d_k <= 64): key pair (2 dpair, 2 dpair + 1)
+    // of this lane's TPL tokens; padding rows get g = 0 (a = 1)
+    auto load_g = [&](int stage, float2 (&gv)[TPL]) {
+        const int64_t *rowt = sRow + stage * 64 + 16 * warp + tb;
 #pragma unroll
-        for (int t = 0; t < 16; t += 2) {
+        for (int t = 0; t < TPL; t += 2) {
             const longlong2 rr = *reinterpret_cast<const longlong2 *>(rowt + t);
             const int64_t r2[2] = {rr.x, rr.y};
 #pragma unroll
             for (int u = 0; u < 2; ++u)
-                gv[t + u] = (lane_on && r2[u] >= 0 && GTR_INB(r2[u] * DK + 2 * lane + 1, rows * DK, BS_WALK_G))
-                                ? __ldcs(reinterpret_cast<const float2 *>(args.g + r2[u] * DK + 2 * lane))
+                gv[t + u] = (lane_on && r2[u] >= 0 && GTR_INB(r2[u] * DK + 2 * dpair + 1, rows * DK, BS_WALK_G))
+                                ? __ldcs(reinterpret_cast<const float2 *>(args.g + r2[u] * DK + 2 * dpair))
                                 : make_float2(0.f, 0.f);
         }
     };
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     next_step(it1, c1);
     issue_loads(it, c, 0);
     issue_loads(it1, c1, 1);
-    float2 gnext[16];
+    float2 gnext[TPL];
     if constexpr (!L::kGsmem) {
         if (it < args.items) load_g(0, gnext);
     }
@@ -338,10 +346,10 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
         next_step(itn, cn);
 
         // ---- a_t = exp(g_t) of this warp's 16 tokens; per-warp decay totals
-        float2 av[PPL][16];
+        float2 av[PPL][TPL];
         if constexpr (!L::kGsmem) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) av[0][t] = gnext[t];
+            for (int t = 0; t < TPL; ++t) av[0][t] = gnext[t];
             if (itn < args.items) load_g(s ^ 1, gnext);  // next step's g, consumed one step later
         }
         cp_async_wait_group<1>();  // this step's stage (the next one may still be in flight)
@@ -351,40 +359,47 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 #pragma unroll
             for (int p = 0; p < PPL; ++p)
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    av[p][t] = *reinterpret_cast<const float2 *>(sg + (16 * warp + t) * DK + 64 * p + 2 * lane);
+                for (int t = 0; t < TPL; ++t)
+                    av[p][t] = *reinterpret_cast<const float2 *>(sg + (16 * warp + tb + t) * DK + 64 * p + 2 * dpair);
         }
+        float2 oth[PPL];  // kSplit: the other half-warp's decay total over its 8 tokens
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
             float2 tot = make_float2(1.f, 1.f);
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
+            for (int t = 0; t < TPL; ++t) {
                 av[p][t] = make_float2(ex2(av[p][t].x * kLog2e), ex2(av[p][t].y * kLog2e));
                 tot.x *= av[p][t].x;
                 tot.y *= av[p][t].y;
             }
-            if (lane_on) *reinterpret_cast<float2 *>(sTot + warp * DK + 64 * p + 2 * lane) = tot;
+            if constexpr (kSplit) {
+                oth[p] = make_float2(__shfl_xor_sync(0xffffffffu, tot.x, 16), __shfl_xor_sync(0xffffffffu, tot.y, 16));
+                tot.x *= oth[p].x;
+                tot.y *= oth[p].y;
+            }
+            if (lane_on && (!kSplit || lane < 16))
+                *reinterpret_cast<float2 *>(sTot + warp * DK + 64 * p + 2 * dpair) = tot;
         }
         // ---- this lane's column pairs of the warp's 16 rows of q and k, read
         // once (all loads before any store), and the |q~| test
-        uint32_t ro[PPL][16];
-        T2 qv[PPL][16], kv[PPL][16];
+        uint32_t ro[PPL][TPL];
+        T2 qv[PPL][TPL], kv[PPL][TPL];
         float qm = 0.f;
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
             if (!lane_on) break;
-            const int dc = (2 * lane) & 63;
+            const int dc = (2 * dpair) & 63;
             const uint32_t cb = (uint32_t)p * 8192u + (uint32_t)(dc & 7) * 2u;
 #pragma unroll
-            for (int t = 0; t < 16; ++t) {
-                const int row = 16 * warp + t;
+            for (int t = 0; t < TPL; ++t) {
+                const int row = 16 * warp + tb + t;
                 ro[p][t] = cb + (uint32_t)row * 128u + (((uint32_t)(dc >> 3) ^ (uint32_t)(row & 7)) << 4);
             }
 #pragma unroll
-            for (int t = 0; t < 16; ++t) kv[p][t] = *reinterpret_cast<const T2 *>(base + sb + L::SK + ro[p][t]);
+            for (int t = 0; t < TPL; ++t) kv[p][t] = *reinterpret_cast<const T2 *>(base + sb + L::SK + ro[p][t]);
             if (kOut) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
+                for (int t = 0; t < TPL; ++t) {
                     qv[p][t] = *reinterpret_cast<const T2 *>(base + sb + L::SQ + ro[p][t]);
                     const float2 qf = IO::to_f2(qv[p][t]);
                     qm = fmaxf(qm, fmaxf(fabsf(qf.x), fabsf(qf.y)));
@@ -400,7 +415,7 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
             Eb[p] = Sb[p] = gam[p] = make_float2(1.f, 1.f);
-            const int d0 = 64 * p + 2 * lane;
+            const int d0 = 64 * p + 2 * dpair;
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 const float2 tw = lane_on ? *reinterpret_cast<const float2 *>(sTot + w * DK + d0) : make_float2(1.f, 1.f);
@@ -408,6 +423,10 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                 if (w > warp) { Sb[p].x *= tw.x; Sb[p].y *= tw.y; }
                 gam[p].x *= tw.x;
                 gam[p].y *= tw.y;
+            }
+            if constexpr (kSplit) {  // the other half-warp's tokens come before (lanes 16-31) or after
+                if (lane >= 16) { Eb[p].x *= oth[p].x; Eb[p].y *= oth[p].y; }
+                else { Sb[p].x *= oth[p].x; Sb[p].y *= oth[p].y; }
             }
         }
         // every warp covers every key dimension with the same products, so
@@ -423,12 +442,12 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 #pragma unroll
         for (int p = 0; p < PPL; ++p) {
             if (!lane_on) break;
-            const int d0 = 64 * p + 2 * lane;
+            const int d0 = 64 * p + 2 * dpair;
             if (kOut) {
                 float2 E = exact ? make_float2(Eb[p].x * qscale, Eb[p].y * qscale)
                                  : make_float2(Eb[p].x * (qscale / gam[p].x), Eb[p].y * (qscale / gam[p].y));
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
+                for (int t = 0; t < TPL; ++t) {
                     E.x *= av[p][t].x;
                     E.y *= av[p][t].y;
                     *reinterpret_cast<T2 *>(base + sb + L::SQ + ro[p][t]) = __hmul2(qv[p][t], IO::from_f2(E.x, E.y));
@@ -436,12 +455,12 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
             }
             float2 S = Sb[p];  // decay after token t to the chunk end
 #pragma unroll
-            for (int t = 15; t >= 0; --t) {
+            for (int t = TPL - 1; t >= 0; --t) {
                 *reinterpret_cast<T2 *>(base + sb + L::SK + ro[p][t]) = __hmul2(kv[p][t], IO::from_f2(S.x, S.y));
                 S.x *= av[p][t].x;
                 S.y *= av[p][t].y;
             }
-            if (warp == 0) *reinterpret_cast<float2 *>(sGam + d0) = gam[p];
+            if (warp == 0 && (!kSplit || lane < 16)) *reinterpret_cast<float2 *>(sGam + d0) = gam[p];
         }
 
         const bool have_state = MODE == WALK_OUTPUT || (MODE == WALK_SEQ && (c > 0 || args.S0 != nullptr));
