@@ -73,7 +73,7 @@ struct TcArgs {
     unsigned *status;      // FUSED: device status word (GTR_ERR_TIMEOUT on a give-up)
     long long spin_limit;  // FUSED: polls before a wait gives up
     int hold_seq, hold_chunk;  // FUSED test hook: this tile never publishes (-1: off)
-    bool pdl;              // host side: OUTPUT launched with programmatic stream serialization
+    bool pdl;              // host side: SUMMARY / OUTPUT launched with programmatic stream serialization
 };
 
 // ---------------------------------------------------------------- PTX helpers
@@ -222,8 +222,9 @@ template <int DK, int DV, int MODE, int NCH>
 __global__ void __launch_bounds__(TcLayout<DK, DV, NCH, MODE == TC_FUSED>::NT)
 gla_tc_kernel(const TcArgs args) {
     using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
-    // the summary lets a scan launched after it start (the scan waits for it)
-    if (MODE == TC_SUMMARY) grid_dep_launch();
+    // the phases let the grid launched after them start (that grid waits
+    // for this one before it reads what this one writes)
+    if (MODE != TC_FUSED) grid_dep_launch();
     constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
     static_assert(NCH == 1 || MODE == TC_FUSED, "multi-chunk tiles are for the fused schedule");
@@ -308,6 +309,11 @@ gla_tc_kernel(const TcArgs args) {
         Row_(i)[t] = r;
     }
     __syncthreads();
+
+    // a summary launched programmatically waits here for the grid ahead of
+    // it before any access to global memory (that grid may still produce k,
+    // v, g, or read the buffers this one writes)
+    if (MODE == TC_SUMMARY) grid_dep_wait();
 
     // ------------------------------------------------ S1: stage q, k, v, g; prepare qs / ke
     // Every row of the tile is requested at once (cp.async, 16 bytes per
@@ -859,7 +865,7 @@ cudaError_t launch_tc_mode(const TcArgs &a, cudaStream_t st) {
     const int64_t groups = (a.geo.nc + NCH - 1) / NCH;
     const unsigned grid = (unsigned)(groups * a.geo.B * a.geo.heads);
     e = launch_kernel(gla_tc_kernel<DK, DV, MODE, NCH>, dim3(grid), dim3(Lay::NT), smem, st,
-                      MODE == TC_OUTPUT && a.pdl, a);
+                      MODE != TC_FUSED && a.pdl, a);
     count_launch();
     return e;
 }

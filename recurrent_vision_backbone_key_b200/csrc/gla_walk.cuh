@@ -101,7 +101,7 @@ struct WalkArgs {
     const void *gate;      // [B][N][heads][d_v] gate pre-activation (element type)
     const float *norm_w;   // [d_v] RMS-norm weight
     float norm_eps;
-    bool pdl;              // host side: SEQ / OUTPUT launched with programmatic stream serialization
+    bool pdl;              // host side: launched with programmatic stream serialization
 };
 
 template <int DK>
@@ -311,13 +311,12 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     uint32_t ph1 = 0, ph2 = 0;
     bool mma_ok = true;
 
-    // the whole-sequence walk, launched programmatically: the set-up above
-    // overlaps the grid ahead of it, which it waits for before any access
-    // to global memory
-    if (MODE == WALK_SEQ) {
-        grid_dep_launch();
-        grid_dep_wait();
-    }
+    // launched programmatically, the set-up above overlaps the grid ahead of
+    // it; the whole-sequence walk and phase 1 wait for that grid before any
+    // access to global memory (phase 3 before it reads S_enter, below); the
+    // grid after this one may start at once
+    grid_dep_launch();
+    if (MODE != WALK_OUTPUT) grid_dep_wait();
     int it = blockIdx.x, c = it < args.items ? first_chunk(it) : 0;
     int it1 = it, c1 = c;
     next_step(it1, c1);
@@ -329,10 +328,8 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
     }
     (void)gnext;
     // phase 3 reads S_enter, written by the scan: with a programmatic launch
-    // the loads above are in flight while the scan finishes; phase 1 lets the
-    // scan launched after it start (the scan waits for it)
+    // the loads above are in flight while the scan finishes
     if (MODE == WALK_OUTPUT) grid_dep_wait();
-    if (MODE == WALK_SUMMARY) grid_dep_launch();
     if (it < args.items) load_item_state(it, c);
 
     for (int step = 0; it < args.items; ++step) {
@@ -805,7 +802,7 @@ cudaError_t launch_walk_t(const WalkArgs &a, int grid, cudaStream_t st) {
     e = cudaFuncSetAttribute(gla_walk_kernel<DK, MODE, GATED, T>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     e = launch_kernel(gla_walk_kernel<DK, MODE, GATED, T>, dim3(grid), dim3(128), L::ALLOC, st,
-                      (MODE == WALK_OUTPUT || MODE == WALK_SEQ) && a.pdl, a);
+                      a.pdl, a);
     count_launch();
     return e;
 }

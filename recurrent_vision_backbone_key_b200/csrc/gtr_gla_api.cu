@@ -344,10 +344,13 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
 
 // Phase 1 and phase 3 on tensor cores: the tcgen05 walk kernel in its
 // single-chunk modes for its shapes, the mma.sync kernel otherwise.
+// pdl: launched with programmatic stream serialization (the kernel waits for
+// the grid ahead of it before it touches global memory).
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
-                       float *gamma, cudaStream_t st, unsigned *status, bool tcgen05 = true) {
+                       float *gamma, cudaStream_t st, unsigned *status, bool tcgen05 = true, bool pdl = false) {
     if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(nullptr, k, v, g, geo, status);
+        a.pdl = pdl;
         a.dS = dS;
         a.gamma = gamma;
         a.items = geo.B * geo.heads * geo.nc * a.vs;
@@ -357,6 +360,7 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
         return launch_walk(a, WALK_SUMMARY, grid, st);
     }
     TcArgs a = make_args(nullptr, k, v, g, geo);
+    a.pdl = pdl;
     a.dS = dS;
     a.gamma = gamma;
     return launch_tc(a, TC_SUMMARY, st);
@@ -398,14 +402,15 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                              align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
     cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
-                         : summary_tc(k, v, g, geo, dS, gamma, st, status, !mma);
+                         : summary_tc(k, v, g, geo, dS, gamma, st, status, !mma, true);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
                                            align256(nseq * geo.nc * geo.dk * sizeof(float)));
-    // the scan and the tensor-core output phase are launched programmatically:
-    // each starts while the grid ahead of it finishes and waits for it only
-    // where it reads that grid's results (the output phase after its loads
-    // and its within-chunk work)
+    // the tensor-core phases and the scan are launched programmatically: each
+    // starts while the grid ahead of it finishes and waits for it where it
+    // first needs it (the summary before any access to global memory, the
+    // scan before it reads dS, the output phase after its loads and its
+    // within-chunk work, before it reads S_enter)
     e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st, true);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
     e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st)
