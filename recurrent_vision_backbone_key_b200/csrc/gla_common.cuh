@@ -92,6 +92,9 @@ size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv);
 // the grid ahead of it before it reads dS).
 cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
                                   float *S_enter, float *agg, cudaStream_t st, bool pdl = false);
+// The same with fp16 dS and S_enter (the running state stays fp32).
+cudaError_t launch_scan_segmented(const __half *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                                  __half *S_enter, float *agg, cudaStream_t st, bool pdl = false);
 void count_launch(int n = 1);
 // Spatial SwiGLU gating with the fused 3x3 depthwise convolution (sswiglu.cu).
 cudaError_t launch_sswiglu(const __half *a, const __half *v, const float *wc, const float *bias, int B, int H, int W,

@@ -150,10 +150,26 @@ __global__ void __launch_bounds__(kThreads) scan_simt_kernel(
 //     of segments 0..s-1, then the segment's chunks again, writing S_enter.
 // Pass 1 only reads dS; pass 2 reads each element before it writes it, so
 // S_enter may be dS.  Aggregates: [seq][nseg - 1][d_k*d_v (D) + d_k (Gam)].
-template <bool APPLY>
-__global__ void __launch_bounds__(kThreads) scan_seg_kernel(const float *dS, const float *__restrict__ gamma,
+// dS and S_enter are fp32 or fp16 (T); the running state and the aggregates
+// are fp32.
+__device__ __forceinline__ float4 load4(const float *p, int64_t i4) { return reinterpret_cast<const float4 *>(p)[i4]; }
+__device__ __forceinline__ float4 load4(const __half *p, int64_t i4) {
+    const uint2 u = reinterpret_cast<const uint2 *>(p)[i4];
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void store4(float *p, int64_t i4, float4 x) { reinterpret_cast<float4 *>(p)[i4] = x; }
+__device__ __forceinline__ void store4(__half *p, int64_t i4, float4 x) {
+    uint2 u;
+    *reinterpret_cast<__half2 *>(&u.x) = __floats2half2_rn(x.x, x.y);
+    *reinterpret_cast<__half2 *>(&u.y) = __floats2half2_rn(x.z, x.w);
+    reinterpret_cast<uint2 *>(p)[i4] = u;
+}
+template <bool APPLY, typename T>
+__global__ void __launch_bounds__(kThreads) scan_seg_kernel(const T *dS, const float *__restrict__ gamma,
                                                             int nseq, int nc, int dk, int dv, int L, int nseg,
-                                                            float *agg, float *S_enter) {
+                                                            float *agg, T *S_enter) {
     // launched programmatically after the summary (or pass 1): let the next
     // grid start, then wait for the one ahead before reading its results
     grid_dep_launch();
@@ -179,14 +195,13 @@ __global__ void __launch_bounds__(kThreads) scan_seg_kernel(const float *dS, con
             S = make_float4(fmaf(G, S.x, D.x), fmaf(G, S.y, D.y), fmaf(G, S.z, D.z), fmaf(G, S.w, D.w));
         }
     }
-    const float4 *src = reinterpret_cast<const float4 *>(dS) + seq * nc * (int64_t)n4 + e4;
-    float4 *dst = reinterpret_cast<float4 *>(S_enter) + seq * nc * (int64_t)n4 + e4;
+    const int64_t base4 = seq * nc * (int64_t)n4 + e4;  // element quad e4 of the sequence's chunk 0
     const float *gm = gamma + seq * nc * dk + i;
     float4 xs[kAhead];
     float as[kAhead];
 #pragma unroll
     for (int u = 0; u < kAhead; ++u) {
-        xs[u] = c0 + u < c1 ? src[(int64_t)(c0 + u) * n4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        xs[u] = c0 + u < c1 ? load4(dS, base4 + (int64_t)(c0 + u) * n4) : make_float4(0.f, 0.f, 0.f, 0.f);
         as[u] = c0 + u < c1 ? gm[(int64_t)(c0 + u) * dk] : 0.f;
     }
     float G = 1.f;
@@ -198,10 +213,10 @@ __global__ void __launch_bounds__(kThreads) scan_seg_kernel(const float *dS, con
                 const float4 x = xs[u];
                 const float a = as[u];
                 if (c + kAhead < c1) {  // chunk c + kAhead, read before anything writes it
-                    xs[u] = src[(int64_t)(c + kAhead) * n4];
+                    xs[u] = load4(dS, base4 + (int64_t)(c + kAhead) * n4);
                     as[u] = gm[(int64_t)(c + kAhead) * dk];
                 }
-                if (APPLY) dst[(int64_t)c * n4] = S;
+                if (APPLY) store4(S_enter, base4 + (int64_t)c * n4, S);
                 S = make_float4(fmaf(a, S.x, x.x), fmaf(a, S.y, x.y), fmaf(a, S.z, x.z), fmaf(a, S.w, x.w));
                 if (!APPLY) G *= a;
             }
@@ -318,21 +333,31 @@ size_t scan_agg_bytes(int64_t nseq, int nc, int dk, int dv) {
     return (size_t)nseq * (scan_segments(nseq, nc, dk, dv) - 1) * ((size_t)dk * dv + dk) * sizeof(float);
 }
 
-cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
-                                  float *S_enter, float *agg, cudaStream_t st, bool pdl) {
+template <typename T>
+cudaError_t launch_scan_segmented_t(const T *dS, const float *gamma, int nseq, int nc, int dk, int dv, T *S_enter,
+                                    float *agg, cudaStream_t st, bool pdl) {
     const int nseg = scan_segments(nseq, nc, dk, dv);
     const int L = (nc + nseg - 1) / nseg;
     const int64_t per = ((int64_t)dk * dv / 4 + kThreads - 1) / kThreads;
     if (nseg > 1) {
-        cudaError_t e = launch_kernel(scan_seg_kernel<false>, dim3((unsigned)(nseq * (int64_t)(nseg - 1) * per)),
+        cudaError_t e = launch_kernel(scan_seg_kernel<false, T>, dim3((unsigned)(nseq * (int64_t)(nseg - 1) * per)),
                                       dim3(kThreads), 0, st, pdl, dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
         count_launch();
         if (e != cudaSuccess) return e;
     }
-    cudaError_t e = launch_kernel(scan_seg_kernel<true>, dim3((unsigned)(nseq * (int64_t)nseg * per)), dim3(kThreads),
+    cudaError_t e = launch_kernel(scan_seg_kernel<true, T>, dim3((unsigned)(nseq * (int64_t)nseg * per)), dim3(kThreads),
                                   0, st, pdl, dS, gamma, nseq, nc, dk, dv, L, nseg, agg, S_enter);
     count_launch();
     return e;
+}
+
+cudaError_t launch_scan_segmented(const float *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                                  float *S_enter, float *agg, cudaStream_t st, bool pdl) {
+    return launch_scan_segmented_t(dS, gamma, nseq, nc, dk, dv, S_enter, agg, st, pdl);
+}
+cudaError_t launch_scan_segmented(const __half *dS, const float *gamma, int nseq, int nc, int dk, int dv,
+                                  __half *S_enter, float *agg, cudaStream_t st, bool pdl) {
+    return launch_scan_segmented_t(dS, gamma, nseq, nc, dk, dv, S_enter, agg, st, pdl);
 }
 
 cudaError_t launch_output_v0(const __half *q, const __half *k, const __half *v, const float *g,

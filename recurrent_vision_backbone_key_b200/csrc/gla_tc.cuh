@@ -67,6 +67,8 @@ struct TcArgs {
     float *dS;             // SUMMARY: [nseq][nc][dk][dv]
     float *gamma;          // SUMMARY: [nseq][nc][dk]
     const float *S_enter;  // OUTPUT:  [nseq][nc][dk][dv]
+    __half *dS_h;          // SUMMARY: dS in fp16 instead (when set)
+    const __half *S_enter_h;  // OUTPUT: S_enter in fp16 instead (when set)
     __half *out;           // OUTPUT / FUSED
     int *ctrl;             // FUSED: [0] ticket, [1] unused, then 4 flags per sequence; zeroed before each launch
     float *ring;           // FUSED: [nseq][2][dk*dv] fragment-ordered states
@@ -688,15 +690,27 @@ gla_tc_kernel(const TcArgs args) {
     if (MODE == TC_SUMMARY) {
         // dS_c[dk][dv] = L^T transposed; gamma_c
         if (!GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SUMMARY)) return;
-        float *dst = args.dS + sdx * DK * DV;
         const int vr = v0 + (lane >> 2);
+        if (args.dS_h) {
+            __half *dst = args.dS_h + sdx * DK * DV;
 #pragma unroll
-        for (int n = 0; n < KT; ++n) {
-            const int kcol = 8 * n + kc;
-            dst[(kcol)*DV + vr] = Lt[n][0];
-            dst[(kcol + 1) * DV + vr] = Lt[n][1];
-            dst[(kcol)*DV + vr + 8] = Lt[n][2];
-            dst[(kcol + 1) * DV + vr + 8] = Lt[n][3];
+            for (int n = 0; n < KT; ++n) {
+                const int kcol = 8 * n + kc;
+                dst[(kcol)*DV + vr] = __float2half_rn(Lt[n][0]);
+                dst[(kcol + 1) * DV + vr] = __float2half_rn(Lt[n][1]);
+                dst[(kcol)*DV + vr + 8] = __float2half_rn(Lt[n][2]);
+                dst[(kcol + 1) * DV + vr + 8] = __float2half_rn(Lt[n][3]);
+            }
+        } else {
+            float *dst = args.dS + sdx * DK * DV;
+#pragma unroll
+            for (int n = 0; n < KT; ++n) {
+                const int kcol = 8 * n + kc;
+                dst[(kcol)*DV + vr] = Lt[n][0];
+                dst[(kcol + 1) * DV + vr] = Lt[n][1];
+                dst[(kcol)*DV + vr + 8] = Lt[n][2];
+                dst[(kcol + 1) * DV + vr + 8] = Lt[n][3];
+            }
         }
         for (int d = tid; d < DK; d += NT) args.gamma[sdx * DK + d] = sGc[d];
         return;
@@ -709,15 +723,28 @@ gla_tc_kernel(const TcArgs args) {
         // everything above reads only q, k, v, g: with a programmatic launch
         // it runs while the scan that writes S_enter finishes
         grid_dep_wait();
-        const float *src = args.S_enter + (GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SENTER) ? sdx : 0) * DK * DV;
+        const int64_t so = (GTR_INB(sdx, (int64_t)nseq * geo.nc, BS_TC_SENTER) ? sdx : 0) * DK * DV;
         const int vr = v0 + (lane >> 2);
+        if (args.S_enter_h) {  // fp16 states: the readout's B fragments are fp16 anyway
+            const __half *src = args.S_enter_h + so;
 #pragma unroll
-        for (int n = 0; n < KT; ++n) {
-            const int kcol = 8 * n + kc;
-            Se[n][0] = src[kcol * DV + vr];
-            Se[n][1] = src[(kcol + 1) * DV + vr];
-            Se[n][2] = src[kcol * DV + vr + 8];
-            Se[n][3] = src[(kcol + 1) * DV + vr + 8];
+            for (int n = 0; n < KT; ++n) {
+                const int kcol = 8 * n + kc;
+                Se[n][0] = __half2float(src[kcol * DV + vr]);
+                Se[n][1] = __half2float(src[(kcol + 1) * DV + vr]);
+                Se[n][2] = __half2float(src[kcol * DV + vr + 8]);
+                Se[n][3] = __half2float(src[(kcol + 1) * DV + vr + 8]);
+            }
+        } else {
+            const float *src = args.S_enter + so;
+#pragma unroll
+            for (int n = 0; n < KT; ++n) {
+                const int kcol = 8 * n + kc;
+                Se[n][0] = src[kcol * DV + vr];
+                Se[n][1] = src[(kcol + 1) * DV + vr];
+                Se[n][2] = src[kcol * DV + vr + 8];
+                Se[n][3] = src[(kcol + 1) * DV + vr + 8];
+            }
         }
         have_state = true;
     } else {  // FUSED

@@ -207,6 +207,7 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
     TcArgs a;
     a.q = q; a.k = k; a.v = v; a.g = g; a.geo = geo;
     a.dS = nullptr; a.gamma = nullptr; a.S_enter = nullptr; a.out = nullptr;
+    a.dS_h = nullptr; a.S_enter_h = nullptr;
     a.ctrl = nullptr; a.ring = nullptr; a.status = nullptr;
     a.spin_limit = kSpinLimit; a.hold_seq = -1; a.hold_chunk = -1;
     a.pdl = false;
@@ -347,7 +348,8 @@ gtr_status_t run_fused(const __half *q, const __half *k, const __half *v, const 
 // pdl: launched with programmatic stream serialization (the kernel waits for
 // the grid ahead of it before it touches global memory).
 cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const Geom &geo, float *dS,
-                       float *gamma, cudaStream_t st, unsigned *status, bool tcgen05 = true, bool pdl = false) {
+                       float *gamma, cudaStream_t st, unsigned *status, bool tcgen05 = true, bool pdl = false,
+                       __half *dS_h = nullptr) {
     if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(nullptr, k, v, g, geo, status);
         a.pdl = pdl;
@@ -362,6 +364,7 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
     TcArgs a = make_args(nullptr, k, v, g, geo);
     a.pdl = pdl;
     a.dS = dS;
+    a.dS_h = dS_h;
     a.gamma = gamma;
     return launch_tc(a, TC_SUMMARY, st);
 }
@@ -369,7 +372,7 @@ cudaError_t summary_tc(const __half *k, const __half *v, const float *g, const G
 // pdl: launched with programmatic stream serialization after the scan.
 cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const float *g,
                       const float *S_enter, const Geom &geo, __half *out, cudaStream_t st, unsigned *status,
-                      bool tcgen05 = true, bool pdl = false) {
+                      bool tcgen05 = true, bool pdl = false, const __half *S_enter_h = nullptr) {
     if (tcgen05 && walk_shape(geo)) {
         WalkArgs a = make_walk_args(q, k, v, g, geo, status);
         a.pdl = pdl;
@@ -384,6 +387,7 @@ cudaError_t output_tc(const __half *q, const __half *k, const __half *v, const f
     TcArgs a = make_args(q, k, v, g, geo);
     a.pdl = pdl;
     a.S_enter = S_enter;
+    a.S_enter_h = S_enter_h;
     a.out = out;
     return launch_tc(a, TC_OUTPUT, st);
 }
@@ -401,8 +405,12 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     float *dS = static_cast<float *>(ws);
     float *gamma = reinterpret_cast<float *>(static_cast<char *>(ws) +
                                              align256(nseq * geo.nc * geo.dk * geo.dv * sizeof(float)));
+    // the mma.sync phases keep dS and S_enter in fp16 (the output phase's
+    // readout takes the entering state as fp16 tensor-core operands anyway;
+    // the scan's running state stays fp32): half the state traffic
+    __half *dSh = mma ? static_cast<__half *>(ws) : nullptr;
     cudaError_t e = simt ? launch_summary_v0(k, v, g, geo, dS, gamma, st)
-                         : summary_tc(k, v, g, geo, dS, gamma, st, status, !mma, true);
+                         : summary_tc(k, v, g, geo, dS, gamma, st, status, !mma, true, dSh);
     if (e != cudaSuccess) return cuda_fail(e, "chunk summary launch");
     float *agg = reinterpret_cast<float *>(reinterpret_cast<char *>(gamma) +
                                            align256(nseq * geo.nc * geo.dk * sizeof(float)));
@@ -411,10 +419,11 @@ gtr_status_t run_three_phase(const __half *q, const __half *k, const __half *v, 
     // first needs it (the summary before any access to global memory, the
     // scan before it reads dS, the output phase after its loads and its
     // within-chunk work, before it reads S_enter)
-    e = launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st, true);
+    e = mma ? launch_scan_segmented(dSh, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dSh, agg, st, true)
+            : launch_scan_segmented(dS, gamma, (int)nseq, geo.nc, geo.dk, geo.dv, dS, agg, st, true);
     if (e != cudaSuccess) return cuda_fail(e, "boundary scan launch");
     e = simt ? launch_output_v0(q, k, v, g, dS, geo, out, st)
-             : output_tc(q, k, v, g, dS, geo, out, st, status, !mma, true);
+             : output_tc(q, k, v, g, dS, geo, out, st, status, !mma, true, dSh);
     if (e != cudaSuccess) return cuda_fail(e, "chunk output launch");
     return GTR_OK;
 }
