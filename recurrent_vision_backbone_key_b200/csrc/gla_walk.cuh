@@ -81,6 +81,14 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 
 enum WalkMode : int { WALK_SEQ = 0, WALK_SUMMARY = 1, WALK_OUTPUT = 2 };
 
+// silu(x) = x * sigmoid(x), sigmoid(x) = 1/2 + tanh(x/2)/2 with the hardware
+// tanh approximation: one special-function operation.
+__device__ __forceinline__ float silu_tanh(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;\n" : "=f"(t) : "f"(0.5f * x));
+    return x * fmaf(0.5f, t, 0.5f);
+}
+
 // Largest total decay over a chunk (nats) for the whole-chunk tensor-core form.
 constexpr float kWalkChunkRange = 8.0f;
 
@@ -727,10 +735,10 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
                         const float2 w = __ldg(reinterpret_cast<const float2 *>(args.norm_w + col));
                         const float2 r0 = IO::to_f2(*reinterpret_cast<const T2 *>(base + L::SP + sw128(t, col)));
                         const float2 r1 = IO::to_f2(*reinterpret_cast<const T2 *>(base + L::SP + sw128(t + 8, col)));
-                        o[4 * n + 0] *= inv0 * w.x * __fdividef(r0.x, 1.f + __expf(-r0.x));
-                        o[4 * n + 1] *= inv0 * w.y * __fdividef(r0.y, 1.f + __expf(-r0.y));
-                        o[4 * n + 2] *= inv1 * w.x * __fdividef(r1.x, 1.f + __expf(-r1.x));
-                        o[4 * n + 3] *= inv1 * w.y * __fdividef(r1.y, 1.f + __expf(-r1.y));
+                        o[4 * n + 0] *= inv0 * w.x * silu_tanh(r0.x);
+                        o[4 * n + 1] *= inv0 * w.y * silu_tanh(r0.y);
+                        o[4 * n + 2] *= inv1 * w.x * silu_tanh(r1.x);
+                        o[4 * n + 3] *= inv1 * w.y * silu_tanh(r1.y);
                     }
                 }
 #pragma unroll
