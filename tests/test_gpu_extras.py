@@ -233,3 +233,44 @@ def test_deployment_shape_full_size_sampled(oracle_mod):
             sl = lambda x: x[b:b + 1, :, h:h + 1, :].cpu()
             compare(out[b:b + 1, :, h:h + 1, :], oracle_mod.gla_serial(sl(q), sl(k), sl(v), sl(g), w.grid_h,
                                                                        w.grid_w, 2), tol=tol)
+
+
+def _picks(B, heads, n, seed):
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0), (B - 1, heads - 1)}
+    while len(picks) < n:
+        picks.add((int(rng.integers(B)), int(rng.integers(heads))))
+    return sorted(picks)
+
+
+def test_bf16_batched_full_size_sampled(oracle_mod):
+    """bf16 I/O at the batched size (d = 64, the launch the bf16 bench line
+    times), L->R and T->B, 24 sampled sequences each."""
+    from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs
+    w = WORKLOADS["batched"]
+    q, k, v, g = make_workload_inputs(w, seed=6, device="cuda", dtype=torch.bfloat16)
+    out = torch.empty_like(v)
+    for direction in (0, 2):
+        gtr_gla.check(gtr_gla.gtr_gla_forward_bf16(q, k, v, g, w.B, w.heads, w.grid_h, w.grid_w, w.d_k, w.d_v,
+                                                   direction, 64, out))
+        torch.cuda.synchronize()
+        for b, h in _picks(w.B, w.heads, 24, seed=direction + 11):
+            sl = lambda x: x[b:b + 1, :, h:h + 1, :].cpu()
+            compare(out[b:b + 1, :, h:h + 1, :], oracle_mod.gla_serial(sl(q), sl(k), sl(v), sl(g), w.grid_h,
+                                                                       w.grid_w, direction), tol=BF16_TOL)
+
+
+def test_state_batched_full_size_sampled(oracle_mod):
+    """State in and out at the batched size (the launch the state bench line
+    times), T->B, 24 sampled sequences: outputs and final states."""
+    from recurrent_vision_backbone_key_b200.synthetic import WORKLOADS, make_workload_inputs
+    w = WORKLOADS["batched"]
+    q, k, v, g = make_workload_inputs(w, seed=8, device="cuda")
+    S0 = _state(w.B, w.heads, w.d_k, w.d_v, seed=9, scale=0.5)
+    out, SN = run_state(q, k, v, g, S0.cuda(), w.grid_h, w.grid_w, 2)
+    for b, h in _picks(w.B, w.heads, 24, seed=13):
+        sl = lambda x: x[b:b + 1, :, h:h + 1, :].cpu()
+        ref_out, ref_SN = oracle_mod.gla_serial_state(sl(q), sl(k), sl(v), sl(g), w.grid_h, w.grid_w, 2,
+                                                      S0[b:b + 1, h:h + 1].double().numpy())
+        compare(out[b:b + 1, :, h:h + 1, :], ref_out)
+        compare(SN[b:b + 1, h:h + 1], ref_SN)
