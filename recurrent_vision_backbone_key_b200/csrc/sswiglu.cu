@@ -14,15 +14,17 @@
 // tokens) are two TMA tile loads of 4-D tensor maps [B][H][W][C], issued by
 // one thread; the halo's cells outside the grid and channels past C read as
 // zero, so the stencil needs no border tests (the channel coordinate, the
-// innermost, is a multiple of 32: 64-byte aligned).  One CTA of 128 threads
-// per tile, five resident per SM (90 registers, 20 KB of shared memory).
-// Thread (column c, channel quad j) keeps its 9 x 4 filter taps in registers
-// and walks the tile's 8 rows down its column with a 3 x 3 window held in
-// fp32: each step loads one new row of three 8-byte vectors, converts it
-// once, and applies the nine taps with packed fp32x2 FMAs (two channels per
-// instruction, fp32 accumulation).  silu takes one special-function operation
-// (sigmoid as 1/2 + tanh(x/2)/2 with the hardware tanh approximation, whose
-// error is far inside the output's bar).
+// innermost, is a multiple of 32: 64-byte aligned).  One CTA of 64 threads
+// per tile, eight resident per SM (114 registers, 20 KB of shared memory).
+// Thread (column pair, channel quad j) keeps its 9 x 4 filter taps in
+// registers and walks the tile's 8 rows down its two columns with a 3 x 4
+// window held in fp32: each step loads one new row of four 8-byte vectors,
+// converts it once, and applies the nine taps to each column with packed
+// fp32x2 FMAs (two channels per instruction, fp32 accumulation).  Two
+// columns per thread halve the per-thread set-up (taps, addresses) per
+// output and share the window's middle columns.  silu takes one
+// special-function operation (sigmoid as 1/2 + tanh(x/2)/2 with the hardware
+// tanh approximation, whose error is far inside the output's bar).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -39,7 +41,7 @@ namespace {
 constexpr int kRows = 8, kCols = 16, kCh = 32;  // tile: grid rows, grid columns, channels
 constexpr int kHr = kRows + 2, kHc = kCols + 2; // with the halo
 constexpr int kQuads = kCh / 4;                 // 8-byte channel quads per token
-constexpr int kThreads = kCols * kQuads;        // one thread per (column, channel quad)
+constexpr int kThreads = kCols / 2 * kQuads;    // one thread per (column pair, channel quad)
 
 constexpr uint32_t kTileBytes = kHr * kHc * kCh * 2, kGateBytes = kRows * kCols * kCh * 2;
 
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(kThreads)
     __syncthreads();  // the barrier is initialised before anyone waits on it
 
     // ---- this thread's channel quad: 9 x 4 taps and the bias (while the tiles land)
-    const int j = tid % kQuads, tc = tid / kQuads;
+    const int j = tid % kQuads, tc = 2 * (tid / kQuads);  // first of the thread's two columns
     const int ch = c0 + 4 * j;
     const bool ch_ok = ch < C;  // C is a multiple of 8, so the whole quad
     float2 w[9][2], bs[2];
@@ -138,40 +140,44 @@ __global__ void __launch_bounds__(kThreads)
         return;
     }
 
-    // ---- walk down column col0 + tc: window rows (i-1, i, i+1) x columns
-    // (tc-1, tc, tc+1) of the halo block, in fp32
+    // ---- walk down columns col0 + tc and col0 + tc + 1: window rows
+    // (i-1, i, i+1) x columns (tc-1 .. tc+2) of the halo block, in fp32
     const int gc = col0 + tc;
     if (gc >= W || !ch_ok) return;
+    const bool two = gc + 1 < W;
     auto at = [&](int hr, int hc) { return to_quad(tile[(hr * kHc + hc) * kQuads + j]); };
-    Quad win[3][3];
+    Quad win[3][4];
 #pragma unroll
     for (int dy = 0; dy < 2; ++dy)
 #pragma unroll
-        for (int dx = 0; dx < 3; ++dx) win[dy][dx] = at(dy, tc + dx);
+        for (int dx = 0; dx < 4; ++dx) win[dy][dx] = at(dy, tc + dx);
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
         const int gr = r0 + i;
         if (gr >= H) break;
 #pragma unroll
-        for (int dx = 0; dx < 3; ++dx) win[2][dx] = at(i + 2, tc + dx);
-        float2 lo = bs[0], hi = bs[1];
+        for (int dx = 0; dx < 4; ++dx) win[2][dx] = at(i + 2, tc + dx);
 #pragma unroll
-        for (int dy = 0; dy < 3; ++dy)
+        for (int cc = 0; cc < 2; ++cc) {
+            float2 lo = bs[0], hi = bs[1];
 #pragma unroll
-            for (int dx = 0; dx < 3; ++dx) {
-                lo = ffma2(w[3 * dy + dx][0], win[dy][dx].lo, lo);
-                hi = ffma2(w[3 * dy + dx][1], win[dy][dx].hi, hi);
+            for (int dy = 0; dy < 3; ++dy)
+#pragma unroll
+                for (int dx = 0; dx < 3; ++dx) {
+                    lo = ffma2(w[3 * dy + dx][0], win[dy][dx + cc].lo, lo);
+                    hi = ffma2(w[3 * dy + dx][1], win[dy][dx + cc].hi, hi);
+                }
+            const int64_t o = (((int64_t)b * H + gr) * W + gc + cc) * C + ch;
+            if ((cc == 0 || two) && GTR_INB(o + 3, elems, BS_SSWIGLU_OUT)) {
+                const Quad g = to_quad(gtile[(i * kCols + tc + cc) * kQuads + j]);
+                uint2 out;
+                *reinterpret_cast<__half2 *>(&out.x) = __floats2half2_rn(silu(g.lo.x) * lo.x, silu(g.lo.y) * lo.y);
+                *reinterpret_cast<__half2 *>(&out.y) = __floats2half2_rn(silu(g.hi.x) * hi.x, silu(g.hi.y) * hi.y);
+                __stcs(reinterpret_cast<uint2 *>(y + o), out);
             }
-        const int64_t o = (((int64_t)b * H + gr) * W + gc) * C + ch;
-        if (GTR_INB(o + 3, elems, BS_SSWIGLU_OUT)) {
-            const Quad g = to_quad(gtile[(i * kCols + tc) * kQuads + j]);
-            uint2 out;
-            *reinterpret_cast<__half2 *>(&out.x) = __floats2half2_rn(silu(g.lo.x) * lo.x, silu(g.lo.y) * lo.y);
-            *reinterpret_cast<__half2 *>(&out.y) = __floats2half2_rn(silu(g.hi.x) * hi.x, silu(g.hi.y) * hi.y);
-            __stcs(reinterpret_cast<uint2 *>(y + o), out);
         }
 #pragma unroll
-        for (int dx = 0; dx < 3; ++dx) {
+        for (int dx = 0; dx < 4; ++dx) {
             win[0][dx] = win[1][dx];
             win[1][dx] = win[2][dx];
         }
