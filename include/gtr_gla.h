@@ -127,7 +127,16 @@ typedef enum {
  * it cannot).  Growing cannot be captured: a call that needs to grow it
  * inside a stream capture returns GTR_ERR_INVALID_ARG, so make the first call
  * of the largest size on that stream outside any capture.  After that, calls
- * on the stream can be captured into a CUDA graph and replayed. */
+ * on the stream can be captured into a CUDA graph and replayed.
+ * Stream order: some schedules (the walk, the three phases) launch their
+ * kernels with programmatic stream serialization.  Each such kernel waits for
+ * the kernel ahead of it on `stream` to complete before it touches q, k, v,
+ * g, out or the workspace, so the call is ordered after earlier work on the
+ * stream exactly as a normal launch is.  Each also lets the grid launched
+ * after it start early: a kernel the caller launches next with programmatic
+ * stream serialization must itself wait for its predecessor
+ * (cudaGridDependencySynchronize / griddepcontrol.wait) before it reads out,
+ * as that attribute requires anyway; a normal launch waits as usual. */
 gtr_status_t gtr_gla_forward(const void *q, const void *k, const void *v, const float *g,
                              int B, int heads, int grid_h, int grid_w, int d_k, int d_v,
                              int direction, int chunk, void *out, void *stream);
