@@ -224,9 +224,9 @@ template <int DK, int DV, int MODE, int NCH>
 __global__ void __launch_bounds__(TcLayout<DK, DV, NCH, MODE == TC_FUSED>::NT)
 gla_tc_kernel(const TcArgs args) {
     using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
-    // the phases let the grid launched after them start (that grid waits
-    // for this one before it reads what this one writes)
-    if (MODE != TC_FUSED) grid_dep_launch();
+    // the output phase lets the grid launched after it start at once (that
+    // grid waits for this one before it reads what this one writes); the
+    // summary does so only after its own wait, below
     constexpr int LDK = Lay::LDK, LDV = Lay::LDV, LDA = Lay::LDA, NT = Lay::NT, NW = Lay::NW;
     constexpr int KT = DK / 8;  // 8-wide key tiles of the state
     static_assert(NCH == 1 || MODE == TC_FUSED, "multi-chunk tiles are for the fused schedule");
@@ -316,6 +316,11 @@ gla_tc_kernel(const TcArgs args) {
     // it before any access to global memory (that grid may still produce k,
     // v, g, or read the buffers this one writes)
     if (MODE == TC_SUMMARY) grid_dep_wait();
+    // A grid launched after this one may start now.  The output phase (two
+    // launches on) reads q, k, v, g before it waits for its predecessor, so
+    // the first kernel of a call must not let the others start before
+    // everything ahead of the call is complete.
+    if (MODE != TC_FUSED) grid_dep_launch();
 
     // ------------------------------------------------ S1: stage q, k, v, g; prepare qs / ke
     // Every row of the tile is requested at once (cp.async, 16 bytes per

@@ -321,10 +321,12 @@ __global__ void __launch_bounds__(128, WalkLayout<DK>::MIN_CTAS) gla_walk_kernel
 
     // launched programmatically, the set-up above overlaps the grid ahead of
     // it; the whole-sequence walk and phase 1 wait for that grid before any
-    // access to global memory (phase 3 before it reads S_enter, below); the
-    // grid after this one may start at once
-    grid_dep_launch();
+    // access to global memory (phase 3 before it reads S_enter, below), and
+    // only then let the grid after this one start (phase 3 reads q, k, v, g
+    // before its wait, so nothing ahead of a call may still run when it
+    // starts)
     if (MODE != WALK_OUTPUT) grid_dep_wait();
+    grid_dep_launch();
     int it = blockIdx.x, c = it < args.items ? first_chunk(it) : 0;
     int it1 = it, c1 = c;
     next_step(it1, c1);

@@ -53,9 +53,12 @@ def test_forward_replayed_from_cuda_graph(oracle_mod, schedule):
     del graph
 
 
-def test_walk_after_a_producer_kernel(oracle_mod):
-    """The walk's inputs written by a kernel just ahead of it on the same
-    stream (the walk waits for that grid before it reads global memory)."""
+@pytest.mark.parametrize("schedule", ["walk_tcgen05", "three_phase_mma", "three_phase"])
+def test_forward_after_a_producer_kernel(oracle_mod, schedule):
+    """The forward's q written by a kernel just ahead of it on the same
+    stream: the first kernel of the call waits for that grid before it reads
+    global memory and lets the next one start only then (the output phase of
+    the three-phase schedules reads q before its own wait)."""
     B, H, W, heads, d = 4, 40, 40, 12, 64
     q, k, v, g = gpu_inputs(B, H, W, heads, d, d, seed=73)
     qn = torch.full_like(q, float("nan"))
@@ -64,7 +67,7 @@ def test_walk_after_a_producer_kernel(oracle_mod):
     for _ in range(3):
         qn.fill_(float("nan"))
         torch.mul(q, 1.0, out=qn)  # a kernel producing q immediately before the forward
-        gtr_gla.forward(qn, k, v, g, H, W, direction=0, schedule="walk_tcgen05", out=out, stream=st)
+        gtr_gla.forward(qn, k, v, g, H, W, direction=0, schedule=schedule, out=out, stream=st)
     torch.cuda.synchronize()
     ref = oracle_mod.gla_serial(q.cpu(), k.cpu(), v.cpu(), g.cpu(), H, W, 0)
     compare(out.cpu(), ref)
