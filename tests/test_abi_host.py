@@ -249,6 +249,9 @@ def test_sswiglu_entry_point_validates(lib):
     assert call(w=3 * A + 2) == 3
     assert call(out=A + 64) == 4
     assert call(out=3 * A) == 4
+    # grid limits of the launch: B along z, 32-channel groups along y
+    assert call(B=65536) == 2 and "too large" in lib.last_error()
+    assert call(C=65536 * 32 + 8) == 2
     before = lib.gtr_gla_launch_count()
     assert call(B=0) == 0 and call(grid_h=0) == 0 and call(C=0) == 0
     assert lib.gtr_gla_launch_count() == before
