@@ -165,7 +165,11 @@ __device__ __forceinline__ void st_release(int *p, int v) {
 // ------------------------------------------------------------ smem layout
 
 // One block of shared memory per chunk of the tile (NCH chunks per tile).
-template <int DK, int DV, int NCH, bool MID>
+// GDIRECT: g is read from global memory straight into registers by the
+// prep, not staged, and the tf32 diagonal factors are built one sub-chunk
+// at a time; the output phase at d_k = 64 takes this to fit five CTAs per
+// SM instead of four (43.6 KB against 52.8 KB at C = 64).
+template <int DK, int DV, int NCH, bool MID, bool GDIRECT = false>
 struct TcLayout {
     static constexpr int LDK = DK + 8;  // fp16 row stride (halves): 16-byte rows, conflict-free ldmatrix
     static constexpr int LDV = DV + 8;
@@ -184,14 +188,15 @@ struct TcLayout {
     __host__ __device__ static size_t gc(int C) { return eb(C) + (size_t)(C / 16) * DK * 2; }  // gamma_c
     __host__ __device__ static size_t row(int C) { return gc(C) + (size_t)DK * 4; }            // token-head row index
     __host__ __device__ static size_t flags(int C) { return row(C) + (size_t)C * 8; }          // exact-path sub-chunks
-    // scratch, used in turn for the staged g rows (fp32 [C][DK]), the exact
+    // scratch, used in turn for the staged g rows (fp32 [C][DK], unless
+    // GDIRECT), the tf32 diagonal factors, the exact
     // diagonal path's raw operands, the state handed from the first chunk of
     // a tile to the second, and the output staging
     __host__ __device__ static size_t scratch(int C) { return flags(C) + 64; }
     __host__ __device__ static size_t scratch_bytes(int C) {
-        size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8, gs = (size_t)C * DK * 4;
+        size_t o = (size_t)C * LDV * 2, e = (size_t)16 * DK * 8, gs = GDIRECT ? 0 : (size_t)C * DK * 4;
         size_t hs = NCH > 1 ? (size_t)DK * DV * 4 : 0;
-        size_t md = (size_t)(C >= 32 ? 2 : 1) * 32 * DK * 4;  // tf32 diagonal factors
+        size_t md = (size_t)(C >= 32 ? kMidGroup : 1) * 32 * DK * 4;  // tf32 diagonal factors
         size_t m = o > e ? o : e;
         m = m > gs ? m : gs;
         m = m > md ? m : md;
@@ -204,6 +209,9 @@ struct TcLayout {
     // [nsub][2][16][DK]).  The output phase of the three-phase schedule keeps
     // the smaller layout, which fits two CTAs per SM.
     static constexpr bool kMidSmem = MID && DK >= 128 && DV >= 128;
+    static constexpr bool kGDirect = GDIRECT;
+    // tf32 sub-chunks whose factors are built together
+    static constexpr int kMidGroup = kMidSmem ? 4 : (GDIRECT ? 1 : 2);
     __host__ __device__ static size_t prep(int C) { return scratch(C) + scratch_bytes(C); }
     __host__ __device__ static size_t fac(int C) { return prep(C) + (kMidSmem ? (size_t)2 * C * LDK * 2 : 0); }
     __host__ __device__ static size_t block(int C) {
@@ -212,6 +220,8 @@ struct TcLayout {
     __host__ __device__ static size_t misc(int C) { return NCH * block(C); }  // tile index
     __host__ __device__ static size_t bytes(int C) { return misc(C) + 64; }
 };
+template <int DK, int DV, int MODE, int NCH>
+using TcLayoutOf = TcLayout<DK, DV, NCH, MODE == TC_FUSED, MODE == TC_OUTPUT && DK == 64>;
 
 // --------------------------------------------------------------- the kernel
 //
@@ -221,9 +231,9 @@ struct TcLayout {
 // through shared memory, so only every NCH-th chunk boundary goes through L2.
 
 template <int DK, int DV, int MODE, int NCH>
-__global__ void __launch_bounds__(TcLayout<DK, DV, NCH, MODE == TC_FUSED>::NT)
+__global__ void __launch_bounds__(TcLayoutOf<DK, DV, MODE, NCH>::NT)
 gla_tc_kernel(const TcArgs args) {
-    using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
+    using Lay = TcLayoutOf<DK, DV, MODE, NCH>;
     // the output phase lets the grid launched after it start at once (that
     // grid waits for this one before it reads what this one writes); the
     // summary does so only after its own wait, below
@@ -328,7 +338,7 @@ gla_tc_kernel(const TcArgs args) {
     // in flight together; q and k land in the operand buffers and are turned
     // into qs / ke in place (d_k = d_v = 128: into the second pair of
     // buffers, the raw tiles kept for the tf32 diagonal form), g lands in the
-    // scratch region.
+    // scratch region (GDIRECT: g is read by the prep itself).
     {
         constexpr int QCH = DK / 8, VCH = DV / 8, GCH = DK / 4;
         for (int idx = tid; idx < NCH * C * VCH; idx += NT) {
@@ -347,7 +357,7 @@ gla_tc_kernel(const TcArgs args) {
             if (MODE != TC_SUMMARY) cp_async16(Q_(i) + t * LDK + j * 8, args.q + o, ok);
             cp_async16(K_(i) + t * LDK + j * 8, args.k + o, ok);
         }
-        for (int idx = tid; idx < NCH * C * GCH; idx += NT) {
+        for (int idx = tid; idx < (Lay::kGDirect ? 0 : NCH * C * GCH); idx += NT) {
             const int i = part_of(idx, C * GCH), rem = idx - i * (C * GCH);
             const int t = rem / GCH, j = rem - t * GCH;
             const int64_t r = Row_(i)[t];
@@ -372,7 +382,14 @@ gla_tc_kernel(const TcArgs args) {
             const int row = 16 * u + t;
             if (MODE != TC_SUMMARY) qv[t] = *reinterpret_cast<const __half2 *>(sQ + row * LDK + d0);
             kv[t] = *reinterpret_cast<const __half2 *>(sK + row * LDK + d0);
-            av[t] = *reinterpret_cast<const float2 *>(sG + row * DK + d0);
+            if constexpr (Lay::kGDirect) {
+                const int64_t r = Row_(i)[row];
+                av[t] = (r >= 0 && GTR_INB(r * DK + d0 + 1, rows * DK, BS_TC_LOAD))
+                            ? __ldg(reinterpret_cast<const float2 *>(args.g + r * DK + d0))
+                            : make_float2(0.f, 0.f);
+            } else {
+                av[t] = *reinterpret_cast<const float2 *>(sG + row * DK + d0);
+            }
         }
         // forward: a_t = exp(g_t), P_t = prod a_0..a_t, qs_t = q~_t P_t
         float2 P = make_float2(1.f, 1.f), P7 = P;
@@ -491,9 +508,10 @@ gla_tc_kernel(const TcArgs args) {
             for (int u = 0; u < 4; ++u)
                 if (u < nsub && fl[u] == DIAG_TF32) mids |= (uint32_t)u << (4 * nm++);
             // with kMidSmem every tf32 sub-chunk at once, from the raw q, k
-            // and the staged g still in shared memory; else two at a time in
-            // the scratch region, from the raw operands in global memory
-            constexpr int kGroup = Lay::kMidSmem ? 4 : 2;
+            // and the staged g still in shared memory; else kMidGroup (two,
+            // or one with GDIRECT) at a time in the scratch region, from the
+            // raw operands in global memory
+            constexpr int kGroup = Lay::kMidGroup;
             float *xf = Lay::kMidSmem ? Fac_(i) : reinterpret_cast<float *>(Scr_(i));
             const int64_t *sRow = Row_(i);
             __half *sA = A_(i);
@@ -889,7 +907,7 @@ gla_tc_kernel(const TcArgs args) {
 // Launch helper used by the per-d_k translation units.
 template <int DK, int DV, int MODE, int NCH>
 cudaError_t launch_tc_mode(const TcArgs &a, cudaStream_t st) {
-    using Lay = TcLayout<DK, DV, NCH, MODE == TC_FUSED>;
+    using Lay = TcLayoutOf<DK, DV, MODE, NCH>;
     const size_t smem = Lay::bytes(a.geo.chunk);
     cudaError_t e = cudaFuncSetAttribute(gla_tc_kernel<DK, DV, MODE, NCH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
