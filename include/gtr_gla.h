@@ -91,10 +91,10 @@ typedef enum {
                                        tcgen05 tensor cores for chunk 64, d_k in {32, 64, 128},
                                        d_v in {64, 128} (mma.sync for other shapes) */
     GTR_SCHED_THREE_PHASE_SIMT = 3, /* the same three phases on CUDA cores only (comparison) */
-    GTR_SCHED_FUSED_TCGEN05 = 4,    /* fused, one (sequence, chunk) tile per CTA with the boundary
-                                       state chained between CTAs, whole-chunk products on
-                                       tcgen05 (d_k = d_v = 64, chunk 64; other shapes run
-                                       GTR_SCHED_FUSED) */
+    GTR_SCHED_FUSED_TCGEN05 = 4,    /* fused, one (sequence, chunk, 64 value columns) tile per CTA
+                                       with the boundary state chained between CTAs, whole-chunk
+                                       products on tcgen05 (d_k = d_v in {64, 128}, chunk 64;
+                                       other shapes run GTR_SCHED_FUSED) */
     GTR_SCHED_WALK_TCGEN05 = 5,     /* one CTA per (sequence, 64 value columns) walks the chunks
                                        in scan order with its slice of the state on chip,
                                        whole-chunk products on tcgen05 (chunk 64, d_k in
@@ -111,7 +111,8 @@ typedef enum {
     GTR_PLAN_THREE_PHASE_SIMT = 1,  /* the same three phases on CUDA cores */
     GTR_PLAN_FUSED_MMA = 2,         /* fused mma.sync kernel, one chunk per tile */
     GTR_PLAN_FUSED_MMA_PAIR = 3,    /* fused mma.sync kernel, two chunks per tile (d_v <= 64) */
-    GTR_PLAN_FUSED_TCGEN05 = 4,     /* fused tcgen05 kernel, chained tiles (d_k = d_v = 64, chunk 64) */
+    GTR_PLAN_FUSED_TCGEN05 = 4,     /* fused tcgen05 kernel, chained tiles (d_k = d_v in {64, 128},
+                                       chunk 64) */
     GTR_PLAN_WALK_TCGEN05 = 5,      /* tcgen05 walk kernel, one CTA per (sequence, value slice) */
     GTR_PLAN_THREE_PHASE_MMA = 6    /* the three phases with mma.sync phases */
 } gtr_plan_t;

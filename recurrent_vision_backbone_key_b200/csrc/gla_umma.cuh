@@ -1,11 +1,11 @@
 // gla_umma.cuh -- fused GLA forward on the 5th-generation tensor cores
 // (tcgen05 MMAs from shared-memory descriptors into tensor memory) for
-// d_k = d_v = 64 and chunks of 64 tokens.
+// d_k = d_v in {64, 128} and chunks of 64 tokens.
 //
-// Same schedule as the fused mode of gla_tc.cuh (one (sequence, chunk) tile
-// per CTA, chunk-major tickets, boundary state chained through an L2 ring with
-// release/acquire flags, bounded waits), with the chunk's dense products done
-// as whole-chunk 64x64x64 MMAs:
+// Same schedule as the fused mode of gla_tc.cuh (one (sequence, chunk, 64
+// value columns) tile per CTA, chunk-major tickets, boundary state chained
+// through an L2 ring with release/acquire flags, bounded waits), with the
+// chunk's dense products done as whole-chunk M = 64 MMAs:
 //   with a_t = exp(g_t), E_t = a_0..a_t (decay since the chunk start),
 //   Suf_t = a_{t+1}..a_63 (decay to the chunk end), gamma_c = E_63:
 //     ke_s  = k_s Suf_s                       (<= |k|)
@@ -25,11 +25,15 @@
 // Operands live in shared memory as 64 x 64 fp16 row-major tiles with 128-byte
 // rows in the 128-byte swizzled canonical layout (16-byte chunk j of row r
 // stored at chunk j ^ (r mod 8)), read as K-major or MN-major by the MMA
-// descriptors.  Accumulators: with M = 64, row m of an accumulator sits in TMEM
-// lane (m mod 16) + 32 (m / 16) + base, base 0 or 16, so two of them share 64
-// columns: A (base 0) and dS^T (base 16) in one MMA pass, then O over A.
-// Warp w reads rows 16w..16w+15 of either with the 16x256b load, in the m16n8
-// accumulator-fragment layout.
+// descriptors; a 64 x 128 operand (q, k, S'^T at d_k = 128) is two such tiles,
+// key dims 0..63 then 64..127.  Accumulators: with M = 64, row m of an
+// accumulator sits in TMEM lane (m mod 16) + 32 (m / 16) + base, base 0 or 16,
+// so two of them share columns: A (base 0, 64 columns) and dS^T (base 16, d_k
+// columns) in one MMA pass, then O over A.  Warp w reads rows 16w..16w+15 of
+// either with the 16x256b load, in the m16n8 accumulator-fragment layout.
+// At d_k = 128 the two value halves of a chunk are two CTAs with adjacent
+// tickets: each preps the same q, k, g rows (the second read comes from L2)
+// and carries its own 128 x 64 slice of the state.
 #pragma once
 
 #include "gla_tc.cuh"
@@ -41,30 +45,37 @@ namespace gtr {
 constexpr float kChunkRange = 8.0f;
 
 // ---------------------------------------------------------------- layout
+template <int DK>
 struct UmmaLayout {
+    static constexpr uint32_t KTILE = DK * 128;  // a 64-row operand over all key dims (DK/64 tiles)
     // all offsets relative to a 1024-byte aligned base; every tile is swizzled
-    static constexpr uint32_t QH = 0;          // raw q, then the qh (or qe) tile in place
-    static constexpr uint32_t KE = 8192;       // raw k, then the ke tile in place; then S'^T
-    static constexpr uint32_t SP = KE;         // (scaled entering state)^T, rows = value columns,
-                                               // written once the summary MMA has read ke
-    static constexpr uint32_t V = 16384;       // v tile (also read as MN-major)
-    static constexpr uint32_t P = 24576;       // exact path's staging, then the masked scores,
-                                               // then the output staging
-    static constexpr uint32_t VEC = 32768;     // gamma_c[64], unused[64], sub-chunk totals [4][64] (fp32)
-    static constexpr uint32_t ROW = VEC + 6 * 64 * 4;  // int64 [64]
+    static constexpr uint32_t QH = 0;            // raw q, then the qh (or qe) tile in place
+    static constexpr uint32_t KE = KTILE;        // raw k, then the ke tile in place; then S'^T
+    static constexpr uint32_t SP = KE;           // (scaled entering state)^T, rows = value columns,
+                                                 // written once the summary MMA has read ke
+    static constexpr uint32_t V = 2 * KTILE;     // v tile, 64 value columns (also read as MN-major)
+    static constexpr uint32_t P = V + 8192;      // exact path's staging, then the masked scores,
+                                                 // then the output staging
+    static constexpr uint32_t VEC = P + 8192;    // gamma_c[DK], unused[DK], sub-chunk totals [4][DK] (fp32)
+    static constexpr uint32_t ROW = VEC + 6 * DK * 4;  // int64 [64]
     static constexpr uint32_t MISC = ROW + 64 * 8;     // tile, tmem base, mbarrier (8-aligned)
     static constexpr uint32_t BYTES = MISC + 64;
     static constexpr uint32_t ALLOC = BYTES + 1024;    // slack for aligning the base
+    static constexpr uint32_t TMEM_COLS = DK;          // dS^T is the widest accumulator
+    static constexpr int CTAS_PER_SM = DK == 64 ? 6 : 4;
 };
 
 // ---------------------------------------------------------------- the kernel
-// Chain of boundary states: warp w owns value rows 16w..16w+15 of S^T (its
-// TMEM lanes), and that slice of S_leave depends only on the same slice of
-// S_enter and of dS.  So each warp waits for, reads and publishes its own
-// slice, with one flag per (sequence, warp): no CTA barrier on the chain.
-__global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
-    using L = UmmaLayout;
-    constexpr int DK = 64, DV = 64, C = 64, KT = 8;
+// Chain of boundary states: warp w owns value rows 16w..16w+15 of the CTA's
+// slice of S^T (its TMEM lanes), and that slice of S_leave depends only on
+// the same slice of S_enter and of dS.  So each warp waits for, reads and
+// publishes its own slice, with one flag per (sequence, value half, warp): no
+// CTA barrier on the chain.
+template <int DK>
+__global__ void __launch_bounds__(128, UmmaLayout<DK>::CTAS_PER_SM) gla_umma_kernel(const TcArgs args) {
+    using L = UmmaLayout<DK>;
+    // DVC value columns per CTA, NVH CTAs per (sequence, chunk); d_v = d_k
+    constexpr int DVC = 64, NVH = DK / 64, DV = DK, C = 64, KT = DK / 8, NKA = DK / 64;
     extern __shared__ __align__(128) unsigned char smem_raw[];
     // 1024-byte aligned base (the swizzled operand tiles need it)
     const uint32_t raw_addr = smem_u32(smem_raw);
@@ -74,16 +85,18 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int tr = lane >> 2, kc = 2 * (lane & 3);
     float *vGc = reinterpret_cast<float *>(base + L::VEC);
-    float *vTot = vGc + 128;  // [4][64]
+    float *vTot = vGc + 2 * DK;  // [4][DK]
     int64_t *sRow = reinterpret_cast<int64_t *>(base + L::ROW);
     int *misc = reinterpret_cast<int *>(base + L::MISC);  // [0] tile [2] tmem base; mbar at +16
     const uint32_t mbar = base_addr + L::MISC + 16;
     const int nseq = geo.B * geo.heads;
+    const int nslot = nseq * NVH;  // chains: one per (sequence, value half)
     const int64_t rows = (int64_t)geo.B * geo.N * geo.heads;  // token-head rows of every tensor
 
     // ---- tensor memory first (before the ticket: a CTA waiting for TMEM holds no ticket)
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 64;\n" ::"r"(base_addr + L::MISC + 8)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(base_addr + L::MISC + 8),
+                     "r"(L::TMEM_COLS)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
     }
@@ -98,11 +111,13 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[2];
     const int tile = misc[0];
-    bool ok_tile = tile < geo.nc * nseq;
+    bool ok_tile = tile < geo.nc * nslot;
     if (!ok_tile && tid == 0) atomicOr(args.status, 6u);
 
-    const int c = ok_tile ? tile / nseq : 0;
-    const int seq = ok_tile ? tile - c * nseq : 0;
+    // chunk-major tickets; the value halves of a (sequence, chunk) adjacent
+    const int c = ok_tile ? tile / nslot : 0;
+    const int slot = ok_tile ? tile - c * nslot : 0;
+    const int seq = slot / NVH, vh = slot - seq * NVH;
     const int b = seq / geo.heads, h = seq - b * geo.heads;
     const int t0 = c * C;
     const int len = ok_tile ? min(C, geo.N - t0) : 0;
@@ -121,92 +136,119 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         }
         __syncwarp();
 
-        // ---- q, k, v rows into swizzled tiles (one cp.async batch per warp)
-        for (int idx = lane; idx < 16 * 8; idx += 32) {
-            const int t = 16 * warp + (idx >> 3), j = idx & 7;
+        // ---- q, k, v rows into swizzled tiles (one cp.async batch per warp);
+        // 16-byte piece j of a q / k row goes to key tile j / 8, pieces
+        // 0..7 of the CTA's 64 value columns to the v tile
+        constexpr int QP = DK / 8;  // 16-byte pieces of a q or k row
+        for (int idx = lane; idx < 16 * QP; idx += 32) {
+            const int t = 16 * warp + idx / QP, j = idx % QP;
             const int64_t r = sRow[t];
-            const bool ok = r >= 0 && GTR_INB(r * 64 + j * 8 + 7, rows * 64, BS_UMMA_QKV);
-            const int64_t o = ok ? r * 64 + j * 8 : 0;
-            const uint32_t so = t * 128 + (((j ^ (t & 7)) & 7) << 4);
+            const bool ok = r >= 0 && GTR_INB(r * DK + j * 8 + 7, rows * DK, BS_UMMA_QKV);
+            const int64_t o = ok ? r * DK + j * 8 : 0;
+            const uint32_t sw = ((((j & 7) ^ (t & 7)) & 7) << 4);
+            const uint32_t so = (j >> 3) * 8192 + t * 128 + sw;
             cp_async16(base + L::QH + so, args.q + o, ok);
             cp_async16(base + L::KE + so, args.k + o, ok);
-            cp_async16(base + L::V + so, args.v + o, ok);
+            if (j < 8) {
+                const bool okv = r >= 0 && GTR_INB(r * DV + vh * DVC + j * 8 + 7, rows * DV, BS_UMMA_QKV);
+                cp_async16(base + L::V + t * 128 + sw, args.v + (okv ? r * DV + vh * DVC + j * 8 : 0), okv);
+            }
         }
         cp_async_commit();
 
         // ---- g straight into registers: warp u takes sub-chunk u (tokens
-        // 16u..16u+15), lane dp the key dims (2dp, 2dp+1); one 256-byte row
-        // per warp load.  a_t = exp(g_t); padding rows get g = 0 (a = 1).
-        const int u = warp, d0 = 2 * lane;
-        float2 av[16];
+        // 16u..16u+15), lane dp the key dims 64p + (2dp, 2dp+1) of each
+        // 64-dim part p; one 256-byte row piece per warp load.  a_t = exp(g_t);
+        // padding rows get g = 0 (a = 1).
+        const int u = warp;
+        float2 av[NKA][16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            const int64_t r = sRow[16 * u + t];
-            av[t] = (r >= 0 && GTR_INB(r * 64 + d0 + 1, rows * 64, BS_UMMA_G))
-                        ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * 64 + d0))
-                        : make_float2(0.f, 0.f);
-        }
-        float2 tot = make_float2(1.f, 1.f);
+        for (int p = 0; p < NKA; ++p) {
+            const int d0 = 64 * p + 2 * lane;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) {
-            av[t] = make_float2(ex2(av[t].x * kLog2e), ex2(av[t].y * kLog2e));
-            tot.x *= av[t].x;
-            tot.y *= av[t].y;
+            for (int t = 0; t < 16; ++t) {
+                const int64_t r = sRow[16 * u + t];
+                av[p][t] = (r >= 0 && GTR_INB(r * DK + d0 + 1, rows * DK, BS_UMMA_G))
+                               ? __ldcs(reinterpret_cast<const float2 *>(args.g + r * DK + d0))
+                               : make_float2(0.f, 0.f);
+            }
         }
-        *reinterpret_cast<float2 *>(vTot + u * 64 + d0) = tot;
+#pragma unroll
+        for (int p = 0; p < NKA; ++p) {
+            float2 tot = make_float2(1.f, 1.f);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+                av[p][t] = make_float2(ex2(av[p][t].x * kLog2e), ex2(av[p][t].y * kLog2e));
+                tot.x *= av[p][t].x;
+                tot.y *= av[p][t].y;
+            }
+            *reinterpret_cast<float2 *>(vTot + u * DK + 64 * p + 2 * lane) = tot;
+        }
         cp_async_wait_all();
         __syncthreads();  // sub-chunk totals and the q, k, v tiles visible
 
-        float2 Ebase = make_float2(1.f, 1.f), Sbase = make_float2(1.f, 1.f), gam = make_float2(1.f, 1.f);
-#pragma unroll
-        for (int w = 0; w < 4; ++w) {
-            const float2 tw = *reinterpret_cast<const float2 *>(vTot + w * 64 + d0);
-            if (w < u) { Ebase.x *= tw.x; Ebase.y *= tw.y; }
-            if (w > u) { Sbase.x *= tw.x; Sbase.y *= tw.y; }
-            gam.x *= tw.x;
-            gam.y *= tw.y;
-        }
-        // Every warp covers all 64 key dims with the same products, so the
-        // vote is the same in every warp.
+        float2 Ebase[NKA], Sbase[NKA], gam[NKA];
+        bool in_range = true;
         const float lo = 3.3546263e-4f;  // e^-kChunkRange
-        const bool gam_ok = __all_sync(0xffffffffu, gam.x >= lo && gam.y >= lo && gam.x <= 1.f / lo &&
-                                                        gam.y <= 1.f / lo);
+#pragma unroll
+        for (int p = 0; p < NKA; ++p) {
+            const int d0 = 64 * p + 2 * lane;
+            Ebase[p] = Sbase[p] = gam[p] = make_float2(1.f, 1.f);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 tw = *reinterpret_cast<const float2 *>(vTot + w * DK + d0);
+                if (w < u) { Ebase[p].x *= tw.x; Ebase[p].y *= tw.y; }
+                if (w > u) { Sbase[p].x *= tw.x; Sbase[p].y *= tw.y; }
+                gam[p].x *= tw.x;
+                gam[p].y *= tw.y;
+            }
+            in_range = in_range && gam[p].x >= lo && gam[p].y >= lo && gam[p].x <= 1.f / lo && gam[p].y <= 1.f / lo;
+        }
+        // Every warp covers all key dims with the same products, so the vote
+        // is the same in every warp.
+        const bool gam_ok = __all_sync(0xffffffffu, in_range);
         // qh = q~ E_t / gamma_c (whole-chunk form) or qe = q~ E_t, in place
         __half2 qmax = __float2half2_rn(0.f);
-        {
+#pragma unroll
+        for (int p = 0; p < NKA; ++p) {
+            const int d0 = 2 * lane;  // inside key tile p
             // E_t / gamma_c * qscale (or E_t * qscale), carried as one product
-            float2 E = gam_ok ? make_float2(Ebase.x * (qscale / gam.x), Ebase.y * (qscale / gam.y))
-                              : make_float2(Ebase.x * qscale, Ebase.y * qscale);
+            float2 E = gam_ok ? make_float2(Ebase[p].x * (qscale / gam[p].x), Ebase[p].y * (qscale / gam[p].y))
+                              : make_float2(Ebase[p].x * qscale, Ebase[p].y * qscale);
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-                __half2 *p = reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0));
-                const __half2 qv = *p;
+                __half2 *pq = reinterpret_cast<__half2 *>(base + L::QH + p * 8192 + sw128(16 * u + t, d0));
+                const __half2 qv = *pq;
                 qmax = __hmax2(qmax, __habs2(qv));
-                E.x *= av[t].x;
-                E.y *= av[t].y;
-                *p = __hmul2(qv, __floats2half2_rn(E.x, E.y));
+                E.x *= av[p][t].x;
+                E.y *= av[p][t].y;
+                *pq = __hmul2(qv, __floats2half2_rn(E.x, E.y));
             }
-            float2 S = Sbase;  // decay after token t to the chunk end
+            float2 S = Sbase[p];  // decay after token t to the chunk end
 #pragma unroll
             for (int t = 15; t >= 0; --t) {
-                __half2 *p = reinterpret_cast<__half2 *>(base + L::KE + sw128(16 * u + t, d0));
-                *p = __hmul2(*p, __floats2half2_rn(S.x, S.y));
-                S.x *= av[t].x;
-                S.y *= av[t].y;
+                __half2 *pk = reinterpret_cast<__half2 *>(base + L::KE + p * 8192 + sw128(16 * u + t, d0));
+                *pk = __hmul2(*pk, __floats2half2_rn(S.x, S.y));
+                S.x *= av[p][t].x;
+                S.y *= av[p][t].y;
             }
         }
         const float2 qm = __half22float2(qmax);
-        if (warp == 0) *reinterpret_cast<float2 *>(vGc + d0) = gam;
+        if (warp == 0) {
+#pragma unroll
+            for (int p = 0; p < NKA; ++p) *reinterpret_cast<float2 *>(vGc + 64 * p + 2 * lane) = gam[p];
+        }
         fence_async_shared();
         tc_fence_before();
         // the whole-chunk form needs the gate range and |q~| <= 16 (qh then fits fp16)
         const bool exact = __syncthreads_or(!gam_ok || fmaxf(qm.x, qm.y) * qscale > 16.f) != 0;
 
-        // Two MMA passes through the same 64 TMEM columns.  Pass 1: A = qh ke^T
-        // (whole-chunk form only) in TMEM lanes 0-15 of each 32-lane group and
-        // dS^T = V^T ke in lanes 16-31 (an M = 64 accumulator uses half of each
-        // group).  Pass 2: O = P V + qh S' over A.  `phase` is the parity of the
-        // next mbarrier completion.
+        // Two MMA passes through the same TMEM columns.  Pass 1: A = qh ke^T
+        // (whole-chunk form only; columns 0-63) in TMEM lanes 0-15 of each
+        // 32-lane group and dS^T = V^T ke (columns 0..DK-1, one N = 64 MMA
+        // chain per key tile) in lanes 16-31 (an M = 64 accumulator uses half
+        // of each group).  Pass 2: O = P V + qh S' over A.  `phase` is the
+        // parity of the next mbarrier completion.
         uint32_t phase = 0;
         const uint32_t aQH = base_addr + L::QH, aKE = base_addr + L::KE, aV = base_addr + L::V;
         constexpr uint32_t kDsLanes = 16u << 16;
@@ -215,15 +257,19 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             if (!exact) {
                 const uint32_t id = umma_idesc_f16(0, 0);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024), umma_desc_sw128(aKE + 32 * ks, 16, 1024),
-                             id, ks > 0);
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t ko = (ks >> 2) * 8192 + 32 * (ks & 3);  // key tile, 16-dim step
+                    umma_f16(tmem, umma_desc_sw128(aQH + ko, 16, 1024), umma_desc_sw128(aKE + ko, 16, 1024), id,
+                             ks > 0);
+                }
             }
             const uint32_t id2 = umma_idesc_f16(1, 1);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                umma_f16(tmem + kDsLanes, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
-                         umma_desc_sw128(aKE + 2048 * ks, 8192, 1024), id2, ks > 0);
+            for (int na = 0; na < NKA; ++na)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    umma_f16(tmem + kDsLanes + 64 * na, umma_desc_sw128(aV + 2048 * ks, 8192, 1024),
+                             umma_desc_sw128(aKE + na * 8192 + 2048 * ks, 8192, 1024), id2, ks > 0);
             umma_commit(mbar);
         }
 
@@ -232,19 +278,23 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         if (exact) {
             if (gam_ok) {
                 // qh was written with 1 / gamma_c: rewrite qe = q~ E_t from the raw rows
-                float2 E = Ebase;
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int64_t r = sRow[16 * u + t];
-                    const bool ok = r >= 0 && GTR_INB(r * 64 + d0 + 1, rows * 64, BS_UMMA_EXACT);
-                    const float2 gv = ok ? *reinterpret_cast<const float2 *>(args.g + r * 64 + d0)
-                                         : make_float2(0.f, 0.f);
-                    const __half2 qv = ok ? *reinterpret_cast<const __half2 *>(args.q + r * 64 + d0)
-                                          : __float2half2_rn(0.f);
-                    E.x *= ex2(gv.x * kLog2e);
-                    E.y *= ex2(gv.y * kLog2e);
-                    *reinterpret_cast<__half2 *>(base + L::QH + sw128(16 * u + t, d0)) =
-                        __hmul2(qv, __floats2half2_rn(E.x * qscale, E.y * qscale));
+                for (int p = 0; p < NKA; ++p) {
+                    const int d0 = 64 * p + 2 * lane;
+                    float2 E = Ebase[p];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const int64_t r = sRow[16 * u + t];
+                        const bool ok = r >= 0 && GTR_INB(r * DK + d0 + 1, rows * DK, BS_UMMA_EXACT);
+                        const float2 gv = ok ? *reinterpret_cast<const float2 *>(args.g + r * DK + d0)
+                                             : make_float2(0.f, 0.f);
+                        const __half2 qv = ok ? *reinterpret_cast<const __half2 *>(args.q + r * DK + d0)
+                                              : __float2half2_rn(0.f);
+                        E.x *= ex2(gv.x * kLog2e);
+                        E.y *= ex2(gv.y * kLog2e);
+                        *reinterpret_cast<__half2 *>(base + L::QH + p * 8192 + sw128(16 * u + t, 2 * lane)) =
+                            __hmul2(qv, __floats2half2_rn(E.x * qscale, E.y * qscale));
+                    }
                 }
                 fence_async_shared();
             }
@@ -252,18 +302,18 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             const int t = tid >> 1, sb = 32 * (tid & 1);
 #pragma unroll
             for (int j = 0; j < 32; ++j) pe[j] = 0.f;
-            // log2-domain in-chunk prefix of g, four quarters of 16 dims,
+            // log2-domain in-chunk prefix of g, DK/16 parts of 16 dims,
             // staged in the (not yet used) score region
             __half *xq = reinterpret_cast<__half *>(base + L::P);          // [64][16]
             __half *xk = reinterpret_cast<__half *>(base + L::P + 2048);   // [64][16]
             float *xb = reinterpret_cast<float *>(base + L::P + 4096);     // [64][16]
-            for (int hd = 0; hd < 4; ++hd) {
+            for (int hd = 0; hd < DK / 16; ++hd) {
                 __syncthreads();
                 for (int idx = tid; idx < 64 * 16; idx += 128) {
                     const int tt = idx >> 4, d = idx & 15;
                     const int64_t r = sRow[tt];
-                    const int64_t o = (r < 0 ? 0 : r) * 64 + 16 * hd + d;
-                    const bool ok = r >= 0 && GTR_INB(o, rows * 64, BS_UMMA_EXACT);
+                    const int64_t o = (r < 0 ? 0 : r) * DK + 16 * hd + d;
+                    const bool ok = r >= 0 && GTR_INB(o, rows * DK, BS_UMMA_EXACT);
                     xq[idx] = ok ? args.q[o] : __float2half(0.f);
                     xk[idx] = ok ? args.k[o] : __float2half(0.f);
                     xb[idx] = ok ? args.g[o] * kLog2e : 0.f;
@@ -297,12 +347,15 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 
         // ---- this warp's slice of the state entering the chunk (bounded
         // wait on the predecessor's flag for the same slice), while pass 1 runs
+        // ring slot (chain, chunk parity): the chain's DK x 64 slice of the
+        // state, warp-major float4 fragments
+        constexpr int64_t kSlot = (int64_t)DK * DVC;
+        const int64_t ring_n = (int64_t)nslot * 2 * kSlot;
         float Se[KT][4];
-        int *flag = args.ctrl + 2 + (int64_t)seq * 4 + warp;
+        int *flag = args.ctrl + 2 + (int64_t)slot * 4 + warp;
         if (c > 0) {
-            const float4 *ring_in =
-                reinterpret_cast<const float4 *>(args.ring + ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV));
-            if (lane == 0 && GTR_INB(2 + (int64_t)seq * 4 + warp, 2 + (int64_t)nseq * 4, BS_UMMA_FLAG)) {
+            const float4 *ring_in = reinterpret_cast<const float4 *>(args.ring + ((int64_t)slot * 2 + ((c - 1) & 1)) * kSlot);
+            if (lane == 0 && GTR_INB(2 + (int64_t)slot * 4 + warp, 2 + (int64_t)nslot * 4, BS_UMMA_FLAG)) {
                 long long spins = 0;
                 while (ld_acquire(flag) < c) {
                     if (++spins > args.spin_limit) {
@@ -315,8 +368,8 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
             __syncwarp();
 #pragma unroll
             for (int n = 0; n < KT; ++n) {
-                const int64_t e = ((int64_t)seq * 2 + ((c - 1) & 1)) * (DK * DV) + ((warp * KT + n) * 32 + lane) * 4;
-                const float4 x = GTR_INB(e + 3, (int64_t)nseq * 2 * DK * DV, BS_UMMA_RING)
+                const int64_t e = ((int64_t)slot * 2 + ((c - 1) & 1)) * kSlot + ((warp * KT + n) * 32 + lane) * 4;
+                const float4 x = GTR_INB(e + 3, ring_n, BS_UMMA_RING)
                                      ? __ldcg(ring_in + ((warp * KT + n) * 32 + lane))
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
                 Se[n][0] = x.x; Se[n][1] = x.y; Se[n][2] = x.z; Se[n][3] = x.w;
@@ -335,9 +388,9 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
         {
             const bool hold = (seq == args.hold_seq && c == args.hold_chunk);
             const bool publish = c + 1 < geo.nc && !hold;
-            float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)seq * 2 + (c & 1)) * (DK * DV));
+            float4 *dst = reinterpret_cast<float4 *>(args.ring + ((int64_t)slot * 2 + (c & 1)) * kSlot);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            for (int hf = 0; hf < DK / 32; ++hf) {
                 float dS[16];
                 tmem_ld_16x32(tmem + kDsLanes + ((uint32_t)(32 * warp) << 16) + 32 * hf, dS);
                 tc_wait_ld();
@@ -351,15 +404,15 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                         x.y = fmaf(gg.y, Se[n][1], dS[4 * m + 1]);
                         x.z = fmaf(gg.x, Se[n][2], dS[4 * m + 2]);
                         x.w = fmaf(gg.y, Se[n][3], dS[4 * m + 3]);
-                        const int64_t e = ((int64_t)seq * 2 + (c & 1)) * (DK * DV) + ((warp * KT + n) * 32 + lane) * 4;
-                        if (GTR_INB(e + 3, (int64_t)nseq * 2 * DK * DV, BS_UMMA_RING))
+                        const int64_t e = ((int64_t)slot * 2 + (c & 1)) * kSlot + ((warp * KT + n) * 32 + lane) * 4;
+                        if (GTR_INB(e + 3, ring_n, BS_UMMA_RING))
                             __stcg(dst + ((warp * KT + n) * 32 + lane), x);
                     }
                 }
             }
             if (publish) {
                 __syncwarp();
-                if (lane == 0 && GTR_INB(2 + (int64_t)seq * 4 + warp, 2 + (int64_t)nseq * 4, BS_UMMA_FLAG))
+                if (lane == 0 && GTR_INB(2 + (int64_t)slot * 4 + warp, 2 + (int64_t)nslot * 4, BS_UMMA_FLAG))
                     st_release(flag, c + 1);
             }
         }
@@ -385,9 +438,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
         for (int n = 0; n < KT; ++n) {
             const float2 sc = exact ? make_float2(1.f, 1.f) : *reinterpret_cast<const float2 *>(vGc + 8 * n + kc);
-            const int dv0 = 16 * warp + tr, dk = 8 * n + kc;
-            *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
-            *reinterpret_cast<uint32_t *>(base + L::SP + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
+            const int dv0 = 16 * warp + tr, dk = 8 * (n & 7) + kc;  // key tile n / 8
+            unsigned char *sp = base + L::SP + (n >> 3) * 8192;
+            *reinterpret_cast<uint32_t *>(sp + sw128(dv0, dk)) = pack_h2(sc.x * Se[n][0], sc.y * Se[n][1]);
+            *reinterpret_cast<uint32_t *>(sp + sw128(dv0 + 8, dk)) = pack_h2(sc.x * Se[n][2], sc.y * Se[n][3]);
         }
         fence_async_shared();
         tc_fence_before();
@@ -404,9 +458,10 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
                          id_pv, ks > 0);
             if (c > 0) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    umma_f16(tmem, umma_desc_sw128(aQH + 32 * ks, 16, 1024),
-                             umma_desc_sw128(aSP + 32 * ks, 16, 1024), id_qs, 1);
+                for (int ks = 0; ks < DK / 16; ++ks) {
+                    const uint32_t ko = (ks >> 2) * 8192 + 32 * (ks & 3);
+                    umma_f16(tmem, umma_desc_sw128(aQH + ko, 16, 1024), umma_desc_sw128(aSP + ko, 16, 1024), id_qs, 1);
+                }
             }
             umma_commit(mbar);
         }
@@ -431,8 +486,8 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int t = 16 * warp + 4 * i + (lane >> 3), j = lane & 7;
-                if (t < len && sRow[t] >= 0 && GTR_INB(sRow[t] * DV + j * 8 + 7, rows * DV, BS_UMMA_OUT))
-                    *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + j * 8) =
+                if (t < len && sRow[t] >= 0 && GTR_INB(sRow[t] * DV + vh * DVC + j * 8 + 7, rows * DV, BS_UMMA_OUT))
+                    *reinterpret_cast<int4 *>(args.out + sRow[t] * DV + vh * DVC + j * 8) =
                         *reinterpret_cast<const int4 *>(st + t * 128 + (((j ^ (t & 7)) & 7) << 4));
             }
         }
@@ -443,19 +498,21 @@ __global__ void __launch_bounds__(128, 6) gla_umma_kernel(const TcArgs args) {
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 64;\n" ::"r"(tmem) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(L::TMEM_COLS) : "memory");
     }
 }
 
-inline cudaError_t launch_umma(const TcArgs &a, cudaStream_t st) {
-    const size_t smem = UmmaLayout::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(gla_umma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <int DK>
+cudaError_t launch_umma(const TcArgs &a, cudaStream_t st) {
+    const size_t smem = UmmaLayout<DK>::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(gla_umma_kernel<DK>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    // six CTAs of ~36 KB per SM: ask for the largest shared-memory carveout
-    e = cudaFuncSetAttribute(gla_umma_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    // six CTAs of ~36 KB (d_k = 64) or four of ~53 KB (d_k = 128) per SM:
+    // ask for the largest shared-memory carveout
+    e = cudaFuncSetAttribute(gla_umma_kernel<DK>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
-    const unsigned grid = (unsigned)((int64_t)a.geo.nc * a.geo.B * a.geo.heads);
-    gla_umma_kernel<<<grid, 128, smem, st>>>(a);
+    const unsigned grid = (unsigned)((int64_t)a.geo.nc * a.geo.B * a.geo.heads * (DK / 64));
+    gla_umma_kernel<DK><<<grid, 128, smem, st>>>(a);
     count_launch();
     return cudaGetLastError();
 }

@@ -161,10 +161,13 @@ size_t three_phase_ws(const Geom &g) {
            align256(nseq * g.nc * g.dk * sizeof(float)) + align256(scan_agg_bytes((int64_t)nseq, g.nc, g.dk, g.dv));
 }
 
-// Fused kernels: control words (ticket, unused, four flags per sequence: the
-// mma.sync kernel uses one per sequence, the tcgen05 kernel one per warp)
-// then a two-slot ring of boundary states per sequence.
-size_t fused_ctrl_bytes(const Geom &g) { return align256(((size_t)g.B * g.heads * 4 + 2) * sizeof(int)); }
+// Fused kernels: control words (ticket, unused, four flags per sequence and
+// 64 value columns: the mma.sync kernel uses one per sequence, the tcgen05
+// kernel one per (value half, warp)) then a two-slot ring of boundary states
+// per sequence.
+size_t fused_ctrl_bytes(const Geom &g) {
+    return align256(((size_t)g.B * g.heads * 4 * ((g.dv + 63) / 64) + 2) * sizeof(int));
+}
 size_t fused_ws(const Geom &g) {
     return fused_ctrl_bytes(g) + (size_t)g.B * g.heads * 2 * g.dk * g.dv * sizeof(float);
 }
@@ -214,7 +217,8 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
     return a;
 }
 
-bool tcgen05_shape(const Geom &g) { return g.dk == 64 && g.dv == 64 && g.chunk == 64; }
+// Shapes of the chained tcgen05 kernel.
+bool tcgen05_shape(const Geom &g) { return g.dk == g.dv && (g.dk == 64 || g.dk == 128) && g.chunk == 64; }
 // Shapes of the tcgen05 walk kernel (and of the tcgen05 three-phase phases).
 bool walk_shape(const Geom &g) {
     return g.chunk == 64 && (g.dk == 32 || g.dk == 64 || g.dk == 128) && (g.dv == 64 || g.dv == 128) &&
@@ -250,9 +254,11 @@ gtr_plan_t plan_for(const Geom &geo, int schedule, int sms, bool chain_only = fa
     // Few sequences leave the chain of boundary states as the critical path:
     // then two chunks per tile halve its length (d_v <= 64).  Many sequences
     // keep every SM busy anyway: then one chunk per tile gives more resident
-    // CTAs.  The chained tcgen05 kernel does one chunk per tile.
+    // CTAs.  The chained tcgen05 kernel does one chunk per tile (AUTO takes
+    // it at d_k = 64).
     const bool pair = nseq < 2 * (int64_t)sms;
-    if (tcgen05_shape(geo) && (schedule == GTR_SCHED_FUSED_TCGEN05 || (schedule == GTR_SCHED_AUTO && !pair)))
+    if (tcgen05_shape(geo) &&
+        (schedule == GTR_SCHED_FUSED_TCGEN05 || (schedule == GTR_SCHED_AUTO && !pair && geo.dk == 64)))
         return GTR_PLAN_FUSED_TCGEN05;
     return (pair && geo.dv <= 64) ? GTR_PLAN_FUSED_MMA_PAIR : GTR_PLAN_FUSED_MMA;
 }

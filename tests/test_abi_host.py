@@ -143,6 +143,9 @@ def test_dispatch_plan(lib):
     # explicit schedules
     assert plan(8, 8, 64, 64, 64, 64, 64, "fused_tcgen05") == 4
     assert plan(8, 8, 64, 64, 32, 64, 64, "fused_tcgen05") == 3  # not its shape
+    assert plan(8, 8, 64, 64, 128, 128, 64, "fused_tcgen05") == 4  # d_k = d_v = 128: value-half tiles
+    assert plan(8, 8, 64, 64, 128, 64, 64, "fused_tcgen05") == 3  # d_k != d_v: not its shape
+    assert plan(64, 8, 64, 64, 128, 128, 64, "auto") == 2  # AUTO keeps d=128 on mma.sync
     assert plan(32, 12, 40, 40, 64, 64, 64, "fused") == 2
     assert plan(8, 8, 256, 256, 128, 128, 64, "walk_tcgen05") == 5
     assert plan(8, 8, 64, 64, 32, 64, 64, "walk_tcgen05") == 5

@@ -96,6 +96,21 @@ def test_checked_build_tf32_diagonal_d128(clib, oracle_mod, gates):
         compare(out.cpu(), oracle_mod.gla_serial(q, k, v, g, H, W, direction))
 
 
+@pytest.mark.parametrize("gates", ["mild", "strong"])
+def test_checked_build_chained_tcgen05_d128(clib, oracle_mod, gates):
+    """d_k = d_v = 128 on the chained tcgen05 kernel: two value-half CTAs
+    per chunk, each chaining its 128 x 64 state slice through the ring over
+    three chunks (the last one short); strong gates take the exact score
+    path, which reads the raw rows again."""
+    H, W, heads = 13, 11, 3
+    q, k, v, g = make_inputs(2, H, W, heads, 128, 128, seed=59, gate=gates)
+    dq, dk_, dvv, dg = (x.cuda() for x in (q, k, v, g))
+    for direction in range(4):
+        out = run_checked(clib, dq, dk_, dvv, dg, H, W, direction, 64, "fused_tcgen05")
+        assert_no_skips(clib)
+        compare(out.cpu(), oracle_mod.gla_serial(q, k, v, g, H, W, direction))
+
+
 def test_checked_build_other_entry_points(clib, oracle_mod):
     """The host-buffer entry point and the no-allocation entry point."""
     B, H, W, heads = 2, 7, 9, 3
