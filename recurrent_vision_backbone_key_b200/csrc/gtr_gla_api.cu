@@ -217,8 +217,12 @@ TcArgs make_args(const __half *q, const __half *k, const __half *v, const float 
     return a;
 }
 
-// Shapes of the chained tcgen05 kernel.
-bool tcgen05_shape(const Geom &g) { return g.dk == g.dv && (g.dk == 64 || g.dk == 128) && g.chunk == 64; }
+// Shapes of the chained tcgen05 kernel (its tile index, chunk-major over
+// (sequence, 64 value columns), is a 32-bit int).
+bool tcgen05_shape(const Geom &g) {
+    return g.dk == g.dv && (g.dk == 64 || g.dk == 128) && g.chunk == 64 &&
+           (int64_t)g.B * g.heads * g.nc * (g.dv / 64) < ((int64_t)1 << 31);
+}
 // Shapes of the tcgen05 walk kernel (and of the tcgen05 three-phase phases).
 bool walk_shape(const Geom &g) {
     return g.chunk == 64 && (g.dk == 32 || g.dk == 64 || g.dk == 128) && (g.dv == 64 || g.dv == 128) &&

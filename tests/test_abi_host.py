@@ -146,6 +146,11 @@ def test_dispatch_plan(lib):
     assert plan(8, 8, 64, 64, 128, 128, 64, "fused_tcgen05") == 4  # d_k = d_v = 128: value-half tiles
     assert plan(8, 8, 64, 64, 128, 64, 64, "fused_tcgen05") == 3  # d_k != d_v: not its shape
     assert plan(64, 8, 64, 64, 128, 128, 64, "auto") == 2  # AUTO keeps d=128 on mma.sync
+    # d = 128 doubles the chained kernel's tiles (two value halves per chunk):
+    # 2^30 chunk tiles give 2^31, past its 32-bit tile index
+    assert plan(16384, 64, 256, 256, 128, 128, 64, "fused_tcgen05") == 2
+    assert plan(8192, 64, 256, 256, 128, 128, 64, "fused_tcgen05") == 4
+    assert plan(16384, 64, 256, 256, 64, 64, 64, "fused_tcgen05") == 4
     assert plan(32, 12, 40, 40, 64, 64, 64, "fused") == 2
     assert plan(8, 8, 256, 256, 128, 128, 64, "walk_tcgen05") == 5
     assert plan(8, 8, 64, 64, 32, 64, 64, "walk_tcgen05") == 5
