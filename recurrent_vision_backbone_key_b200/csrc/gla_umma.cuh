@@ -63,6 +63,12 @@ struct UmmaLayout {
     static constexpr uint32_t ALLOC = BYTES + 1024;    // slack for aligning the base
     static constexpr uint32_t TMEM_COLS = DK;          // dS^T is the widest accumulator
     static constexpr int CTAS_PER_SM = DK == 64 ? 6 : 4;
+    // swizzled operand tiles on 1024-byte boundaries; the resident CTAs fit
+    // the SM's 228 KB of shared memory (1 KB reserved per CTA) and its 512
+    // TMEM columns
+    static_assert(QH % 1024 == 0 && KE % 1024 == 0 && V % 1024 == 0 && P % 1024 == 0, "tile alignment");
+    static_assert(CTAS_PER_SM * (ALLOC + 1024) <= 228 * 1024, "shared memory per SM");
+    static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "tensor memory per SM");
 };
 
 // ---------------------------------------------------------------- the kernel
