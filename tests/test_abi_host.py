@@ -118,6 +118,14 @@ def test_workspace_bytes(lib):
     assert n7 >= n and n7 >= lib.gtr_gla_workspace_bytes_ex(2, 3, 10, 10, 32, 64, 16, "fused")
     assert lib.gtr_gla_workspace_bytes(0, 3, 10, 10, 32, 64, 16) == 0
     assert lib.gtr_gla_workspace_bytes(1, 1, 4, 4, 24, 16, 16) == 0
+    # the chained kernels' workspace: control words (ticket, unused, four
+    # flags per (sequence, 64 value columns)) padded to 256 bytes, a two-slot
+    # fp32 ring of d_k x d_v states per sequence, the stream's status word
+    a256 = lambda x: (x + 255) // 256 * 256
+    for (B, heads, d) in ((2, 3, 64), (2, 3, 128), (5, 7, 128)):
+        nseq = B * heads
+        want = a256((nseq * 4 * (d // 64) + 2) * 4) + nseq * 2 * d * d * 4 + 256
+        assert lib.gtr_gla_workspace_bytes_ex(B, heads, 10, 10, d, d, 64, "fused_tcgen05") == want
 
 
 def test_dispatch_plan(lib):
